@@ -1,0 +1,404 @@
+#!/usr/bin/env python
+"""Benchmark of the fused MoE layer forward (moe_fused_forward) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--config qwen36|nemotron|large_e|tiny] [--T 4096] [--routing router|zipf]
+                    [--no-sweep]
+
+A step is one complete layer forward (router logits, top-k, permutation, FC1 + activation,
+FC2 + weighted combine, shared expert, finalize) over T tokens of synthetic input drawn
+by the seeded generator.  Rank 0 prints one JSON line.  With N > 1 (torchrun, one
+process per GPU) every rank runs an independent replica on its own batch (the layer
+has no cross-token exchange), the timed region is bracketed by barriers and
+synchronisation, and the time is the maximum over ranks.
+
+``--impl reference`` times the CPU oracle (single-threaded FP64 C) on a bounded token
+sample of the same workload, on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from mixture_experts_layer_35_b200 import inputs as gen  # noqa: E402
+
+L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2: written between timed steps
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------- plumbing
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, local, world
+
+
+def dist_init(world: int, backend: str):
+    if world > 1 and not torch.distributed.is_initialized():
+        torch.distributed.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=300))
+
+
+def barrier(world: int, device=None):
+    if world > 1:
+        if device is not None and device.type == "cuda":
+            torch.distributed.barrier(device_ids=[device.index])
+        else:
+            torch.distributed.barrier()
+
+
+def max_over_ranks(value: float, world: int, device) -> float:
+    if world == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(gpu_index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r.split(",") for r in out.strip().splitlines() if r.count(",") >= 7]
+        if not rows:
+            return None
+        sm = [float(r[0]) for r in rows if r[0].strip().replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({n for r in rows for n, v in zip(names, r[4:8]) if v.strip() == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- algorithmic accounting
+def accounting(shape, T: int, U: int, router: bool, Is: int):
+    """Algorithmic bytes / flops of the layer and of each kernel.  U = distinct routed
+    experts touched by the call.  Weights of untouched experts are not counted; h, acc,
+    permutation indices are implementation traffic, except where a kernel's own
+    operand is h (FC2 reads it, FC1 writes it)."""
+    H, I, E, K = shape.H, shape.I, shape.E, shape.K
+    rows1 = 2 * I if shape.act == "swiglu" else I
+    rows1s = 2 * Is if shape.act == "swiglu" else Is
+    h_bytes = (T * K * I + T * Is) * 2
+    k = {}
+    k["router"] = {"bytes": E * H * 2 + T * H * 2 + T * E * 4, "flops": 2 * T * E * H}
+    k["topk"] = {"bytes": T * E * 4 + T * K * 8, "flops": 0}
+    k["permute"] = {"bytes": T * K * 4 * 2, "flops": 0}
+    k["fc1"] = {"bytes": U * rows1 * H * 2 + rows1s * H * 2 + T * H * 2 + h_bytes,
+                "flops": 2 * T * K * rows1 * H + 2 * T * rows1s * H}
+    k["fc2"] = {"bytes": U * H * I * 2 + H * Is * 2 + h_bytes + T * H * 2,
+                "flops": 2 * T * K * H * I + 2 * T * H * Is}
+    k["finalize"] = {"bytes": T * H * (4 + 2 + (2 if Is else 0)), "flops": 0}
+    layer_bytes = U * (rows1 + I) * H * 2 + (E * H * 2 if router else 0) + 2 * T * H * 2 + \
+        (rows1s + Is) * H * 2 + 4 * E
+    layer_flops = 2 * T * K * (rows1 + I) * H + (2 * T * E * H if router else 0) + 2 * T * (rows1s + Is) * H
+    return {"layer": {"bytes": layer_bytes, "flops": layer_flops}, "kernels": k}
+
+
+def kernel_names(path: str, router: bool):
+    names = ["router"] if router else []
+    return names + (["fc1", "fc2"] if path == "small" else ["topk", "permute", "fc1", "fc2", "finalize"])
+
+
+def roofline_of(acc: dict, dur_s: float, peaks: dict):
+    t_hbm = acc["bytes"] / (peaks["hbm_gbs"] * 1e9)
+    t_tc = acc["flops"] / (peaks["bf16_tflops"] * 1e12)
+    if t_tc > t_hbm:
+        ach = acc["flops"] / dur_s / 1e12
+        return {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": ach / peaks["bf16_tflops"]}
+    ach = acc["bytes"] / dur_s / 1e9
+    return {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": ach / peaks["hbm_gbs"]}
+
+
+# ---------------------------------------------------------------- our arm
+class Bench:
+    def __init__(self, shape, T, device, seed, routing, path="auto"):
+        import mixture_experts_layer_35_b200.moe as moe
+        self.moe = moe
+        self.shape, self.T, self.device = shape, T, device
+        self.d = gen.make_layer(shape, T, seed=seed, device=str(device), routing=routing)
+        self.logits = self.d["router_logits"]
+        w = {k: self.d[k] for k in ("router_w", "bias", "w13", "w2", "ws13", "ws2") if self.d.get(k) is not None}
+        self.layer = moe.MoELayer(shape, w, path=path)
+        self.desc = self.layer.desc(T, self.logits)
+        self.ws = self.layer.workspace(self.desc, device)
+        self.out = torch.empty((T, shape.H), dtype=torch.bfloat16, device=device)
+        self.path = moe.select_path(self.desc)
+        self.launches = moe.launches(self.desc)
+        self.Is = shape.I_shared if w.get("ws13") is not None else 0
+        self.flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+
+    def flush(self):
+        self.flush_buf.fill_(1)
+
+    def step(self, x=None, out=None, stream=None):
+        self.moe.fused_forward_raw(self.desc, self.d["x"] if x is None else x, self.out if out is None else out,
+                                   self.ws, stream=stream)
+
+    def distinct_experts(self):
+        _, _, ids, _ = self.layer.forward(self.d["x"], router_logits=self.logits, return_routing=True)
+        torch.cuda.synchronize(self.device)
+        return int(torch.unique(ids).numel())
+
+    def timed(self, steps: int, warmup: int, world: int = 1, clocks=None):
+        for _ in range(warmup):
+            self.flush()
+            self.step()
+        torch.cuda.synchronize(self.device)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        barrier(world, self.device)
+        torch.cuda.synchronize(self.device)
+        sampler = ClockSampler(self.device.index) if clocks else None
+        for a, b in evs:
+            self.flush()
+            a.record()
+            self.step()
+            b.record()
+        torch.cuda.synchronize(self.device)
+        clk = sampler.stop() if sampler else None
+        barrier(world, self.device)
+        per = [a.elapsed_time(b) for a, b in evs]
+        return per, clk
+
+    def per_kernel(self, steps: int):
+        n = self.launches
+        tot = np.zeros(n)
+        for _ in range(steps):
+            self.flush()
+            evs = [torch.cuda.Event(enable_timing=True) for _ in range(n + 1)]
+            self.moe.fused_forward_timed(self.desc, self.d["x"], self.out, self.ws, evs)
+            torch.cuda.synchronize(self.device)
+            tot += np.array([evs[i].elapsed_time(evs[i + 1]) for i in range(n)])
+        return tot / steps
+
+    def e2e(self, steps: int, warmup: int):
+        T, H = self.T, self.shape.H
+        x_host = self.d["x"].to("cpu").pin_memory()
+        out_host = torch.empty((T, H), dtype=torch.bfloat16).pin_memory()
+        x_dev = torch.empty_like(self.d["x"])
+        for _ in range(warmup):
+            x_dev.copy_(x_host, non_blocking=True)
+            self.step(x=x_dev)
+            out_host.copy_(self.out, non_blocking=True)
+        torch.cuda.synchronize(self.device)
+        ms = []
+        for _ in range(steps):
+            self.flush()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            x_dev.copy_(x_host, non_blocking=True)
+            self.step(x=x_dev)
+            out_host.copy_(self.out, non_blocking=True)
+            b.record()
+            torch.cuda.synchronize(self.device)
+            ms.append(a.elapsed_time(b))
+        return ms, T * H * 2, T * H * 2
+
+
+def cpu_oracle_rate(shape, d, budget_s: float, max_tokens: int):
+    """Tokens/s of the single-threaded CPU oracle on a bounded sample of the workload."""
+    import oracle
+    h = gen.to_numpy_inputs(d)
+    T = h["x"].shape[0]
+    rows = np.random.default_rng(0).permutation(T)[:max_tokens].astype(np.int32)
+    done, t0 = 0, time.perf_counter()
+    while done < len(rows) and time.perf_counter() - t0 < budget_s:
+        oracle.forward(shape, h, rows[done:done + 1])
+        done += 1
+    dt = time.perf_counter() - t0
+    return done / dt, done, dt
+
+
+def run_ours(args, rank, local, world):
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    dist_init(world, "nccl")
+    shape = gen.SHORT[args.config]
+    peaks, peaks_src = load_peaks()
+    b = Bench(shape, args.T, device, seed=args.seed + rank, routing=args.routing)
+    per, clk = b.timed(args.steps, args.warmup, world, clocks=True)
+    local_ms = float(sum(per))
+    total_ms = max_over_ranks(local_ms, world, device)
+    ms_step = total_ms / args.steps
+    value = world * args.T * args.steps / (total_ms / 1e3)
+
+    U = b.distinct_experts()
+    router = b.logits is None
+    acc = accounting(shape, args.T, U, router, b.Is)
+    kt = b.per_kernel(max(3, min(args.steps, 10)))
+    names = kernel_names(b.path, router)
+    dom = int(np.argmax(kt))
+    dom_name = names[dom]
+    roof = roofline_of(acc["kernels"][dom_name], kt[dom] / 1e3, peaks)
+    roof["kernel"] = f"{dom_name} ({b.path} path)"
+    roof["traffic"] = None
+    roof["peak_source"] = f"of {peaks_src}"
+    layer_roof = roofline_of(acc["layer"], ms_step / 1e3, peaks)
+    e2e_ms, bi, bo = b.e2e(args.steps, args.warmup)
+    e2e_total = max_over_ranks(float(sum(e2e_ms)), world, device)
+    e2e_value = world * args.T * args.steps / (e2e_total / 1e3)
+
+    line = {
+        "metric": "fused MoE layer tokens/s (one full layer forward per step)",
+        "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded generator, random-init weights of the layer's shape)",
+        "config": {"workload": f"{shape.name} T={args.T} routing={args.routing}", "tokens_per_step": args.T,
+                   "path": b.path, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write), steps timed with CUDA events",
+                   "distinct_experts": U},
+        "roofline": roof,
+        "layer_roofline": layer_roof,
+        "kernel_ms": {n: round(float(v), 5) for n, v in zip(names, kt)},
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo},
+        "gpu_launches": b.launches * args.steps,
+        "clocks": clk,
+        "us_per_step_p10_p50_p90": [float(np.percentile(per, q)) * 1e3 for q in (10, 50, 90)],
+    }
+    del b
+    torch.cuda.empty_cache()
+    if rank == 0 and world == 1 and not args.no_sweep:
+        line["sweep"] = sweep(args, device, peaks)
+    if rank == 0 and world == 1:
+        dcpu = gen.make_layer(shape, args.T, seed=args.seed, device=str(device), routing=args.routing)
+        rate, n, dt = cpu_oracle_rate(shape, dcpu, args.cpu_budget, 400)
+        line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                                "sample": f"{n} tokens of the same workload in {dt:.1f} s (single-threaded FP64 C)"}
+        del dcpu
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    barrier(world, device)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+def sweep(args, device, peaks):
+    """Per-T latency curve of the layer (median of short timed runs, L2 flushed)."""
+    rows = []
+    plan = [("qwen36", t) for t in gen.T_SWEEP]
+    if args.sweep_all:
+        plan += [("nemotron", t) for t in gen.T_SWEEP] + [("large_e", t) for t in gen.LARGE_E_T]
+    cache = {}
+    for cfg, T in plan:
+        shape = gen.SHORT[cfg]
+        try:
+            b = Bench(shape, T, device, seed=1, routing="router")
+            per, _ = b.timed(8, 2)
+            med = statistics.median(per)
+            U = b.distinct_experts()
+            acc = accounting(shape, T, U, True, b.Is)["layer"]
+            rf = roofline_of(acc, med / 1e3, peaks)
+            rows.append({"config": cfg, "T": T, "path": b.path, "us": med * 1e3, "tokens_per_s": T / (med / 1e3),
+                         "distinct_experts": U, "bound": rf["bound"], "frac_of_roofline": rf["frac"],
+                         "achieved": rf["achieved"], "unit": rf["unit"]})
+            del b
+        except Exception as e:  # report, keep sweeping
+            rows.append({"config": cfg, "T": T, "error": str(e)[:200]})
+        cache.clear()
+        torch.cuda.empty_cache()
+    return rows
+
+
+# ---------------------------------------------------------------- reference arm (CPU oracle)
+def run_reference(args, rank, local, world):
+    if rank != 0:
+        return
+    shape = gen.SHORT[args.config]
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    d = gen.make_layer(shape, args.T, seed=args.seed, device=dev, routing=args.routing)
+    import oracle
+    h = gen.to_numpy_inputs(d)
+    del d
+    sample = max(1, args.ref_tokens)
+    rng = np.random.default_rng(0)
+    times = []
+    for i in range(args.warmup + args.steps):
+        rows = rng.choice(args.T, sample, replace=False).astype(np.int32)
+        t0 = time.perf_counter()
+        oracle.forward(shape, h, rows)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            times.append(dt)
+    tot = sum(times)
+    value = sample * args.steps / tot
+    line = {"impl": "reference", "metric": "fused MoE layer tokens/s (one full layer forward per step)",
+            "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": tot / args.steps * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic (seeded generator)",
+            "config": {"workload": f"{shape.name} T={args.T} routing={args.routing}",
+                       "sample": f"{sample} tokens per step"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                             "sample": f"{sample} random tokens of the workload per step, single-threaded FP64 C"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--config", choices=sorted(gen.SHORT), default="qwen36")
+    p.add_argument("--T", type=int, default=4096)
+    p.add_argument("--routing", choices=["router", "zipf"], default="router")
+    p.add_argument("--seed", type=int, default=0)
+    p.add_argument("--no-sweep", action="store_true")
+    p.add_argument("--sweep-all", action="store_true")
+    p.add_argument("--cpu-budget", type=float, default=15.0)
+    p.add_argument("--ref-tokens", type=int, default=4)
+    args = p.parse_args(argv)
+    args.warmup = max(args.warmup, 3)
+    rank, local, world = dist_env()
+    if args.impl == "reference":
+        run_reference(args, rank, local, world)
+    else:
+        run_ours(args, rank, local, world)
+
+
+if __name__ == "__main__":
+    main()

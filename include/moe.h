@@ -1,0 +1,185 @@
+/*
+ * moe.h -- C ABI of libmoe.so, a B200 (sm_100a) fused Mixture-of-Experts layer forward.
+ *
+ * The operation (per token t, hidden size H, E routed experts, top-k K):
+ *   1. router logits    l[t,e] = x[t,:] . Wr[e,:]            (BF16 in, FP32 accumulate)
+ *   2. router top-k     "Laguna exact M=8 BF16-input router top-k preregistration",
+ *                       section "Question and arithmetic contract": FP32 sigmoid (or
+ *                       softmax) scores, an FP32 correction bias used only for selection,
+ *                       lower-expert-ID tie break, top K, renormalised unbiased weights.
+ *   3. permutation      token slots grouped by expert (FlashInfer PR #4646, walkthrough:
+ *                       "routing permutation").
+ *   4. FC1 + activation h = SwiGLU(W13[e] x) = silu(gate) * up, or ReLU^2(W1[e] x)
+ *                       (FlashInfer PR #4646, description: SwiGLU gated / ReLU2 ungated).
+ *   5. FC2 + combine    routed[t] = sum_k w[t,k] * W2[e_k] h[t,k], FP32 accumulation.
+ *   6. shared expert    out = bf16( bf16(routed) + bf16(shared FFN(x)) ), the order of
+ *                       "MTP1 isolated gather/shared-add closure" (b70-optimization-lab):
+ *                       routed FP32 accumulation -> BF16 -> shared BF16 add -> BF16.
+ *
+ * Conventions for every entry point
+ *   - All tensor pointers are DEVICE pointers on the current CUDA device, row-major and
+ *     contiguous, 16-byte aligned.  BF16 tensors are raw bfloat16 bit patterns.
+ *   - The caller owns every buffer.  The library never allocates, frees or synchronises
+ *     (moe_get_error is the one call that synchronises its stream).
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default stream).
+ *   - Arguments are validated on the host before anything is enqueued; on error nothing
+ *     is launched and the status says why.  T == 0 (moe_fused_forward) and M == 0
+ *     (moe_router_topk) return MOE_OK and launch nothing.
+ *   - There is no hidden global state: concurrent calls are safe when they use distinct
+ *     outputs and workspaces.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size or enum value */
+    MOE_ERR_UNSUPPORTED = 2,  /* valid but outside what this build supports (limits below) */
+    MOE_ERR_WORKSPACE = 3,    /* workspace missing, misaligned (256 B) or too small */
+    MOE_ERR_CUDA = 4,         /* a CUDA runtime call failed (launch, attribute, driver entry) */
+    MOE_ERR_DEVICE = 5        /* the device error word is set (see moe_get_error) */
+} moe_status_t;
+
+typedef enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID = 1 } moe_score_t;
+typedef enum { MOE_ACT_SWIGLU = 0, MOE_ACT_RELU2 = 1 } moe_act_t;
+typedef enum { MOE_DT_BF16 = 0, MOE_DT_FP32 = 1 } moe_dtype_t;
+/* Execution path of moe_fused_forward.  AUTO picks by token count (see
+ * moe_select_path).  SMALL streams only the routed experts' weights with CUDA-core dot
+ * products spread over all SMs; LARGE runs the grouped tcgen05 tensor-core GEMMs. */
+typedef enum { MOE_PATH_AUTO = 0, MOE_PATH_SMALL = 1, MOE_PATH_LARGE = 2 } moe_path_t;
+
+/* Device error codes written to the workspace error word. */
+#define MOE_DEVERR_BAD_EXPERT_ID 0x1   /* an expert id outside [0, E) reached the permute */
+#define MOE_DEVERR_WAIT_TIMEOUT 0x2    /* a bounded device-side wait gave up */
+
+/* Limits of this build. */
+#define MOE_MAX_EXPERTS 1024
+#define MOE_MAX_TOPK 32
+#define MOE_MAX_TOKENS 65536
+
+/* ------------------------------------------------------------------------------------
+ * moe_router_topk -- router scores + top-k + weights for M rows of logits.
+ * Passage: "Laguna exact M=8 BF16-input router top-k preregistration", "Question and
+ * arithmetic contract" (BF16 logits -> exact widening -> FP32 sigmoid -> + FP32 bias for
+ * selection only -> lower-expert-ID tie break -> top k -> renormalise the unbiased FP32
+ * sigmoid weights) and "Four-card component gate" (source index slot * M + row).
+ *   logits     [M, E] BF16 (logits_dtype = MOE_DT_BF16) or FP32 (MOE_DT_FP32).
+ *   score      MOE_SCORE_SIGMOID: s = sigmoid(l) in FP32 (correctly rounded), key = s + b
+ *              (FP32 add).  MOE_SCORE_SOFTMAX: key = l (+ b if bias), weights from the
+ *              softmax of the logits.
+ *   bias       [E] FP32 or NULL (= zero).  Used for selection only.
+ *   renorm     1: weights renormalised over the K selected experts (sigmoid: s_k / sum s;
+ *              softmax: exp(l_k - lmax) / sum over the selected); 0: sigmoid -> s_k,
+ *              softmax -> full softmax probability over all E.
+ *   topk_w     [M, K] FP32 out, slot k = k-th largest key (ties -> lower expert id).
+ *   topk_ids   [M, K] int32 out.
+ *   src_idx    [M, K] int32 out, src_idx[m,k] = k * M + m.  May be NULL.
+ * Limits: 1 <= E <= MOE_MAX_EXPERTS, 1 <= K <= min(E, MOE_MAX_TOPK), 0 <= M.
+ * NaN logits are selected last (treated as -inf); their weights are undefined.
+ * ---------------------------------------------------------------------------------- */
+moe_status_t moe_router_topk(const void* logits, int logits_dtype, int M, int E, int top_k,
+                             int score, const float* bias, int renorm, float* topk_w,
+                             int32_t* topk_ids, int32_t* src_idx, void* stream);
+
+/* ------------------------------------------------------------------------------------
+ * moe_permute -- group the M*K token slots by expert.
+ * Passage: FlashInfer PR #4646, walkthrough (routing permutation) and review notes on
+ * the permute scan (padded-count reduction, exclusive scan, per-expert offsets).  This
+ * build is unpadded and deterministic.
+ *   topk_ids        [M, K] int32 in; ids must lie in [0, E).
+ *   expert_offsets  [E + 1] int32 out: exclusive prefix sum of the per-expert counts,
+ *                   expert_offsets[E] = M * K.
+ *   perm            [M * K] int32 out: source indices src = k * M + m, grouped by expert
+ *                   in ascending expert order and by ascending token m within an expert.
+ *   inv             [M * K] int32 out: inv[src] = position of src in perm.  May be NULL.
+ *   ws, ws_bytes    device workspace of at least moe_permute_workspace_size(M, K, E) bytes,
+ *                   256-byte aligned.  Holds the device error word.
+ * M == 0 still writes expert_offsets (all zero).
+ * An id outside [0, E) sets MOE_DEVERR_BAD_EXPERT_ID in the error word (read it with
+ * moe_get_error); that slot is left out of perm and the outputs are then incomplete.
+ * Limits: M * K <= MOE_MAX_TOKENS * 8, E <= MOE_MAX_EXPERTS, K <= MOE_MAX_TOPK.
+ * ---------------------------------------------------------------------------------- */
+size_t moe_permute_workspace_size(int M, int K, int E);
+moe_status_t moe_permute(const int32_t* topk_ids, int M, int K, int E, int32_t* expert_offsets,
+                         int32_t* perm, int32_t* inv, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------------------
+ * moe_fused_forward -- the whole layer (steps 1-6 above) for T tokens.
+ * Layer description: */
+typedef struct {
+    int T;            /* tokens, 0 <= T <= MOE_MAX_TOKENS */
+    int H;            /* hidden size, multiple of 8 */
+    int I;            /* routed-expert intermediate size, multiple of 8 */
+    int E;            /* routed experts, 1..MOE_MAX_EXPERTS */
+    int top_k;        /* 1..min(E, MOE_MAX_TOPK) */
+    int act;          /* moe_act_t */
+    int score;        /* moe_score_t */
+    int renorm;       /* 0 or 1, as in moe_router_topk */
+    int I_shared;     /* shared-expert intermediate size (multiple of 8), 0 = none */
+    int path;         /* moe_path_t */
+    const void* router_w;        /* [E, H] BF16; may be NULL when router_logits is given */
+    const float* router_logits;  /* [T, E] FP32 logits to route on instead of x . Wr^T, or NULL */
+    const float* bias;           /* [E] FP32 selection bias or NULL */
+    const void* w13;             /* SwiGLU: [E, 2I, H] BF16, rows [0,I) gate, [I,2I) up;
+                                    ReLU^2: [E, I, H] BF16 */
+    const void* w2;              /* [E, H, I] BF16 */
+    const void* ws13;            /* shared expert, [2I_s, H] or [I_s, H] BF16, or NULL */
+    const void* ws2;             /* shared expert, [H, I_s] BF16, or NULL */
+} moe_layer_desc;
+
+/* Bytes of workspace moe_fused_forward needs for this description (either path). */
+size_t moe_workspace_size(const moe_layer_desc* d);
+
+/* Path MOE_PATH_AUTO resolves to for this description (MOE_PATH_SMALL or _LARGE). */
+int moe_select_path(const moe_layer_desc* d);
+
+/*   x            [T, H] BF16 in.
+ *   out          [T, H] BF16 out; must not alias any input.
+ *   topk_w_out   [T, K] FP32 out or NULL (routing weights, as moe_router_topk).
+ *   topk_ids_out [T, K] int32 out or NULL.
+ *   logits_out   [T, E] FP32 out or NULL (the router logits used; a copy of
+ *                router_logits when those are given).
+ *   ws, ws_bytes workspace of at least moe_workspace_size(d) bytes, 256-byte aligned;
+ *                its first 256 bytes hold the device error word.
+ * The shared expert uses the routed activation and no gate.  Routing is computed with
+ * an FP32 logit accumulation whose order differs from a reference FP64 sum; experts
+ * whose keys differ by less than that rounding may be chosen either way. */
+moe_status_t moe_fused_forward(const moe_layer_desc* d, const void* x, void* out,
+                               float* topk_w_out, int32_t* topk_ids_out, float* logits_out,
+                               void* ws, size_t ws_bytes, void* stream);
+
+/* Number of kernels moe_fused_forward enqueues for this description (for accounting). */
+int moe_fused_forward_launches(const moe_layer_desc* d);
+
+/* moe_fused_forward with per-kernel timing: `events` holds n_events >= launches + 1
+ * cudaEvent_t handles created by the caller; event i is recorded on `stream` before the
+ * i-th kernel and event `launches` after the last.  Recording events between the kernels
+ * disables their programmatic overlap, so this variant is for attribution, not for the
+ * headline timing.  Same arguments and errors as moe_fused_forward, plus
+ * MOE_ERR_INVALID_ARG when n_events is too small. */
+moe_status_t moe_fused_forward_timed(const moe_layer_desc* d, const void* x, void* out, float* topk_w_out,
+                                     int32_t* topk_ids_out, float* logits_out, void* ws, size_t ws_bytes,
+                                     void* stream, void* const* events, int n_events);
+
+/* ------------------------------------------------------------------------------------
+ * moe_get_error -- read and clear the device error word at the start of `ws`
+ * (a moe_fused_forward or moe_permute workspace).  Synchronises `stream`.
+ *   code  out: OR of MOE_DEVERR_* flags set since the last read (0 = none).
+ * Returns MOE_ERR_DEVICE when code != 0, MOE_OK otherwise, MOE_ERR_CUDA if the copy fails.
+ * ---------------------------------------------------------------------------------- */
+moe_status_t moe_get_error(void* ws, int* code, void* stream);
+
+/* Human-readable name of a status code (static storage). */
+const char* moe_status_string(moe_status_t s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_H */

@@ -1,0 +1,451 @@
+// api.cu -- the C ABI of libmoe.so: host-side validation, workspace layout, path
+// selection, tensor-map encoding and the launch sequence of each path.  Nothing here
+// allocates or synchronises device memory (except moe_get_error).
+#include <cstring>
+
+#include "kernels.cuh"
+
+using namespace moe;
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+
+// Workspace carve-up of moe_fused_forward, 256-byte aligned regions after the header.
+struct WsLayout {
+    size_t logits, topk_w, topk_ids, offsets, tiles1, tiles2, perm, h, hs, acc, ys, total;
+};
+WsLayout layout(const moe_layer_desc* d) {
+    const size_t T = (size_t)d->T, E = (size_t)d->E, K = (size_t)d->top_k, H = (size_t)d->H, I = (size_t)d->I,
+                 Is = (size_t)d->I_shared;
+    WsLayout L;
+    size_t o = kHeaderBytes;
+    auto take = [&](size_t bytes) {
+        const size_t r = o;
+        o = align_up(o + bytes, 256);
+        return r;
+    };
+    L.logits = take(T * E * 4);
+    L.topk_w = take(T * K * 4);
+    L.topk_ids = take(T * K * 4);
+    L.offsets = take((E + 2) * 4);
+    L.tiles1 = take((E + 2) * 4);
+    L.tiles2 = take((E + 2) * 4);
+    L.perm = take(T * K * 4);
+    L.h = take(T * K * I * 2);
+    L.hs = take(T * Is * 2);
+    L.acc = take(T * H * 4);
+    L.ys = take(Is ? T * H * 2 : 0);
+    L.total = o;
+    return L;
+}
+
+moe_status_t validate_desc(const moe_layer_desc* d) {
+    if (!d) return MOE_ERR_INVALID_ARG;
+    if (d->T < 0 || d->H < 8 || d->I < 8 || d->E < 1 || d->top_k < 1) return MOE_ERR_INVALID_ARG;
+    if (d->H % 8 || d->I % 8 || d->I_shared < 0 || d->I_shared % 8) return MOE_ERR_INVALID_ARG;
+    if (d->act != MOE_ACT_SWIGLU && d->act != MOE_ACT_RELU2) return MOE_ERR_INVALID_ARG;
+    if (d->score != MOE_SCORE_SOFTMAX && d->score != MOE_SCORE_SIGMOID) return MOE_ERR_INVALID_ARG;
+    if (d->renorm != 0 && d->renorm != 1) return MOE_ERR_INVALID_ARG;
+    if (d->path < MOE_PATH_AUTO || d->path > MOE_PATH_LARGE) return MOE_ERR_INVALID_ARG;
+    if (d->top_k > d->E) return MOE_ERR_INVALID_ARG;
+    if (d->E > MOE_MAX_EXPERTS || d->top_k > MOE_MAX_TOPK || d->T > MOE_MAX_TOKENS) return MOE_ERR_UNSUPPORTED;
+    if (d->I_shared > 0 && d->E + 1 > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
+    if (!d->router_w && !d->router_logits) return MOE_ERR_INVALID_ARG;
+    if (!d->w13 || !d->w2) return MOE_ERR_INVALID_ARG;
+    if (d->I_shared > 0 && (!d->ws13 || !d->ws2)) return MOE_ERR_INVALID_ARG;
+    const void* ptrs[] = {d->router_w, d->router_logits, d->bias, d->w13, d->w2, d->ws13, d->ws2};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
+// Token-count rule of MOE_PATH_AUTO.  The streaming path reads each routed expert once
+// and wins while the experts see few tokens; the tensor-core path wins once its MMA
+// work per weight byte pays for the tile machinery.
+int auto_path(const moe_layer_desc* d) {
+    if (!small_path_supported(d->T, d->H, d->I, d->I_shared)) return MOE_PATH_LARGE;
+    return d->T <= 8 ? MOE_PATH_SMALL : MOE_PATH_LARGE;
+}
+int resolve_path(const moe_layer_desc* d) {
+    if (d->path == MOE_PATH_AUTO) return auto_path(d);
+    return d->path;
+}
+
+int num_sms() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+    return n;
+}
+
+// ---------------------------------------------------------------- tensor maps
+bool map2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows) {
+    EncodeTiledFn enc = get_encode_tiled();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {inner, rows};
+    cuuint64_t strides[1] = {inner * 2};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t es[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+bool map3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t depth, uint32_t box_rows) {
+    EncodeTiledFn enc = get_encode_tiled();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {inner, rows, depth};
+    cuuint64_t strides[2] = {inner * 2, inner * rows * 2};
+    cuuint32_t box[3] = {64, box_rows, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+#define MOE_CK(x)                                 \
+    do {                                          \
+        if ((x) != cudaSuccess) return MOE_ERR_CUDA; \
+    } while (0)
+
+// Router logits x . Wr^T on the tensor cores for many tokens (A = Wr, B = x rows).
+moe_status_t run_router_dense(const moe_layer_desc* d, const bf16* x, float* logits, float* copy, int sms,
+                              cudaStream_t s, int* err, bool pdl) {
+    GemmArgs g;
+    std::memset(&g, 0, sizeof(g));
+    g.T = d->T;
+    g.kdim = d->H;
+    g.nfeat_r = cdiv(d->E, 128);
+    g.feat_r = d->E;
+    g.E = 1;
+    g.dense = 1;
+    g.logits = logits;
+    g.logits_copy = copy;
+    g.err = err;
+    GemmMaps m;
+    std::memset(&m, 0, sizeof(m));
+    if (!map2d(&m.a_r, d->router_w, d->H, d->E, 128) || !map2d(&m.b_r, x, d->H, d->T, 16)) return MOE_ERR_CUDA;
+    m.a_s = m.a_r;
+    m.b_s = m.b_r;
+    const int tiles = g.nfeat_r * cdiv(d->T, 128);
+    MOE_CK(launch_gemm(GM_DENSE, g, m, std::min(sms, tiles), s, pdl));
+    return MOE_OK;
+}
+
+}  // namespace
+
+namespace moe {
+EncodeTiledFn get_encode_tiled() {
+    static EncodeTiledFn fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+}  // namespace moe
+
+extern "C" {
+
+const char* moe_status_string(moe_status_t s) {
+    switch (s) {
+        case MOE_OK: return "MOE_OK";
+        case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+        case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+        case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+        case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+        case MOE_ERR_DEVICE: return "MOE_ERR_DEVICE";
+    }
+    return "MOE_ERR_UNKNOWN";
+}
+
+moe_status_t moe_router_topk(const void* logits, int logits_dtype, int M, int E, int top_k, int score,
+                             const float* bias, int renorm, float* topk_w, int32_t* topk_ids, int32_t* src_idx,
+                             void* stream) {
+    if (M < 0 || E < 1 || top_k < 1 || top_k > E) return MOE_ERR_INVALID_ARG;
+    if (logits_dtype != MOE_DT_BF16 && logits_dtype != MOE_DT_FP32) return MOE_ERR_INVALID_ARG;
+    if (score != MOE_SCORE_SOFTMAX && score != MOE_SCORE_SIGMOID) return MOE_ERR_INVALID_ARG;
+    if (renorm != 0 && renorm != 1) return MOE_ERR_INVALID_ARG;
+    if (E > MOE_MAX_EXPERTS || top_k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED;
+    if (M == 0) return MOE_OK;
+    if (!logits || !topk_w || !topk_ids) return MOE_ERR_INVALID_ARG;
+    const void* ptrs[] = {logits, bias, topk_w, topk_ids, src_idx};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return MOE_ERR_INVALID_ARG;
+    if (launch_topk(logits, logits_dtype == MOE_DT_BF16, M, E, top_k, score, bias, renorm, topk_w, topk_ids, src_idx,
+                    nullptr, nullptr, (cudaStream_t)stream, false) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
+size_t moe_permute_workspace_size(int M, int K, int E) {
+    (void)M;
+    (void)K;
+    (void)E;
+    return kHeaderBytes;
+}
+
+moe_status_t moe_permute(const int32_t* topk_ids, int M, int K, int E, int32_t* expert_offsets, int32_t* perm,
+                         int32_t* inv, void* ws, size_t ws_bytes, void* stream) {
+    if (M < 0 || K < 1 || E < 1) return MOE_ERR_INVALID_ARG;
+    if (E > MOE_MAX_EXPERTS || K > MOE_MAX_TOPK || (long long)M * K > (long long)MOE_MAX_TOKENS * 8)
+        return MOE_ERR_UNSUPPORTED;
+    if (!ws || !aligned256(ws) || ws_bytes < moe_permute_workspace_size(M, K, E)) return MOE_ERR_WORKSPACE;
+    if (!expert_offsets || (M > 0 && (!topk_ids || !perm))) return MOE_ERR_INVALID_ARG;
+    const void* ptrs[] = {topk_ids, expert_offsets, perm, inv};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return MOE_ERR_INVALID_ARG;
+    PermuteArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.ids = topk_ids;
+    a.M = M;
+    a.K = K;
+    a.E = E;
+    a.offsets = expert_offsets;
+    a.perm = perm;
+    a.inv = inv;
+    a.err = &static_cast<WsHeader*>(ws)->err;
+    a.bn = 128;
+    if (launch_permute(a, (cudaStream_t)stream, false) != cudaSuccess) return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
+size_t moe_workspace_size(const moe_layer_desc* d) {
+    if (validate_desc(d) != MOE_OK) return 0;
+    return layout(d).total;
+}
+
+int moe_select_path(const moe_layer_desc* d) {
+    if (validate_desc(d) != MOE_OK) return -1;
+    return resolve_path(d);
+}
+
+int moe_fused_forward_launches(const moe_layer_desc* d) {
+    if (validate_desc(d) != MOE_OK || d->T == 0) return 0;
+    const int router = d->router_logits ? 0 : 1;
+    if (resolve_path(d) == MOE_PATH_SMALL) return router + 2;
+    return router + 5;  // topk, permute, fc1, fc2, finalize
+}
+
+static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, void* out_, float* topk_w_out,
+                                       int32_t* topk_ids_out, float* logits_out, void* ws, size_t ws_bytes,
+                                       void* stream, void* const* events, int n_events) {
+    moe_status_t st = validate_desc(d);
+    if (st != MOE_OK) return st;
+    if (d->T == 0) return MOE_OK;
+    if (!x_ || !out_ || !aligned16(x_) || !aligned16(out_)) return MOE_ERR_INVALID_ARG;
+    if ((topk_w_out && !aligned16(topk_w_out)) || (topk_ids_out && !aligned16(topk_ids_out)) ||
+        (logits_out && !aligned16(logits_out)))
+        return MOE_ERR_INVALID_ARG;
+    const WsLayout L = layout(d);
+    if (!ws || !aligned256(ws) || ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+    const int path = resolve_path(d);
+    if (path == MOE_PATH_SMALL && !small_path_supported(d->T, d->H, d->I, d->I_shared)) return MOE_ERR_UNSUPPORTED;
+
+    cudaStream_t s = (cudaStream_t)stream;
+    if (events && n_events < moe_fused_forward_launches(d) + 1) return MOE_ERR_INVALID_ARG;
+    int ev_i = 0;
+    // Records the next timing event (between kernels) when the caller asked for them.
+    auto mark = [&]() -> bool {
+        if (!events) return true;
+        return cudaEventRecord((cudaEvent_t)events[ev_i++], s) == cudaSuccess;
+    };
+    const bool timed = events != nullptr;
+    uint8_t* w8 = static_cast<uint8_t*>(ws);
+    int* err = &static_cast<WsHeader*>(ws)->err;
+    const bf16* x = static_cast<const bf16*>(x_);
+    bf16* out = static_cast<bf16*>(out_);
+    const int T = d->T, H = d->H, I = d->I, E = d->E, K = d->top_k, Is = d->I_shared;
+    const int sms = num_sms();
+
+    // 1. router logits
+    const float* logits = d->router_logits;
+    bool pdl = false;
+    if (!logits) {
+        float* lg = logits_out ? logits_out : reinterpret_cast<float*>(w8 + L.logits);
+        if (!mark()) return MOE_ERR_CUDA;
+        if (T <= 64) {
+            MOE_CK(launch_router_small(x, static_cast<const bf16*>(d->router_w), T, H, E, lg, nullptr, s, false));
+        } else {
+            st = run_router_dense(d, x, lg, nullptr, sms, s, err, false);
+            if (st != MOE_OK) return st;
+        }
+        logits = lg;
+        pdl = !timed;
+    } else if (logits_out) {
+        MOE_CK(cudaMemcpyAsync(logits_out, logits, (size_t)T * E * 4, cudaMemcpyDeviceToDevice, s));
+    }
+
+    if (path == MOE_PATH_SMALL) {
+        SmallArgs a;
+        std::memset(&a, 0, sizeof(a));
+        a.T = T;
+        a.H = H;
+        a.I = I;
+        a.E = E;
+        a.K = K;
+        a.act = d->act;
+        a.score = d->score;
+        a.renorm = d->renorm;
+        a.Is = Is;
+        a.logits = logits;
+        a.bias = d->bias;
+        a.x = x;
+        a.w13 = static_cast<const bf16*>(d->w13);
+        a.w2 = static_cast<const bf16*>(d->w2);
+        a.ws13 = static_cast<const bf16*>(d->ws13);
+        a.ws2 = static_cast<const bf16*>(d->ws2);
+        a.w_out = topk_w_out;
+        a.id_out = topk_ids_out;
+        a.h = reinterpret_cast<bf16*>(w8 + L.h);
+        a.hs = reinterpret_cast<bf16*>(w8 + L.hs);
+        a.out = out;
+        const std::function<bool()> mark_fn = mark;
+        MOE_CK(launch_small(a, sms, s, pdl, timed ? &mark_fn : nullptr));
+        if (!mark()) return MOE_ERR_CUDA;
+        return MOE_OK;
+    }
+
+    // ---- many-token path
+    float* tw = reinterpret_cast<float*>(w8 + L.topk_w);
+    int32_t* tid = reinterpret_cast<int32_t*>(w8 + L.topk_ids);
+    int32_t* offsets = reinterpret_cast<int32_t*>(w8 + L.offsets);
+    int32_t* tiles1 = reinterpret_cast<int32_t*>(w8 + L.tiles1);
+    int32_t* tiles2 = reinterpret_cast<int32_t*>(w8 + L.tiles2);
+    int32_t* perm = reinterpret_cast<int32_t*>(w8 + L.perm);
+    bf16* h = reinterpret_cast<bf16*>(w8 + L.h);
+    bf16* hs = reinterpret_cast<bf16*>(w8 + L.hs);
+    float* acc = reinterpret_cast<float*>(w8 + L.acc);
+    bf16* ys = Is ? reinterpret_cast<bf16*>(w8 + L.ys) : nullptr;
+
+    const bool chain = !timed;  // programmatic overlap between consecutive kernels
+    // 2. top-k
+    if (!mark()) return MOE_ERR_CUDA;
+    MOE_CK(launch_topk(logits, false, T, E, K, d->score, d->bias, d->renorm, tw, tid, nullptr, topk_w_out,
+                       topk_ids_out, s, pdl && chain));
+    // 3. permutation + tile tables
+    const bool swiglu = d->act == MOE_ACT_SWIGLU;
+    PermuteArgs pa;
+    std::memset(&pa, 0, sizeof(pa));
+    pa.ids = tid;
+    pa.M = T;
+    pa.K = K;
+    pa.E = E;
+    pa.offsets = offsets;
+    pa.perm = perm;
+    pa.err = err;
+    pa.has_shared = Is > 0;
+    pa.bn = 128;
+    pa.nfeat1_r = cdiv(I, 128);
+    pa.nfeat1_s = cdiv(Is, 128);
+    pa.nfeat2_r = cdiv(H, 128);
+    pa.nfeat2_s = cdiv(H, 128);
+    pa.tiles1 = tiles1;
+    pa.tiles2 = tiles2;
+    if (!mark()) return MOE_ERR_CUDA;
+    MOE_CK(launch_permute(pa, s, chain));
+
+    // 4. FC1 (+ activation), zeroing acc for FC2
+    const uint64_t rows1 = swiglu ? 2ull * I : (uint64_t)I;
+    const uint64_t rows1s = swiglu ? 2ull * Is : (uint64_t)Is;
+    GemmMaps m1;
+    std::memset(&m1, 0, sizeof(m1));
+    if (!map3d(&m1.a_r, d->w13, H, rows1, E, 128)) return MOE_ERR_CUDA;
+    if (Is) {
+        if (!map2d(&m1.a_s, d->ws13, H, rows1s, 128)) return MOE_ERR_CUDA;
+    } else {
+        m1.a_s = m1.a_r;
+    }
+    m1.b_r = m1.a_r;
+    m1.b_s = m1.a_r;
+    GemmArgs g1;
+    std::memset(&g1, 0, sizeof(g1));
+    g1.T = T;
+    g1.K = K;
+    g1.kdim = H;
+    g1.kdim_s = H;
+    g1.nfeat_r = cdiv(I, 128);
+    g1.nfeat_s = cdiv(Is, 128);
+    g1.feat_r = I;
+    g1.feat_s = Is;
+    g1.up_r = I;
+    g1.up_s = Is;
+    g1.E = E;
+    g1.has_shared = Is > 0;
+    g1.offsets = offsets;
+    g1.tiles = tiles1;
+    g1.perm = perm;
+    g1.topk_w = tw;
+    g1.xsrc = x;
+    g1.h = h;
+    g1.hs = hs;
+    g1.zero_ptr = acc;
+    g1.zero_n = (size_t)T * H;
+    g1.err = err;
+    if (!mark()) return MOE_ERR_CUDA;
+    MOE_CK(launch_gemm(swiglu ? GM_FC1_SWIGLU : GM_FC1_RELU2, g1, m1, sms, s, chain));
+
+    // 5. FC2 + weighted scatter-add (shared expert -> ys)
+    GemmMaps m2;
+    std::memset(&m2, 0, sizeof(m2));
+    if (!map3d(&m2.a_r, d->w2, I, H, E, 128) || !map2d(&m2.b_r, h, I, (uint64_t)T * K, 16)) return MOE_ERR_CUDA;
+    if (Is) {
+        if (!map2d(&m2.a_s, d->ws2, Is, H, 128) || !map2d(&m2.b_s, hs, Is, T, 16)) return MOE_ERR_CUDA;
+    } else {
+        m2.a_s = m2.a_r;
+        m2.b_s = m2.b_r;
+    }
+    GemmArgs g2 = g1;
+    g2.kdim = I;
+    g2.kdim_s = Is;
+    g2.nfeat_r = cdiv(H, 128);
+    g2.nfeat_s = cdiv(H, 128);
+    g2.feat_r = H;
+    g2.feat_s = H;
+    g2.tiles = tiles2;
+    g2.acc = acc;
+    g2.ys = ys;
+    g2.zero_ptr = nullptr;
+    g2.zero_n = 0;
+    if (!mark()) return MOE_ERR_CUDA;
+    MOE_CK(launch_gemm(GM_FC2, g2, m2, sms, s, chain));
+
+    // 6. finalize
+    if (!mark()) return MOE_ERR_CUDA;
+    MOE_CK(launch_finalize(acc, ys, out, (size_t)T * H, sms, s, chain));
+    if (!mark()) return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
+moe_status_t moe_fused_forward(const moe_layer_desc* d, const void* x, void* out, float* topk_w_out,
+                               int32_t* topk_ids_out, float* logits_out, void* ws, size_t ws_bytes, void* stream) {
+    return fused_forward_impl(d, x, out, topk_w_out, topk_ids_out, logits_out, ws, ws_bytes, stream, nullptr, 0);
+}
+
+moe_status_t moe_fused_forward_timed(const moe_layer_desc* d, const void* x, void* out, float* topk_w_out,
+                                     int32_t* topk_ids_out, float* logits_out, void* ws, size_t ws_bytes,
+                                     void* stream, void* const* events, int n_events) {
+    if (!events) return MOE_ERR_INVALID_ARG;
+    return fused_forward_impl(d, x, out, topk_w_out, topk_ids_out, logits_out, ws, ws_bytes, stream, events,
+                              n_events);
+}
+
+moe_status_t moe_get_error(void* ws, int* code, void* stream) {
+    if (!ws || !code) return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    int* err = &static_cast<WsHeader*>(ws)->err;
+    int v = 0;
+    if (cudaMemcpyAsync(&v, err, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaMemsetAsync(err, 0, sizeof(int), s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+    *code = v;
+    return v ? MOE_ERR_DEVICE : MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,435 @@
+// gemm.cu -- grouped BF16 GEMMs of the many-token path on the 5th-generation tensor
+// cores (tcgen05.mma, FP32 accumulators in TMEM), and the finalize kernel.
+//
+// Orientation ("swap AB"): the MMA's M side is 128 output features of one expert's
+// weight matrix, its N side is up to 128 routed token rows of that expert, so a tile's
+// MMA N is the expert's actual row count rounded up to 16 (no padding to 128 when an
+// expert receives few tokens).  K runs over the reduction dimension in 64-element steps
+// (one 128-byte swizzle row of BF16).
+//
+//   FC1 (FlashInfer PR #4646 walkthrough: grouped BF16 GEMM + activation): A = W13[e]
+//       rows of 128 features (SwiGLU: the gate and up halves as two accumulators), B =
+//       the expert's tokens gathered row by row from x with cp.async into the swizzled
+//       layout; epilogue applies SwiGLU / ReLU^2 and stores h (BF16) in permuted order.
+//   FC2: A = W2[e] rows of 128 output features, B = the expert's contiguous h rows
+//       (TMA, 16-row boxes); epilogue scales by the routing weight and adds into the
+//       FP32 accumulator acc[t, :] with red.global.add ("weighted output combination").
+//       The shared expert is one more group whose FC2 output is rounded to BF16 into ys.
+//   DENSE: router logits, A = Wr (128 experts per tile), B = x rows (TMA).
+//
+// Warp roles (one CTA per SM, persistent over a group-major tile list):
+//   warp 0      TMA producer (weights; FC2/DENSE token rows)
+//   warp 1      TMEM allocator and single-thread MMA issuer
+//   warps 2-5   epilogue: tcgen05.ld of the accumulator (warp w reads TMEM lanes of
+//               quarter w % 4), activation / scaling, stores
+//   warps 6-9   FC1 only: cp.async gather of token rows of x
+// Shared memory holds a ring of stages (full/empty mbarriers); TMEM holds two
+// accumulator buffers so the epilogue of one tile overlaps the mainloop of the next.
+#include "kernels.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int BM = 128, BN = 128, BK = 64;
+constexpr int A_BYTES = BM * BK * 2;  // 16 KB
+constexpr int B_BYTES = BN * BK * 2;  // 16 KB
+constexpr int BBOX = 16;              // token rows per TMA box of the B operand
+
+template <int MODE>
+struct Cfg {
+    static constexpr bool kGather = (MODE == GM_FC1_SWIGLU || MODE == GM_FC1_RELU2);
+    static constexpr bool kSwiglu = (MODE == GM_FC1_SWIGLU);
+    static constexpr int kNA = kSwiglu ? 2 : 1;
+    static constexpr int kStageBytes = kNA * A_BYTES + B_BYTES;
+    static constexpr int kStages = kSwiglu ? 4 : 6;
+    static constexpr int kAccCols = kSwiglu ? 2 * BN : BN;
+    static constexpr int kTmemCols = kSwiglu ? 512 : 256;
+    static constexpr int kThreads = kGather ? 320 : 192;
+    static constexpr int kLag = 2;
+    static constexpr int kMaxGroups = MOE_MAX_EXPERTS + 1;
+    // dynamic smem: alignment slack, stages, barriers, flags, tile and offset tables
+    static constexpr size_t kSmem =
+        1024 + (size_t)kStages * kStageBytes + 256 + (size_t)(kMaxGroups + 1) * 4 * 2 + 64;
+};
+
+struct TileInfo {
+    int g, ft, n, row0, shared;
+};
+
+__device__ __forceinline__ TileInfo decode_tile(const GemmArgs& a, const int* s_tiles, const int* s_offs, int G,
+                                                int tile) {
+    TileInfo ti;
+    if (a.dense) {
+        const int ntok = cdiv(a.T, BN);
+        ti.g = 0;
+        ti.ft = tile / ntok;
+        const int tt = tile - ti.ft * ntok;
+        ti.row0 = tt * BN;
+        ti.n = min(BN, a.T - ti.row0);
+        ti.shared = 0;
+        return ti;
+    }
+    int lo = 0, hi = G;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (s_tiles[mid] <= tile) lo = mid;
+        else hi = mid;
+    }
+    const int g = lo;
+    const int local = tile - s_tiles[g];
+    const bool sh = a.has_shared && g == a.E;
+    const int rows = sh ? a.T : (s_offs[g + 1] - s_offs[g]);
+    const int ntok = cdiv(rows, BN);
+    ti.g = g;
+    ti.ft = local / ntok;
+    const int tt = local - ti.ft * ntok;
+    ti.row0 = (sh ? 0 : s_offs[g]) + tt * BN;
+    ti.n = min(BN, rows - tt * BN);
+    ti.shared = sh;
+    return ti;
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
+    gemm_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ CUtensorMap tm_a_s,
+                const __grid_constant__ CUtensorMap tm_b_r, const __grid_constant__ CUtensorMap tm_b_s) {
+    using C = Cfg<MODE>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_u32 = smem_u32(smem_raw);
+    const uint32_t base_u32 = (raw_u32 + 1023u) & ~1023u;
+    uint8_t* base = smem_raw + (base_u32 - raw_u32);
+    uint8_t* meta = base + (size_t)C::kStages * C::kStageBytes;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(meta);  // full[S], empty[S], tfull[2], tempty[2]
+    const uint32_t bar_u32 = smem_u32(bars);
+    auto full_bar = [&](int s) { return bar_u32 + 8u * s; };
+    auto empty_bar = [&](int s) { return bar_u32 + 8u * (C::kStages + s); };
+    auto tfull_bar = [&](int b) { return bar_u32 + 8u * (2 * C::kStages + b); };
+    auto tempty_bar = [&](int b) { return bar_u32 + 8u * (2 * C::kStages + 2 + b); };
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(meta + 8 * (2 * C::kStages + 4));
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int* s_tiles = reinterpret_cast<int*>(meta + 256);
+    int* s_offs = s_tiles + C::kMaxGroups + 1;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int G = a.E + (a.has_shared ? 1 : 0);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(full_bar(s), C::kGather ? 1 + 128 : 1);
+            mbar_init(empty_bar(s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(tfull_bar(b), 1);
+            mbar_init(tempty_bar(b), 4);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tm_a_r);
+        if (a.has_shared) tma_prefetch_desc(&tm_a_s);
+        if (!C::kGather) {
+            tma_prefetch_desc(&tm_b_r);
+            if (a.has_shared) tma_prefetch_desc(&tm_b_s);
+        }
+    }
+    if (warp == 1) tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+
+    // Everything below reads what earlier kernels wrote (tile tables, perm, h).
+    pdl_wait();
+    if (!a.dense) {
+        for (int i = threadIdx.x; i <= G; i += blockDim.x) s_tiles[i] = a.tiles[i];
+        for (int i = threadIdx.x; i <= a.E; i += blockDim.x) s_offs[i] = a.offsets[i];
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int total = a.dense ? a.nfeat_r * cdiv(a.T, BN) : s_tiles[G];
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int it = 0;
+            for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
+                const TileInfo ti = decode_tile(a, s_tiles, s_offs, G, tile);
+                const bool sh = ti.shared;
+                const CUtensorMap* ta = sh ? &tm_a_s : &tm_a_r;
+                const CUtensorMap* tb = sh ? &tm_b_s : &tm_b_r;
+                const int kd = sh ? a.kdim_s : a.kdim;
+                const int nk = cdiv(kd, BK);
+                const int frow = ti.ft * BM;
+                const int nbox = cdiv(ti.n, BBOX);
+                const uint32_t bytes = C::kNA * A_BYTES + (C::kGather ? 0u : (uint32_t)nbox * BBOX * BK * 2);
+                for (int kb = 0; kb < nk; ++kb, ++it) {
+                    const int s = it % C::kStages;
+                    const uint32_t ph = (uint32_t)(it / C::kStages) & 1u;
+                    if (!mbar_wait(empty_bar(s), ph ^ 1u, abort_flag, a.err)) break;
+                    const uint32_t st = base_u32 + (uint32_t)s * C::kStageBytes;
+                    mbar_expect_tx(full_bar(s), bytes);
+                    if (sh || a.dense) {
+                        tma_load_2d(st, ta, full_bar(s), kb * BK, frow);
+                        if (C::kSwiglu) tma_load_2d(st + A_BYTES, ta, full_bar(s), kb * BK, a.up_s + frow);
+                    } else {
+                        tma_load_3d(st, ta, full_bar(s), kb * BK, frow, ti.g);
+                        if (C::kSwiglu) tma_load_3d(st + A_BYTES, ta, full_bar(s), kb * BK, a.up_r + frow, ti.g);
+                    }
+                    if (!C::kGather) {
+                        const uint32_t bs = st + C::kNA * A_BYTES;
+                        for (int q = 0; q < nbox; ++q)
+                            tma_load_2d(bs + (uint32_t)q * (BBOX * BK * 2), tb, full_bar(s), kb * BK,
+                                        ti.row0 + q * BBOX);
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int it = 0, tcount = 0;
+            for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x, ++tcount) {
+                const TileInfo ti = decode_tile(a, s_tiles, s_offs, G, tile);
+                const int kd = ti.shared ? a.kdim_s : a.kdim;
+                const int nk = cdiv(kd, BK);
+                const int npad = cdiv(ti.n, 16) * 16;
+                const uint32_t idesc = idesc_bf16_f32(BM, npad);
+                const int buf = tcount & 1;
+                const uint32_t tph = (uint32_t)(tcount >> 1) & 1u;
+                if (!mbar_wait(tempty_bar(buf), tph ^ 1u, abort_flag, a.err)) break;
+                tc_fence_after();
+                const uint32_t d0 = tmem_base + (uint32_t)(buf * C::kAccCols);
+                const uint32_t d1 = d0 + BN;
+                bool ok = true;
+                for (int kb = 0; kb < nk; ++kb, ++it) {
+                    const int s = it % C::kStages;
+                    const uint32_t ph = (uint32_t)(it / C::kStages) & 1u;
+                    if (!mbar_wait(full_bar(s), ph, abort_flag, a.err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t st = base_u32 + (uint32_t)s * C::kStageBytes;
+                    const uint32_t bsm = st + C::kNA * A_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
+                        const uint64_t bdesc = sdesc_sw128(bsm + kk * 32);
+                        tc_mma(d0, sdesc_sw128(st + kk * 32), bdesc, idesc, accum);
+                        if (C::kSwiglu) tc_mma(d1, sdesc_sw128(st + A_BYTES + kk * 32), bdesc, idesc, accum);
+                    }
+                    tc_commit(empty_bar(s));
+                }
+                if (!ok) break;
+                tc_commit(tfull_bar(buf));
+            }
+        }
+    } else if (warp < 6) {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;
+        const int et = threadIdx.x - 64;  // 0..127
+        if (a.zero_ptr) {
+            float4* z = reinterpret_cast<float4*>(a.zero_ptr);
+            const size_t n4 = a.zero_n / 4;
+            for (size_t i = (size_t)blockIdx.x * 128 + et; i < n4; i += (size_t)gridDim.x * 128)
+                z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        int tcount = 0;
+        for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x, ++tcount) {
+            const TileInfo ti = decode_tile(a, s_tiles, s_offs, G, tile);
+            const int buf = tcount & 1;
+            const uint32_t tph = (uint32_t)(tcount >> 1) & 1u;
+            if (!mbar_wait(tfull_bar(buf), tph, abort_flag, a.err)) break;
+            tc_fence_after();
+            const int f = ti.ft * BM + q * 32 + lane;
+            const int feat = ti.shared ? a.feat_s : a.feat_r;
+            const bool fok = f < feat;
+            const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * C::kAccCols);
+            for (int c0 = 0; c0 < ti.n; c0 += 32) {
+                uint32_t v[32];
+                tmem_ld32(tb + c0, v);
+                uint32_t u[32];
+                if (C::kSwiglu) tmem_ld32(tb + BN + c0, u);
+                tmem_ld_wait();
+                if (C::kGather) {
+                    bf16* dst = ti.shared ? a.hs : a.h;
+                    const int ld = feat;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int col = c0 + j;
+                        if (col < ti.n && fok) {
+                            float val;
+                            if (C::kSwiglu) val = act_swiglu(__uint_as_float(v[j]), __uint_as_float(u[j]));
+                            else val = act_relu2(__uint_as_float(v[j]));
+                            dst[(size_t)(ti.row0 + col) * ld + f] = __float2bfloat16_rn(val);
+                        }
+                    }
+                } else if (MODE == GM_FC2) {
+                    if (ti.shared) {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const int col = c0 + j;
+                            if (col < ti.n && fok)
+                                a.ys[(size_t)(ti.row0 + col) * a.feat_s + f] = __float2bfloat16_rn(__uint_as_float(v[j]));
+                        }
+                    } else {
+                        int my_t = 0;
+                        float my_w = 0.0f;
+                        const int colm = c0 + lane;
+                        if (colm < ti.n) {
+                            const int src = a.perm[ti.row0 + colm];
+                            const int kk = src / a.T;
+                            my_t = src - kk * a.T;
+                            my_w = a.topk_w[(size_t)my_t * a.K + kk];
+                        }
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const int t = __shfl_sync(0xffffffffu, my_t, j);
+                            const float w = __shfl_sync(0xffffffffu, my_w, j);
+                            if (c0 + j < ti.n && fok) atomicAdd(a.acc + (size_t)t * a.feat_r + f, w * __uint_as_float(v[j]));
+                        }
+                    }
+                } else {  // GM_DENSE
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int col = c0 + j;
+                        if (col < ti.n && fok) {
+                            const float val = __uint_as_float(v[j]);
+                            a.logits[(size_t)(ti.row0 + col) * a.feat_r + f] = val;
+                            if (a.logits_copy) a.logits_copy[(size_t)(ti.row0 + col) * a.feat_r + f] = val;
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tempty_bar(buf));
+        }
+    } else if (C::kGather) {
+        // ------------------------------------------------------------ FC1 token gather
+        const int p = threadIdx.x - 192;  // 0..127
+        const int chunk = p & 7, rsub = p >> 3;
+        int it = 0;
+        for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
+            const TileInfo ti = decode_tile(a, s_tiles, s_offs, G, tile);
+            const int kd = ti.shared ? a.kdim_s : a.kdim;
+            const int nk = cdiv(kd, BK);
+            const int npad = cdiv(ti.n, 16) * 16;
+            int tok[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int r = rsub + 16 * j;
+                tok[j] = -1;
+                if (r < ti.n) tok[j] = ti.shared ? ti.row0 + r : (a.perm[ti.row0 + r] % a.T);
+            }
+            bool ok = true;
+            for (int kb = 0; kb < nk; ++kb, ++it) {
+                const int s = it % C::kStages;
+                const uint32_t ph = (uint32_t)(it / C::kStages) & 1u;
+                if (!mbar_wait(empty_bar(s), ph ^ 1u, abort_flag, a.err)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t bs = base_u32 + (uint32_t)s * C::kStageBytes + C::kNA * A_BYTES;
+                const int kcol = kb * BK + chunk * 8;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int r = rsub + 16 * j;
+                    if (r < npad) {
+                        const uint32_t dst = bs + (uint32_t)r * 128u + ((uint32_t)(chunk ^ (r & 7)) << 4);
+                        const bool v = tok[j] >= 0 && kcol < kd;
+                        const bf16* src = v ? a.xsrc + (size_t)tok[j] * a.kdim + kcol : a.xsrc;
+                        cp_async16(dst, src, v ? 16u : 0u);
+                    }
+                }
+                cp_async_commit();
+                if (it >= C::kLag) {
+                    cp_async_wait<C::kLag>();
+                    fence_proxy_async_smem();
+                    mbar_arrive(full_bar((it - C::kLag) % C::kStages));
+                }
+            }
+            if (!ok) break;
+        }
+        cp_async_wait<0>();
+        fence_proxy_async_smem();
+        for (int j = max(0, it - C::kLag); j < it; ++j) mbar_arrive(full_bar(j % C::kStages));
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (*abort_flag) {  // let in-flight bulk copies and MMAs land before the CTA retires
+        const uint64_t t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 50000ull) {
+        }
+    }
+    if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
+    pdl_trigger();
+}
+
+// ---------------------------------------------------------------- finalize
+__global__ void __launch_bounds__(256) finalize_kernel(const float* __restrict__ acc, const bf16* __restrict__ ys,
+                                                       bf16* __restrict__ out, size_t n) {
+    pdl_wait();
+    const size_t stride = (size_t)gridDim.x * blockDim.x * 8;
+    for (size_t i = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) * 8; i < n; i += stride) {
+        const float4 a0 = *reinterpret_cast<const float4*>(acc + i);
+        const float4 a1 = *reinterpret_cast<const float4*>(acc + i + 4);
+        float r[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+        if (ys) {
+            const uint4 y = *reinterpret_cast<const uint4*>(ys + i);
+            const uint32_t yw[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                r[2 * j] = __fadd_rn(bf_round(r[2 * j]), bf16lo(yw[j]));
+                r[2 * j + 1] = __fadd_rn(bf_round(r[2 * j + 1]), bf16hi(yw[j]));
+            }
+        }
+        uint4 o;
+        o.x = (uint32_t)f2bf_bits(r[0]) | ((uint32_t)f2bf_bits(r[1]) << 16);
+        o.y = (uint32_t)f2bf_bits(r[2]) | ((uint32_t)f2bf_bits(r[3]) << 16);
+        o.z = (uint32_t)f2bf_bits(r[4]) | ((uint32_t)f2bf_bits(r[5]) << 16);
+        o.w = (uint32_t)f2bf_bits(r[6]) | ((uint32_t)f2bf_bits(r[7]) << 16);
+        *reinterpret_cast<uint4*>(out + i) = o;
+    }
+    pdl_trigger();
+}
+
+}  // namespace
+
+size_t gemm_smem_bytes(int mode) {
+    switch (mode) {
+        case GM_FC1_SWIGLU: return Cfg<GM_FC1_SWIGLU>::kSmem;
+        case GM_FC1_RELU2: return Cfg<GM_FC1_RELU2>::kSmem;
+        case GM_FC2: return Cfg<GM_FC2>::kSmem;
+        default: return Cfg<GM_DENSE>::kSmem;
+    }
+}
+
+template <int MODE>
+static cudaError_t launch_mode(const GemmArgs& a, const GemmMaps& m, int grid, cudaStream_t s, bool pdl) {
+    using C = Cfg<MODE>;
+    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
+    if (e != cudaSuccess) return e;
+    return launch_k(gemm_kernel<MODE>, dim3(grid), dim3(C::kThreads), C::kSmem, s, pdl, a, m.a_r, m.a_s, m.b_r, m.b_s);
+}
+
+cudaError_t launch_gemm(int mode, const GemmArgs& a, const GemmMaps& m, int grid, cudaStream_t s, bool pdl) {
+    switch (mode) {
+        case GM_FC1_SWIGLU: return launch_mode<GM_FC1_SWIGLU>(a, m, grid, s, pdl);
+        case GM_FC1_RELU2: return launch_mode<GM_FC1_RELU2>(a, m, grid, s, pdl);
+        case GM_FC2: return launch_mode<GM_FC2>(a, m, grid, s, pdl);
+        case GM_DENSE: return launch_mode<GM_DENSE>(a, m, grid, s, pdl);
+    }
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_finalize(const float* acc, const bf16* ys, bf16* out, size_t n, int num_sms, cudaStream_t s,
+                            bool pdl) {
+    const size_t groups = n / 8;
+    int grid = (int)std::min<size_t>((groups + 255) / 256, (size_t)num_sms * 4);
+    if (grid < 1) grid = 1;
+    return launch_k(finalize_kernel, dim3(grid), dim3(256), 0, s, pdl, acc, ys, out, n);
+}
+
+}  // namespace moe

@@ -1,0 +1,126 @@
+// kernels.cuh -- launch interfaces between the host API (api.cu) and the kernels.
+#pragma once
+#include <algorithm>
+#include <functional>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+
+// Launch with the programmatic-dependent-launch attribute when `pdl` is set: the kernel
+// may start while the previous kernel in the stream drains; every kernel calls
+// griddepcontrol.wait before it reads what the previous one wrote.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl,
+                     Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
+// ---------------------------------------------------------------- router
+cudaError_t launch_topk(const void* logits, bool bf16_in, int M, int E, int K, int score, const float* bias,
+                        int renorm, float* topk_w, int32_t* topk_ids, int32_t* src_idx, float* w_copy,
+                        int32_t* id_copy, cudaStream_t s, bool pdl);
+cudaError_t launch_router_small(const bf16* x, const bf16* wr, int T, int H, int E, float* logits,
+                                float* logits_copy, cudaStream_t s, bool pdl);
+
+// ---------------------------------------------------------------- few-token path
+static constexpr int kSmallMaxT = 16;
+struct SmallArgs {
+    int T, H, I, E, K, act, score, renorm, Is;
+    const float* logits;  // [T, E]
+    const float* bias;    // [E] or null
+    const bf16* x;
+    const bf16* w13;
+    const bf16* w2;
+    const bf16* ws13;
+    const bf16* ws2;
+    float* w_out;      // [T, K] caller output or null
+    int32_t* id_out;   // [T, K] caller output or null
+    bf16* h;           // [T*K, I], row = slot k*T + t
+    bf16* hs;          // [T, Is]
+    bf16* out;         // [T, H]
+};
+bool small_path_supported(int T, int H, int I, int Is);
+// `mark` (optional) records a timing event before each of the two kernels; when it is
+// given the kernels are launched without programmatic overlap.
+cudaError_t launch_small(const SmallArgs& a, int num_sms, cudaStream_t s, bool pdl_first,
+                         const std::function<bool()>* mark);
+
+// ---------------------------------------------------------------- permutation
+// Tile bookkeeping that the permute kernel writes for the grouped GEMMs (group g < E is
+// routed expert g; g == E is the shared expert when present, with T rows).
+struct PermuteArgs {
+    const int32_t* ids;  // [M, K]
+    int M, K, E;
+    int32_t* offsets;    // [E + 1]
+    int32_t* perm;       // [M*K]
+    int32_t* inv;        // [M*K] or null
+    int* err;
+    // grouped-GEMM tile tables (null when not wanted)
+    int has_shared;      // adds group E with M rows
+    int bn;              // token rows per tile
+    int nfeat1_r, nfeat1_s, nfeat2_r, nfeat2_s;
+    int32_t* tiles1;     // [G + 1] exclusive prefix of FC1 tiles over groups
+    int32_t* tiles2;     // [G + 1] exclusive prefix of FC2 tiles over groups
+};
+size_t permute_smem_bytes(int E);
+cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s, bool pdl);
+
+// ---------------------------------------------------------------- grouped tcgen05 GEMM
+enum GemmMode { GM_FC1_SWIGLU = 0, GM_FC1_RELU2 = 1, GM_FC2 = 2, GM_DENSE = 3 };
+struct GemmArgs {
+    int T, K;            // tokens and top-k (slot decode of perm entries)
+    int kdim;            // reduction length (H for FC1 / router, I or I_s for FC2)
+    int kdim_s;          // reduction length of the shared group
+    int nfeat_r, nfeat_s;  // 128-row feature tiles per routed / shared group
+    int feat_r, feat_s;    // valid output features per routed / shared group
+    int up_r, up_s;        // SwiGLU: row offset of the up half (I, I_s)
+    int E;               // routed groups; group E = shared (if has_shared)
+    int has_shared;
+    int dense;           // GM_DENSE: one group of T rows, tiles = nfeat_r * ceil(T / 128)
+    const int32_t* offsets;  // [E + 1] permuted row offsets of the routed groups
+    const int32_t* tiles;    // [G + 1] tile prefix (group-major)
+    const int32_t* perm;     // [T*K] source slot indices k*T + t
+    const float* topk_w;     // [T, K]
+    const bf16* xsrc;        // FC1 gather source x [T, H]
+    bf16* h;                 // FC1 routed out [T*K, I]
+    bf16* hs;                // FC1 shared out [T, I_s]
+    float* acc;              // FC2 routed out [T, H] (FP32 red.add)
+    bf16* ys;                // FC2 shared out [T, H]
+    float* logits;           // GM_DENSE out [T, E]
+    float* logits_copy;      // GM_DENSE optional second output
+    float* zero_ptr;         // FC1: buffer zeroed by the epilogue warps before their tiles
+    size_t zero_n;           //      (floats, multiple of 4)
+    int* err;
+};
+struct GemmMaps {
+    CUtensorMap a_r;  // routed weights (3D [E][rows][kdim]) or dense A (2D)
+    CUtensorMap a_s;  // shared weights (2D)
+    CUtensorMap b_r;  // FC2: h [T*K, I]; DENSE: x [T, H] (16-row boxes)
+    CUtensorMap b_s;  // FC2: hs [T, I_s]
+};
+cudaError_t launch_gemm(int mode, const GemmArgs& a, const GemmMaps& m, int grid, cudaStream_t s, bool pdl);
+size_t gemm_smem_bytes(int mode);
+int gemm_max_tiles_hint(int mode);
+
+// finalize: out = bf16(bf16(acc) + ys) or bf16(acc)
+cudaError_t launch_finalize(const float* acc, const bf16* ys, bf16* out, size_t n, int num_sms, cudaStream_t s,
+                            bool pdl);
+
+// Driver entry point for tensor-map encoding (resolved once through the runtime).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn get_encode_tiled();
+
+}  // namespace moe

@@ -1,0 +1,218 @@
+"""ctypes binding of libmoe.so (declared in include/moe.h).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA kernels.
+PyTorch supplies device memory and the current CUDA stream.  If the library has not
+been built, importing this module raises -- there is no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe.so")
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_DEVICE = range(6)
+SCORE = {"softmax": 0, "sigmoid": 1}
+ACT = {"swiglu": 0, "relu2": 1}
+PATH = {"auto": 0, "small": 1, "large": 2}
+DT_BF16, DT_FP32 = 0, 1
+DEVERR_BAD_EXPERT_ID, DEVERR_WAIT_TIMEOUT = 0x1, 0x2
+
+# Every symbol include/moe.h declares.
+EXPORTS = ("moe_router_topk", "moe_permute_workspace_size", "moe_permute", "moe_workspace_size",
+           "moe_select_path", "moe_fused_forward", "moe_fused_forward_launches", "moe_fused_forward_timed",
+           "moe_get_error", "moe_status_string")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m mixture_experts_layer_35_b200.build`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+_vp, _ci, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+
+
+class LayerDesc(ctypes.Structure):
+    """Mirror of moe_layer_desc."""
+    _fields_ = [(n, _ci) for n in ("T", "H", "I", "E", "top_k", "act", "score", "renorm", "I_shared", "path")] + [
+        ("router_w", _vp), ("router_logits", _vp), ("bias", _vp), ("w13", _vp), ("w2", _vp),
+        ("ws13", _vp), ("ws2", _vp)]
+
+
+_lib.moe_router_topk.argtypes = [_vp, _ci, _ci, _ci, _ci, _ci, _vp, _ci, _vp, _vp, _vp, _vp]
+_lib.moe_router_topk.restype = _ci
+_lib.moe_permute_workspace_size.argtypes = [_ci, _ci, _ci]
+_lib.moe_permute_workspace_size.restype = _sz
+_lib.moe_permute.argtypes = [_vp, _ci, _ci, _ci, _vp, _vp, _vp, _vp, _sz, _vp]
+_lib.moe_permute.restype = _ci
+_lib.moe_workspace_size.argtypes = [ctypes.POINTER(LayerDesc)]
+_lib.moe_workspace_size.restype = _sz
+_lib.moe_select_path.argtypes = [ctypes.POINTER(LayerDesc)]
+_lib.moe_select_path.restype = _ci
+_lib.moe_fused_forward_launches.argtypes = [ctypes.POINTER(LayerDesc)]
+_lib.moe_fused_forward_launches.restype = _ci
+_lib.moe_fused_forward.argtypes = [ctypes.POINTER(LayerDesc), _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+_lib.moe_fused_forward.restype = _ci
+_lib.moe_fused_forward_timed.argtypes = [ctypes.POINTER(LayerDesc), _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp,
+                                         ctypes.POINTER(_vp), _ci]
+_lib.moe_fused_forward_timed.restype = _ci
+_lib.moe_get_error.argtypes = [_vp, ctypes.POINTER(_ci), _vp]
+_lib.moe_get_error.restype = _ci
+_lib.moe_status_string.argtypes = [_ci]
+_lib.moe_status_string.restype = ctypes.c_char_p
+
+
+class MoEError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)}")
+
+
+def lib():
+    return _lib
+
+
+def status_string(s: int) -> str:
+    return _lib.moe_status_string(s).decode()
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream=None):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else stream
+
+
+def _check(st: int, where: str):
+    if st != MOE_OK:
+        raise MoEError(st, where)
+
+
+def router_topk(logits: torch.Tensor, top_k: int, score: str = "sigmoid", bias: Optional[torch.Tensor] = None,
+                renorm: bool = True, stream=None):
+    """Router top-k on [M, E] BF16 or FP32 device logits -> (weights f32, ids i32, src i32)."""
+    M, E = logits.shape
+    dev = logits.device
+    w = torch.empty((M, top_k), dtype=torch.float32, device=dev)
+    ids = torch.empty((M, top_k), dtype=torch.int32, device=dev)
+    src = torch.empty((M, top_k), dtype=torch.int32, device=dev)
+    dt = DT_BF16 if logits.dtype == torch.bfloat16 else DT_FP32
+    st = _lib.moe_router_topk(_ptr(logits), dt, M, E, top_k, SCORE[score], _ptr(bias), int(renorm),
+                              _ptr(w), _ptr(ids), _ptr(src), _stream(stream))
+    _check(st, "moe_router_topk")
+    return w, ids, src
+
+
+def permute_workspace_size(M: int, K: int, E: int) -> int:
+    return _lib.moe_permute_workspace_size(M, K, E)
+
+
+def permute(ids: torch.Tensor, E: int, ws: Optional[torch.Tensor] = None, stream=None):
+    """[M, K] int32 expert ids -> (offsets [E+1], perm [M*K], inv [M*K]) int32."""
+    M, K = ids.shape
+    dev = ids.device
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    perm = torch.empty(M * K, dtype=torch.int32, device=dev)
+    inv = torch.empty(M * K, dtype=torch.int32, device=dev)
+    if ws is None:
+        ws = torch.zeros(permute_workspace_size(M, K, E), dtype=torch.uint8, device=dev)
+    st = _lib.moe_permute(_ptr(ids), M, K, E, _ptr(offsets), _ptr(perm), _ptr(inv), _ptr(ws), ws.numel(),
+                          _stream(stream))
+    _check(st, "moe_permute")
+    return offsets, perm, inv
+
+
+def get_error(ws: torch.Tensor, stream=None) -> int:
+    code = _ci(0)
+    st = _lib.moe_get_error(_ptr(ws), ctypes.byref(code), _stream(stream))
+    if st not in (MOE_OK, MOE_ERR_DEVICE):
+        raise MoEError(st, "moe_get_error")
+    return code.value
+
+
+def make_desc(T: int, H: int, I: int, E: int, top_k: int, act: str, score: str, renorm: bool, I_shared: int,
+              path: str = "auto", router_w=None, router_logits=None, bias=None, w13=None, w2=None, ws13=None,
+              ws2=None) -> LayerDesc:
+    d = LayerDesc()
+    d.T, d.H, d.I, d.E, d.top_k = T, H, I, E, top_k
+    d.act, d.score, d.renorm, d.I_shared, d.path = ACT[act], SCORE[score], int(renorm), I_shared, PATH[path]
+    d.router_w, d.router_logits, d.bias = _ptr(router_w), _ptr(router_logits), _ptr(bias)
+    d.w13, d.w2, d.ws13, d.ws2 = _ptr(w13), _ptr(w2), _ptr(ws13), _ptr(ws2)
+    return d
+
+
+def workspace_size(desc: LayerDesc) -> int:
+    return _lib.moe_workspace_size(ctypes.byref(desc))
+
+
+def select_path(desc: LayerDesc) -> str:
+    p = _lib.moe_select_path(ctypes.byref(desc))
+    return {1: "small", 2: "large"}.get(p, "invalid")
+
+
+def launches(desc: LayerDesc) -> int:
+    return _lib.moe_fused_forward_launches(ctypes.byref(desc))
+
+
+def fused_forward_raw(desc: LayerDesc, x: torch.Tensor, out: torch.Tensor, ws: torch.Tensor,
+                      topk_w: Optional[torch.Tensor] = None, topk_ids: Optional[torch.Tensor] = None,
+                      logits: Optional[torch.Tensor] = None, stream=None):
+    st = _lib.moe_fused_forward(ctypes.byref(desc), _ptr(x), _ptr(out), _ptr(topk_w), _ptr(topk_ids),
+                                _ptr(logits), _ptr(ws), ws.numel(), _stream(stream))
+    _check(st, "moe_fused_forward")
+
+
+def fused_forward_timed(desc: LayerDesc, x: torch.Tensor, out: torch.Tensor, ws: torch.Tensor, events,
+                        stream=None):
+    """moe_fused_forward recording events[i] before kernel i and events[-1] after the last."""
+    arr = (_vp * len(events))(*[e.cuda_event for e in events])
+    st = _lib.moe_fused_forward_timed(ctypes.byref(desc), _ptr(x), _ptr(out), None, None, None, _ptr(ws),
+                                      ws.numel(), _stream(stream), arr, len(events))
+    _check(st, "moe_fused_forward_timed")
+
+
+class MoELayer:
+    """A layer whose weights live on the device; ``forward`` enqueues moe_fused_forward."""
+
+    def __init__(self, shape, weights: dict, path: str = "auto"):
+        self.shape = shape
+        self.w = weights
+        self.path = path
+        self._ws = None
+
+    def desc(self, T: int, router_logits: Optional[torch.Tensor] = None) -> LayerDesc:
+        s, w = self.shape, self.w
+        Is = s.I_shared if w.get("ws13") is not None else 0
+        return make_desc(T, s.H, s.I, s.E, s.K, s.act, s.score, s.renorm, Is, self.path,
+                         router_w=w.get("router_w"), router_logits=router_logits, bias=w.get("bias"),
+                         w13=w["w13"], w2=w["w2"], ws13=w.get("ws13"), ws2=w.get("ws2"))
+
+    def workspace(self, desc: LayerDesc, device) -> torch.Tensor:
+        need = workspace_size(desc)
+        if need == 0:
+            raise MoEError(MOE_ERR_INVALID_ARG, "moe_workspace_size")
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.zeros(need, dtype=torch.uint8, device=device)
+        return self._ws
+
+    def forward(self, x: torch.Tensor, router_logits: Optional[torch.Tensor] = None, out=None,
+                return_routing: bool = False, stream=None):
+        T = x.shape[0]
+        d = self.desc(T, router_logits)
+        ws = self.workspace(d, x.device)
+        if out is None:
+            out = torch.empty((T, self.shape.H), dtype=torch.bfloat16, device=x.device)
+        tw = ti = lg = None
+        if return_routing:
+            tw = torch.empty((T, self.shape.K), dtype=torch.float32, device=x.device)
+            ti = torch.empty((T, self.shape.K), dtype=torch.int32, device=x.device)
+            lg = torch.empty((T, self.shape.E), dtype=torch.float32, device=x.device)
+        fused_forward_raw(d, x, out, ws, tw, ti, lg, stream)
+        if return_routing:
+            return out, tw, ti, lg
+        return out

@@ -1,0 +1,122 @@
+"""CPU checks of the C ABI: the library loads, exports every function include/moe.h
+declares, and rejects bad arguments on the host before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import mixture_experts_layer_35_b200.moe as moe
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z_]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = _declared()
+    assert set(names) == set(moe.EXPORTS)
+    for n in names:
+        assert hasattr(moe.lib(), n), n
+
+
+def test_status_strings():
+    assert moe.status_string(0) == "MOE_OK"
+    assert moe.status_string(3) == "MOE_ERR_WORKSPACE"
+    assert moe.status_string(99) == "MOE_ERR_UNKNOWN"
+
+
+FAKE = 1 << 20  # a 16-byte aligned, never-dereferenced address
+
+
+def _desc(**kw):
+    base = dict(T=4, H=256, I=128, E=16, top_k=4, act="swiglu", score="sigmoid", renorm=True, I_shared=128)
+    base.update(kw)
+    d = moe.make_desc(**base)
+    d.router_w, d.w13, d.w2, d.ws13, d.ws2 = FAKE, FAKE * 2, FAKE * 3, FAKE * 4, FAKE * 5
+    return d
+
+
+def _fwd(d, x=FAKE * 6, out=FAKE * 7, ws=None, ws_bytes=0):
+    return moe.lib().moe_fused_forward(ctypes.byref(d), x, out, None, None, None, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("H", 250, moe.MOE_ERR_INVALID_ARG),
+    ("I", 4, moe.MOE_ERR_INVALID_ARG),
+    ("top_k", 17, moe.MOE_ERR_INVALID_ARG),
+    ("top_k", 0, moe.MOE_ERR_INVALID_ARG),
+    ("E", 2048, moe.MOE_ERR_UNSUPPORTED),
+    ("act", 7, moe.MOE_ERR_INVALID_ARG),
+    ("score", 5, moe.MOE_ERR_INVALID_ARG),
+    ("path", 9, moe.MOE_ERR_INVALID_ARG),
+    ("T", -1, moe.MOE_ERR_INVALID_ARG),
+    ("T", 1 << 20, moe.MOE_ERR_UNSUPPORTED),
+    ("I_shared", 12, moe.MOE_ERR_INVALID_ARG),
+])
+def test_forward_rejects_bad_descriptions(field, value, status):
+    d = _desc()
+    setattr(d, field, value)
+    assert _fwd(d) == status
+    assert moe.workspace_size(d) == 0
+
+
+def test_forward_rejects_missing_or_misaligned_pointers():
+    d = _desc()
+    d.w13 = None
+    assert _fwd(d) == moe.MOE_ERR_INVALID_ARG
+    d = _desc()
+    d.w2 = FAKE + 4
+    assert _fwd(d) == moe.MOE_ERR_INVALID_ARG
+    d = _desc()
+    d.router_w = None  # and no router logits
+    assert _fwd(d) == moe.MOE_ERR_INVALID_ARG
+    d = _desc()
+    assert _fwd(d, x=FAKE + 2) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_forward_checks_workspace_before_launch():
+    d = _desc()
+    need = moe.workspace_size(d)
+    assert need > 256
+    assert _fwd(d, ws=None, ws_bytes=need) == moe.MOE_ERR_WORKSPACE
+    assert _fwd(d, ws=FAKE * 8, ws_bytes=need - 1) == moe.MOE_ERR_WORKSPACE
+    assert _fwd(d, ws=FAKE * 8 + 16, ws_bytes=need) == moe.MOE_ERR_WORKSPACE
+
+
+def test_zero_tokens_is_a_noop():
+    d = _desc(T=0)
+    assert _fwd(d, ws=None, ws_bytes=0) == moe.MOE_OK
+    assert moe.launches(d) == 0
+
+
+def test_path_selection_and_launch_counts():
+    d = _desc(T=4)
+    assert moe.select_path(d) == "small"
+    assert moe.launches(d) == 3
+    d = _desc(T=4096)
+    assert moe.select_path(d) == "large"
+    assert moe.launches(d) == 6
+    d = _desc(T=4, path="large")
+    assert moe.select_path(d) == "large"
+    d = _desc(T=64, path="small")
+    assert moe.select_path(d) == "small"
+    assert _fwd(d, ws=FAKE * 8, ws_bytes=moe.workspace_size(d)) == moe.MOE_ERR_UNSUPPORTED
+
+
+def test_router_topk_and_permute_validation():
+    L = moe.lib()
+    assert L.moe_router_topk(FAKE, 0, 8, 16, 17, 1, None, 1, FAKE, FAKE, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_router_topk(FAKE, 3, 8, 16, 4, 1, None, 1, FAKE, FAKE, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_router_topk(FAKE, 0, 8, 2048, 4, 1, None, 1, FAKE, FAKE, None, None) == moe.MOE_ERR_UNSUPPORTED
+    assert L.moe_router_topk(None, 0, 0, 16, 4, 1, None, 1, None, None, None, None) == moe.MOE_OK
+    assert L.moe_router_topk(FAKE + 8, 1, 8, 16, 4, 1, None, 1, FAKE, FAKE, None, None) == moe.MOE_ERR_INVALID_ARG
+    need = moe.permute_workspace_size(8, 4, 16)
+    assert L.moe_permute(FAKE, 8, 4, 16, FAKE, FAKE, None, None, need, None) == moe.MOE_ERR_WORKSPACE
+    assert L.moe_permute(FAKE, 8, 4, 16, FAKE, FAKE, None, FAKE * 8, need - 1, None) == moe.MOE_ERR_WORKSPACE
+    assert L.moe_permute(FAKE, 8, 40, 16, FAKE, FAKE, None, FAKE * 8, need, None) == moe.MOE_ERR_UNSUPPORTED
+    assert L.moe_permute(FAKE, -1, 4, 16, FAKE, FAKE, None, FAKE * 8, need, None) == moe.MOE_ERR_INVALID_ARG
