@@ -210,6 +210,8 @@ class Bench:
         for _ in range(steps):
             self.flush()
             evs = [torch.cuda.Event(enable_timing=True) for _ in range(n + 1)]
+            for e in evs:  # torch creates the CUDA event on its first record
+                e.record()
             self.moe.fused_forward_timed(self.desc, self.d["x"], self.out, self.ws, evs)
             torch.cuda.synchronize(self.device)
             tot += np.array([evs[i].elapsed_time(evs[i + 1]) for i in range(n)])
@@ -303,7 +305,7 @@ def run_ours(args, rank, local, world):
     torch.cuda.empty_cache()
     if rank == 0 and world == 1 and not args.no_sweep:
         line["sweep"] = sweep(args, device, peaks)
-    if rank == 0 and world == 1:
+    if rank == 0 and world == 1 and not args.no_cpu:
         dcpu = gen.make_layer(shape, args.T, seed=args.seed, device=str(device), routing=args.routing)
         rate, n, dt = cpu_oracle_rate(shape, dcpu, args.cpu_budget, 400)
         line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": 1, "kind": "oracle",
@@ -389,6 +391,7 @@ def main(argv=None):
     p.add_argument("--seed", type=int, default=0)
     p.add_argument("--no-sweep", action="store_true")
     p.add_argument("--sweep-all", action="store_true")
+    p.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline (profiling runs)")
     p.add_argument("--cpu-budget", type=float, default=15.0)
     p.add_argument("--ref-tokens", type=int, default=4)
     args = p.parse_args(argv)

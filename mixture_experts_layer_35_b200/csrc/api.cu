@@ -267,6 +267,8 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
     // 1. router logits
     const float* logits = d->router_logits;
     bool pdl = false;
+    bool dense_router = false;
+    float* logits_rw = nullptr;
     if (!logits) {
         float* lg = logits_out ? logits_out : reinterpret_cast<float*>(w8 + L.logits);
         if (!mark()) return MOE_ERR_CUDA;
@@ -275,8 +277,10 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
         } else {
             st = run_router_dense(d, x, lg, nullptr, sms, s, err, false);
             if (st != MOE_OK) return st;
+            dense_router = true;
         }
         logits = lg;
+        logits_rw = lg;
         pdl = !timed;
     } else if (logits_out) {
         MOE_CK(cudaMemcpyAsync(logits_out, logits, (size_t)T * E * 4, cudaMemcpyDeviceToDevice, s));
@@ -327,8 +331,9 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
     const bool chain = !timed;  // programmatic overlap between consecutive kernels
     // 2. top-k
     if (!mark()) return MOE_ERR_CUDA;
+    RefineArgs ra = {x, static_cast<const bf16*>(d->router_w), H, logits_rw};
     MOE_CK(launch_topk(logits, false, T, E, K, d->score, d->bias, d->renorm, tw, tid, nullptr, topk_w_out,
-                       topk_ids_out, s, pdl && chain));
+                       topk_ids_out, s, pdl && chain, dense_router ? &ra : nullptr));
     // 3. permutation + tile tables
     const bool swiglu = d->act == MOE_ACT_SWIGLU;
     PermuteArgs pa;

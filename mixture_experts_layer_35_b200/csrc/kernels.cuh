@@ -27,9 +27,16 @@ cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
 }
 
 // ---------------------------------------------------------------- router
+// FP64 re-evaluation of the candidate logits after the tensor-core router (see router.cu).
+struct RefineArgs {
+    const bf16* x;       // [M, H]
+    const bf16* wr;      // [E, H]
+    int H;
+    float* logits_rw;    // refined logits are written back here (the logits buffer)
+};
 cudaError_t launch_topk(const void* logits, bool bf16_in, int M, int E, int K, int score, const float* bias,
                         int renorm, float* topk_w, int32_t* topk_ids, int32_t* src_idx, float* w_copy,
-                        int32_t* id_copy, cudaStream_t s, bool pdl);
+                        int32_t* id_copy, cudaStream_t s, bool pdl, const RefineArgs* refine = nullptr);
 cudaError_t launch_router_small(const bf16* x, const bf16* wr, int T, int H, int E, float* logits,
                                 float* logits_copy, cudaStream_t s, bool pdl);
 

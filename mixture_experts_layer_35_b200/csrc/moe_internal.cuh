@@ -46,6 +46,25 @@ __device__ __forceinline__ float dot8(const uint4& a, const uint4& b, float acc)
     return acc;
 }
 
+// Same in FP64: BF16 x BF16 products are exact in double, so only the additions round.
+__device__ __forceinline__ double dot8_f64(const uint4& a, const uint4& b, double acc) {
+    acc = fma((double)bf16lo(a.x), (double)bf16lo(b.x), acc);
+    acc = fma((double)bf16hi(a.x), (double)bf16hi(b.x), acc);
+    acc = fma((double)bf16lo(a.y), (double)bf16lo(b.y), acc);
+    acc = fma((double)bf16hi(a.y), (double)bf16hi(b.y), acc);
+    acc = fma((double)bf16lo(a.z), (double)bf16lo(b.z), acc);
+    acc = fma((double)bf16hi(a.z), (double)bf16hi(b.z), acc);
+    acc = fma((double)bf16lo(a.w), (double)bf16lo(b.w), acc);
+    acc = fma((double)bf16hi(a.w), (double)bf16hi(b.w), acc);
+    return acc;
+}
+
+__device__ __forceinline__ double warp_sum_f64(double v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
 // Streaming 16-byte load that does not allocate in L1 (weights are read once).
 __device__ __forceinline__ uint4 ld_stream16(const void* p) {
     uint4 r;

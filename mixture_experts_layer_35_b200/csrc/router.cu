@@ -6,12 +6,65 @@
 namespace moe {
 
 // ---------------------------------------------------------------- top-k, one warp per row
-template <int V, bool BF16_IN>
+// With `refine` (logits from the tensor-core router, FP32 accumulation in the MMA's own
+// order): a first selection on those logits; then every expert whose key lies within
+// `kRefineWindow` (relative) of the K-th key -- the selected ones included -- gets its
+// logit recomputed as an FP64 dot product rounded once to FP32, written back, and the
+// selection and weights are redone.  An expert outside the window cannot enter the top
+// K as long as the tensor-core logit error stays below half the window (it is ~1e-6
+// absolute on these workloads against a window of 2e-3), so ids and weights follow the
+// correctly rounded logits.
+static constexpr float kRefineWindow = 2e-3f;
+
+template <int V>
+__device__ __forceinline__ void refine_row(float (&l)[V], int row, int E, int K, int score, const float* bias,
+                                           int renorm, int lane, const bf16* x, const bf16* wr, int H,
+                                           float* logits_rw) {
+    int id;
+    float w, lg;
+    warp_topk_row<V>(l, E, K, score, bias, renorm, lane, id, w, lg);
+    // K-th key of the first selection
+    const int idK = __shfl_sync(0xffffffffu, id, K - 1);
+    const float lK = __shfl_sync(0xffffffffu, lg, K - 1);
+    float kK = (score == MOE_SCORE_SIGMOID) ? sigmoid_f32_rn(lK) : lK;
+    if (bias) kK = __fadd_rn(kK, bias[idK]);
+    const float win = kRefineWindow * fmaxf(1.0f, fabsf(kK)) * (score == MOE_SCORE_SIGMOID ? 0.25f : 1.0f);
+    const bf16* xr = x + (size_t)row * H;
+    const int nch = H >> 3;
+#pragma unroll
+    for (int c = 0; c < V; ++c) {
+        const int e = lane + 32 * c;
+        bool cand = false;
+        if (e < E) {
+            float k = (score == MOE_SCORE_SIGMOID) ? sigmoid_f32_rn(l[c]) : l[c];
+            if (bias) k = __fadd_rn(k, bias[e]);
+            cand = !(k < kK - win);  // also true for NaN
+        }
+        unsigned m = __ballot_sync(0xffffffffu, cand);
+        while (m) {
+            const int src = __ffs(m) - 1;
+            m &= m - 1;
+            const int ee = src + 32 * c;
+            const bf16* wrow = wr + (size_t)ee * H;
+            double acc = 0.0;
+            for (int q = lane; q < nch; q += 32)
+                acc = dot8_f64(ld_nc16(xr + (size_t)q * 8), ld_nc16(wrow + (size_t)q * 8), acc);
+            const float exact = __double2float_rn(warp_sum_f64(acc));
+            if (lane == src) {
+                l[c] = exact;
+                if (logits_rw) logits_rw[(size_t)row * E + ee] = exact;
+            }
+        }
+    }
+}
+
+template <int V, bool BF16_IN, bool REFINE>
 __global__ void __launch_bounds__(256) topk_kernel(const void* __restrict__ logits, int M, int E, int K, int score,
                                                    const float* __restrict__ bias, int renorm,
                                                    float* __restrict__ topk_w, int32_t* __restrict__ topk_ids,
                                                    int32_t* __restrict__ src_idx, float* __restrict__ w_copy,
-                                                   int32_t* __restrict__ id_copy) {
+                                                   int32_t* __restrict__ id_copy, const bf16* __restrict__ x,
+                                                   const bf16* __restrict__ wr, int H, float* logits_rw) {
     pdl_wait();
     const int lane = threadIdx.x & 31;
     const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -21,6 +74,7 @@ __global__ void __launch_bounds__(256) topk_kernel(const void* __restrict__ logi
             load_row_bf16<V>(static_cast<const uint16_t*>(logits) + (size_t)row * E, E, lane, l);
         else
             load_row_f32<V>(static_cast<const float*>(logits) + (size_t)row * E, E, lane, l);
+        if (REFINE) refine_row<V>(l, row, E, K, score, bias, renorm, lane, x, wr, H, logits_rw);
         int id;
         float w, lg;
         warp_topk_row<V>(l, E, K, score, bias, renorm, lane, id, w, lg);
@@ -38,16 +92,24 @@ __global__ void __launch_bounds__(256) topk_kernel(const void* __restrict__ logi
 
 cudaError_t launch_topk(const void* logits, bool bf16_in, int M, int E, int K, int score, const float* bias,
                         int renorm, float* topk_w, int32_t* topk_ids, int32_t* src_idx, float* w_copy,
-                        int32_t* id_copy, cudaStream_t s, bool pdl) {
+                        int32_t* id_copy, cudaStream_t s, bool pdl, const RefineArgs* refine) {
     const int rows_per_block = 8;
     dim3 grid(cdiv(M, rows_per_block)), block(32 * rows_per_block);
     const int v = topk_v(E);
-#define MOE_L(VV)                                                                                                \
-    if (v == VV)                                                                                                 \
-        return bf16_in ? launch_k(topk_kernel<VV, true>, grid, block, 0, s, pdl, logits, M, E, K, score, bias, \
-                                  renorm, topk_w, topk_ids, src_idx, w_copy, id_copy)                            \
-                       : launch_k(topk_kernel<VV, false>, grid, block, 0, s, pdl, logits, M, E, K, score, bias, \
-                                  renorm, topk_w, topk_ids, src_idx, w_copy, id_copy);
+    const bf16* x = refine ? refine->x : nullptr;
+    const bf16* wr = refine ? refine->wr : nullptr;
+    const int H = refine ? refine->H : 0;
+    float* lrw = refine ? refine->logits_rw : nullptr;
+#define MOE_L(VV)                                                                                              \
+    if (v == VV) {                                                                                             \
+        if (refine)                                                                                            \
+            return launch_k(topk_kernel<VV, false, true>, grid, block, 0, s, pdl, logits, M, E, K, score, bias, \
+                            renorm, topk_w, topk_ids, src_idx, w_copy, id_copy, x, wr, H, lrw);                \
+        return bf16_in ? launch_k(topk_kernel<VV, true, false>, grid, block, 0, s, pdl, logits, M, E, K, score, \
+                                  bias, renorm, topk_w, topk_ids, src_idx, w_copy, id_copy, x, wr, H, lrw)     \
+                       : launch_k(topk_kernel<VV, false, false>, grid, block, 0, s, pdl, logits, M, E, K, score, \
+                                  bias, renorm, topk_w, topk_ids, src_idx, w_copy, id_copy, x, wr, H, lrw);    \
+    }
     MOE_L(1) MOE_L(2) MOE_L(4) MOE_L(8) MOE_L(16) MOE_L(32)
 #undef MOE_L
     return cudaErrorInvalidValue;
@@ -56,7 +118,9 @@ cudaError_t launch_topk(const void* logits, bool bf16_in, int M, int E, int K, i
 // ---------------------------------------------------------------- router logits, few tokens
 // l[t, e] = x[t,:] . Wr[e,:].  One warp per expert row: the lanes stream the row in
 // 16-byte chunks once (HBM), and dot each chunk with the matching chunk of every token
-// (x is tiny and stays in L1/L2).  FP32 accumulation, XOR-tree reduction.
+// (x is tiny and stays in L1/L2).  The accumulation is FP64 (BF16 products are exact in
+// double), so the FP32 logit is the correctly rounded dot product except when the exact
+// value lies within ~1e-16 of an FP32 rounding boundary.
 template <int TT>
 __global__ void __launch_bounds__(128) router_logits_small(const bf16* __restrict__ x, const bf16* __restrict__ wr,
                                                            int T, int H, int E, float* __restrict__ logits,
@@ -68,18 +132,18 @@ __global__ void __launch_bounds__(128) router_logits_small(const bf16* __restric
         const int nch = H >> 3;  // 16-byte chunks per row
         const bf16* wrow = wr + (size_t)e * H;
         for (int t0 = 0; t0 < T; t0 += TT) {
-            float acc[TT];
+            double acc[TT];
 #pragma unroll
-            for (int j = 0; j < TT; ++j) acc[j] = 0.0f;
+            for (int j = 0; j < TT; ++j) acc[j] = 0.0;
             for (int c = lane; c < nch; c += 32) {
                 const uint4 w = ld_stream16(wrow + (size_t)c * 8);
 #pragma unroll
                 for (int j = 0; j < TT; ++j)
-                    if (t0 + j < T) acc[j] = dot8(w, ld_nc16(x + (size_t)(t0 + j) * H + (size_t)c * 8), acc[j]);
+                    if (t0 + j < T) acc[j] = dot8_f64(w, ld_nc16(x + (size_t)(t0 + j) * H + (size_t)c * 8), acc[j]);
             }
 #pragma unroll
             for (int j = 0; j < TT; ++j) {
-                const float v = warp_sum(acc[j]);
+                const float v = __double2float_rn(warp_sum_f64(acc[j]));
                 if (lane == 0 && t0 + j < T) {
                     logits[(size_t)(t0 + j) * E + e] = v;
                     if (logits_copy) logits_copy[(size_t)(t0 + j) * E + e] = v;

@@ -49,53 +49,15 @@ def assert_w_close(got, ref, what=""):
     assert rel.max() <= W_REL, f"{what}: routing weight rel err {rel.max():.3e}"
 
 
-def oracle_keys(logits, shape, bias):
-    """Selection keys from the oracle's FP32 logits (for tie margins only)."""
-    l = np.asarray(logits, np.float32)
-    if shape.score == "sigmoid":
-        s = (1.0 / (1.0 + np.exp(-l.astype(np.float64)))).astype(np.float32)
-        return s + (np.zeros_like(s) if bias is None else np.asarray(bias, np.float32))
-    return l if bias is None else (l + np.asarray(bias, np.float32))
-
-
-def routing_rows_unique(ref_logits, shape, bias, logit_tol):
-    """Rows whose top-K set (and slot order) cannot change under a logit perturbation of
-    `logit_tol`: every gap between consecutive keys down to the (K+1)-th exceeds twice
-    the induced key perturbation."""
-    keys = oracle_keys(ref_logits, shape, bias).astype(np.float64)
-    dk = logit_tol * (0.25 if shape.score == "sigmoid" else 1.0)
-    srt = -np.sort(-keys, axis=1)[:, :shape.K + 1]
-    gaps = srt[:, :-1] - srt[:, 1:]
-    return gaps.min(axis=1) > 2 * dk + 1e-12
-
-
 def check_fused_routing(gpu_ids, gpu_w, gpu_logits, ref_ids, ref_w, ref_logits, shape, bias, given_logits):
-    """IDs: bit-exact wherever the selection is unique.  With given logits that is every
-    row.  With logits computed on the GPU (FP32 accumulation in a different order than
-    the oracle's FP64 sum), rows whose key gaps lie within the logit rounding may
-    legitimately differ: there the GPU's choice must still be a valid top-K of the
-    oracle's keys up to that rounding.  Returns the mask of rows whose ids match."""
-    gpu_ids = np.asarray(gpu_ids)
-    ref_ids = np.asarray(ref_ids)
-    if given_logits:
-        np.testing.assert_array_equal(gpu_ids, ref_ids)
-        assert_w_close(gpu_w, ref_w, "routing weights")
-        return np.ones(len(ref_ids), bool)
+    """Routing of the fused path: expert ids bit-exact and weights within 1e-6 relative
+    on every row.  When the GPU computes the logits, the ones it returns lie within
+    1e-5 max|l| of the oracle's FP64-accumulated FP32 logits (the tensor-core router's
+    screening logits; the experts near the top-K boundary are re-evaluated in FP64 and
+    match the oracle's rounding)."""
+    np.testing.assert_array_equal(np.asarray(gpu_ids), np.asarray(ref_ids))
+    assert_w_close(gpu_w, ref_w, "routing weights")
     scale = max(np.abs(ref_logits).max(), 1.0)
-    tol = 1e-5 * scale
     lerr = np.abs(np.asarray(gpu_logits, np.float64) - ref_logits).max()
-    assert lerr <= tol, f"router logits err {lerr:.3e} > {tol:.3e}"
-    unique = routing_rows_unique(ref_logits, shape, bias, tol)
-    np.testing.assert_array_equal(gpu_ids[unique], ref_ids[unique])
-    same = np.all(gpu_ids == ref_ids, axis=1)
-    keys = oracle_keys(ref_logits, shape, bias).astype(np.float64)
-    dk = 2 * tol * (0.25 if shape.score == "sigmoid" else 1.0)
-    for r in np.nonzero(~same)[0]:
-        sel = set(gpu_ids[r].tolist())
-        assert len(sel) == shape.K
-        kin = min(keys[r, e] for e in sel)
-        kout = max((keys[r, e] for e in range(shape.E) if e not in sel), default=-np.inf)
-        assert kin >= kout - dk, f"row {r}: GPU selection is not a top-{shape.K} within rounding"
-    assert_w_close(gpu_w[same], ref_w[same], "routing weights")
-    assert (~same).sum() <= max(2, len(same) // 100)
-    return same
+    assert lerr <= 1e-5 * scale, f"router logits err {lerr:.3e} > {1e-5 * scale:.3e}"
+    return np.ones(len(ref_ids), bool)

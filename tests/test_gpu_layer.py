@@ -109,6 +109,21 @@ def test_full_shapes_prefill_sampled_rows(shape, T, routing, nrows):
     _check(shape, d, "auto", rows=rows, given_logits=(routing == "zipf"))
 
 
+@pytest.mark.parametrize("shape,T", [(gen.QWEN36, 4096), (gen.LARGE_E, 512), (gen.NEMOTRON, 300), (MULTI_A, 2000)])
+def test_fused_routing_every_row(shape, T):
+    """Tensor-core router + FP64 refine: ids bit-exact and weights within 1e-6 on every
+    row of the batch, against the oracle's logits and top-k over all rows."""
+    d = _util.device_layer(shape, T, seed=21)
+    layer = moe.MoELayer(shape, _util.weights_of(d), path="large")
+    out, tw, ti, lg = layer.forward(d["x"], return_routing=True)
+    torch.cuda.synchronize()
+    h = _util.host_copy(d)
+    ref_lg = oracle.router_logits(h["x"], h["router_w"])
+    rw, rids, _ = oracle.topk(ref_lg, shape.K, shape.score, h["bias"], shape.renorm)
+    _util.check_fused_routing(ti.cpu().numpy(), tw.cpu().numpy(), lg.cpu().numpy(), rids, rw, ref_lg, shape,
+                              h["bias"], False)
+
+
 def test_small_path_deterministic_and_graph_replay():
     shape = gen.QWEN36
     d = _util.device_layer(shape, 4, seed=5)
