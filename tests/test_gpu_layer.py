@@ -1,9 +1,8 @@
 """moe_fused_forward on the GPU against the CPU oracle, through the C ABI.
 
-Routing ids must match bit-exactly (rows with a genuine FP32 near-tie excepted when the
-logits are computed on the GPU, see tests/_util.check_fused_routing); routing weights
-within 1e-6 relative; layer output within max-abs <= 1e-2 max|ref| and
-mean-abs <= 1e-3 max|ref|.  Hand-derived fixtures must match bit for bit."""
+Routing ids must match bit-exactly on every row and routing weights within 1e-6
+relative (tests/_util.check_fused_routing); layer output within max-abs <= 1e-2 max|ref|
+and mean-abs <= 1e-3 max|ref|.  Hand-derived fixtures must match bit for bit."""
 import numpy as np
 import pytest
 import torch
