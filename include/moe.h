@@ -169,6 +169,31 @@ moe_status_t moe_fused_forward_timed(const moe_layer_desc* d, const void* x, voi
                                      void* stream, void* const* events, int n_events);
 
 /* ------------------------------------------------------------------------------------
+ * moe_fused_forward_noalloc -- moe_fused_forward for callers that cannot allocate.
+ * The pages have no counterpart: this is a deployment variant of this library.
+ * Some callers cannot allocate device memory at the point where they run the layer:
+ * code that runs while a CUDA graph is being captured (allocation calls are not
+ * capturable), runtimes that hand out a fixed memory pool and forbid further
+ * cudaMalloc, or plugins whose host framework owns every allocation.  This entry point
+ * takes the same description and buffers as moe_fused_forward minus the workspace: its
+ * scratch is a static device array of MOE_NOALLOC_SCRATCH_BYTES inside libmoe.so
+ * (every GPU that loads the library holds it until the process exits).  It allocates
+ * nothing and frees nothing.
+ *   - Returns MOE_ERR_WORKSPACE, before launching anything, when the description needs
+ *     more scratch than that (moe_workspace_size(d) > MOE_NOALLOC_SCRATCH_BYTES); the
+ *     other errors are those of moe_fused_forward.
+ *   - The first call on each device (with that device current) looks up the array's
+ *     device address; make that first call before any stream capture begins.
+ *   - All calls on a device share the array: calls whose GPU work overlaps (different
+ *     streams, concurrent graph launches) race and give wrong results.
+ *   - Device error flags are cleared at the start of each call and are not reported.
+ * ---------------------------------------------------------------------------------- */
+#define MOE_NOALLOC_SCRATCH_BYTES (4u << 20)
+moe_status_t moe_fused_forward_noalloc(const moe_layer_desc* d, const void* x, void* out,
+                                       float* topk_w_out, int32_t* topk_ids_out, float* logits_out,
+                                       void* stream);
+
+/* ------------------------------------------------------------------------------------
  * moe_get_error -- read and clear the device error word at the start of `ws`
  * (a moe_fused_forward or moe_permute workspace).  Synchronises `stream`.
  *   code  out: OR of MOE_DEVERR_* flags set since the last read (0 = none).

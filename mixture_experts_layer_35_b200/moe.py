@@ -25,7 +25,7 @@ DEVERR_BAD_EXPERT_ID, DEVERR_WAIT_TIMEOUT = 0x1, 0x2
 # Every symbol include/moe.h declares.
 EXPORTS = ("moe_router_topk", "moe_permute_workspace_size", "moe_permute", "moe_workspace_size",
            "moe_select_path", "moe_fused_forward", "moe_fused_forward_launches", "moe_fused_forward_timed",
-           "moe_get_error", "moe_status_string")
+           "moe_fused_forward_noalloc", "moe_get_error", "moe_status_string")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with `python -m mixture_experts_layer_35_b200.build`")
@@ -58,6 +58,9 @@ _lib.moe_fused_forward.restype = _ci
 _lib.moe_fused_forward_timed.argtypes = [ctypes.POINTER(LayerDesc), _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp,
                                          ctypes.POINTER(_vp), _ci]
 _lib.moe_fused_forward_timed.restype = _ci
+_lib.moe_fused_forward_noalloc.argtypes = [ctypes.POINTER(LayerDesc), _vp, _vp, _vp, _vp, _vp, _vp]
+_lib.moe_fused_forward_noalloc.restype = _ci
+NOALLOC_SCRATCH_BYTES = 4 << 20  # MOE_NOALLOC_SCRATCH_BYTES
 _lib.moe_get_error.argtypes = [_vp, ctypes.POINTER(_ci), _vp]
 _lib.moe_get_error.restype = _ci
 _lib.moe_status_string.argtypes = [_ci]
@@ -174,6 +177,15 @@ def fused_forward_timed(desc: LayerDesc, x: torch.Tensor, out: torch.Tensor, ws:
     st = _lib.moe_fused_forward_timed(ctypes.byref(desc), _ptr(x), _ptr(out), None, None, None, _ptr(ws),
                                       ws.numel(), _stream(stream), arr, len(events))
     _check(st, "moe_fused_forward_timed")
+
+
+def fused_forward_noalloc(desc: LayerDesc, x: torch.Tensor, out: torch.Tensor,
+                          topk_w: Optional[torch.Tensor] = None, topk_ids: Optional[torch.Tensor] = None,
+                          logits: Optional[torch.Tensor] = None, stream=None):
+    """moe_fused_forward_noalloc: no workspace argument; the library's static scratch is used."""
+    st = _lib.moe_fused_forward_noalloc(ctypes.byref(desc), _ptr(x), _ptr(out), _ptr(topk_w), _ptr(topk_ids),
+                                        _ptr(logits), _stream(stream))
+    _check(st, "moe_fused_forward_noalloc")
 
 
 class MoELayer:

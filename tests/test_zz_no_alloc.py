@@ -1,0 +1,47 @@
+"""moe_fused_forward_noalloc through the C ABI: for callers that cannot allocate device
+memory (inside CUDA-graph capture, under a fixed memory pool, or inside a host framework
+that owns all allocations), the layer runs on the library's static scratch array.  Its
+output must match the workspace entry point moe_fused_forward within the layer
+tolerance of the other tests, on two calls in a row (the second call finds the first
+call's leftovers in the shared array).  This file is collected last."""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import mixture_experts_layer_35_b200.moe as moe
+from mixture_experts_layer_35_b200 import inputs as gen
+from tests import _util
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("shape,T,path", [(gen.LARGE_E, 4, "small"), (gen.QWEN36, 64, "large"),
+                                          (gen.TINY, 4, "large")])
+def test_noalloc_matches_workspace_entry_point(shape, T, path):
+    d = _util.device_layer(shape, T, seed=31)
+    layer = moe.MoELayer(shape, _util.weights_of(d), path=path)
+    ref, ref_w, ref_ids, _ = layer.forward(d["x"], return_routing=True)
+    desc = layer.desc(T)
+    assert moe.workspace_size(desc) <= moe.NOALLOC_SCRATCH_BYTES
+    for _ in range(2):  # two calls in a row
+        out = torch.full((T, shape.H), float("nan"), dtype=torch.bfloat16, device="cuda")
+        tw = torch.empty((T, shape.K), dtype=torch.float32, device="cuda")
+        ti = torch.empty((T, shape.K), dtype=torch.int32, device="cuda")
+        moe.fused_forward_noalloc(desc, d["x"], out, tw, ti)
+        torch.cuda.synchronize()
+        assert torch.equal(ti, ref_ids)
+        _util.assert_w_close(tw.cpu().numpy(), ref_w.cpu().numpy())
+        _util.assert_out_close(gen.bf16_bits(out), gen.bf16_bits(ref), "noalloc vs workspace entry point")
+
+
+def test_noalloc_rejects_oversized_calls_before_launch():
+    shape = gen.QWEN36
+    d = _util.device_layer(shape, 1, seed=0)
+    layer = moe.MoELayer(shape, _util.weights_of(d))
+    desc = layer.desc(8192)  # needs ~150 MB of scratch
+    assert moe.workspace_size(desc) > moe.NOALLOC_SCRATCH_BYTES
+    st = moe.lib().moe_fused_forward_noalloc(ctypes.byref(desc), d["x"].data_ptr(), d["x"].data_ptr(), None, None,
+                                             None, None)
+    assert st == moe.MOE_ERR_WORKSPACE
