@@ -78,39 +78,57 @@ def load_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region: a
+    thread issues one-shot queries back to back until stopped (a streaming nvidia-smi
+    killed at the end loses its buffered output)."""
 
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
     def __init__(self, gpu_index: int):
-        self.proc = None
+        import threading
+        self.idx = gpu_index
+        self.rows = []
+        self.raw = []
+        self._stop = threading.Event()
+        self._t = threading.Thread(target=self._loop, daemon=True)
+        self._t.start()
+
+    def _query(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(gpu_index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except (OSError, ValueError):
-            self.proc = None
+            r = subprocess.run(["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                                "--format=csv,noheader,nounits"], capture_output=True, text=True, timeout=10)
+        except (OSError, subprocess.SubprocessError):
+            return
+        for line in r.stdout.strip().splitlines():
+            self.raw.append(line)
+            f = [x.strip() for x in line.split(",")]
+            if len(f) >= 8:
+                self.rows.append(f)
+
+    def _loop(self):
+        while not self._stop.is_set():
+            self._query()
 
     def stop(self):
-        if self.proc is None:
-            return None
-        self.proc.terminate()
-        try:
-            out, _ = self.proc.communicate(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-            out, _ = self.proc.communicate()
-        rows = [r.split(",") for r in out.strip().splitlines() if r.count(",") >= 7]
-        if not rows:
-            return None
-        sm = [float(r[0]) for r in rows if r[0].strip().replace(".", "").isdigit()]
-        mx = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
-        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        reasons = sorted({n for r in rows for n, v in zip(names, r[4:8]) if v.strip() == "Active"})
+        self._stop.set()
+        self._t.join(timeout=15)
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "raw": self.raw[:2]}
+
+        def num(v):
+            try:
+                return float(v)
+            except ValueError:
+                return None
+        sm = [v for v in (num(r[0]) for r in self.rows) if v is not None]
+        mx = [v for v in (num(r[1]) for r in self.rows) if v is not None]
+        reasons = sorted({n for r in self.rows for n, v in zip(self.REASONS, r[4:8]) if v == "Active"})
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+                "reasons": reasons, "samples": len(self.rows)}
 
 
 # ---------------------------------------------------------------- algorithmic accounting
@@ -171,16 +189,29 @@ class Bench:
         self.launches = moe.launches(self.desc)
         self.Is = shape.I_shared if w.get("ws13") is not None else 0
         self.flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+        # One complete layer forward per CUDA-graph replay (the launch sequence is
+        # captured once; replays carry no host launch overhead).
+        self.stream = torch.cuda.Stream(device)
+        self.step_eager(stream=self.stream)  # tensor-map and attribute set-up outside capture
+        torch.cuda.synchronize(device)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph, stream=self.stream):
+            self.step_eager(stream=self.stream)
+        torch.cuda.synchronize(device)
 
     def flush(self):
         self.flush_buf.fill_(1)
 
-    def step(self, x=None, out=None, stream=None):
+    def step_eager(self, x=None, out=None, stream=None):
         self.moe.fused_forward_raw(self.desc, self.d["x"] if x is None else x, self.out if out is None else out,
                                    self.ws, stream=stream)
 
+    def step(self):
+        self.graph.replay()
+
     def distinct_experts(self):
-        _, _, ids, _ = self.layer.forward(self.d["x"], router_logits=self.logits, return_routing=True)
+        _, _, ids, _ = self.layer.forward(self.d["x"], router_logits=self.logits, return_routing=True,
+                                          stream=self.stream)
         torch.cuda.synchronize(self.device)
         return int(torch.unique(ids).numel())
 
@@ -205,13 +236,19 @@ class Bench:
         return per, clk
 
     def per_kernel(self, steps: int):
+        """Average duration of each kernel of the step, from events recorded between the
+        launches (moe_fused_forward_timed).  Each call is enqueued right behind the L2
+        flush, so the host enqueues the kernels while the GPU is still busy and no
+        launch gap enters the intervals; the events do stop consecutive kernels from
+        overlapping, so the sum exceeds the graph-replay step slightly."""
         n = self.launches
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(n + 1)]
+        for e in evs:  # torch creates the CUDA event on its first record
+            e.record()
+        self.kernel_timing = "events between launches enqueued behind the L2 flush"
         tot = np.zeros(n)
         for _ in range(steps):
             self.flush()
-            evs = [torch.cuda.Event(enable_timing=True) for _ in range(n + 1)]
-            for e in evs:  # torch creates the CUDA event on its first record
-                e.record()
             self.moe.fused_forward_timed(self.desc, self.d["x"], self.out, self.ws, evs)
             torch.cuda.synchronize(self.device)
             tot += np.array([evs[i].elapsed_time(evs[i + 1]) for i in range(n)])
@@ -224,7 +261,7 @@ class Bench:
         x_dev = torch.empty_like(self.d["x"])
         for _ in range(warmup):
             x_dev.copy_(x_host, non_blocking=True)
-            self.step(x=x_dev)
+            self.step_eager(x=x_dev)
             out_host.copy_(self.out, non_blocking=True)
         torch.cuda.synchronize(self.device)
         ms = []
@@ -233,7 +270,7 @@ class Bench:
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record()
             x_dev.copy_(x_host, non_blocking=True)
-            self.step(x=x_dev)
+            self.step_eager(x=x_dev)
             out_host.copy_(self.out, non_blocking=True)
             b.record()
             torch.cuda.synchronize(self.device)
@@ -277,6 +314,7 @@ def run_ours(args, rank, local, world):
     dom_name = names[dom]
     roof = roofline_of(acc["kernels"][dom_name], kt[dom] / 1e3, peaks)
     roof["kernel"] = f"{dom_name} ({b.path} path)"
+    roof["timing"] = b.kernel_timing
     roof["traffic"] = None
     roof["peak_source"] = f"of {peaks_src}"
     layer_roof = roofline_of(acc["layer"], ms_step / 1e3, peaks)
@@ -290,6 +328,7 @@ def run_ours(args, rank, local, world):
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic (seeded generator, random-init weights of the layer's shape)",
         "config": {"workload": f"{shape.name} T={args.T} routing={args.routing}", "tokens_per_step": args.T,
+                   "timing": "one CUDA-graph replay of moe_fused_forward per step",
                    "path": b.path, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write), steps timed with CUDA events",
                    "distinct_experts": U},
@@ -382,8 +421,8 @@ def run_reference(args, rank, local, world):
 def main(argv=None):
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=20)
-    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--steps", type=int, default=100)
+    p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--config", choices=sorted(gen.SHORT), default="qwen36")
     p.add_argument("--T", type=int, default=4096)

@@ -14,7 +14,7 @@ bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) 
 
 // Workspace carve-up of moe_fused_forward, 256-byte aligned regions after the header.
 struct WsLayout {
-    size_t logits, topk_w, topk_ids, offsets, tiles1, tiles2, perm, h, hs, acc, ys, total;
+    size_t logits, topk_w, topk_ids, offsets, tiles1, tiles2, counts, perm, h, hs, acc, ys, total;
 };
 WsLayout layout(const moe_layer_desc* d) {
     const size_t T = (size_t)d->T, E = (size_t)d->E, K = (size_t)d->top_k, H = (size_t)d->H, I = (size_t)d->I,
@@ -32,6 +32,7 @@ WsLayout layout(const moe_layer_desc* d) {
     L.offsets = take((E + 2) * 4);
     L.tiles1 = take((E + 2) * 4);
     L.tiles2 = take((E + 2) * 4);
+    L.counts = take(2 * (E + 2) * 4);  // per-expert counts, then per-expert cursors
     L.perm = take(T * K * 4);
     L.h = take(T * K * I * 2);
     L.hs = take(T * Is * 2);
@@ -128,7 +129,7 @@ moe_status_t run_router_dense(const moe_layer_desc* d, const bf16* x, float* log
     if (!map2d(&m.a_r, d->router_w, d->H, d->E, 128) || !map2d(&m.b_r, x, d->H, d->T, 16)) return MOE_ERR_CUDA;
     m.a_s = m.a_r;
     m.b_s = m.b_r;
-    const int tiles = g.nfeat_r * cdiv(d->T, 128);
+    const int tiles = g.nfeat_r * cdiv(d->T, kDenseTokenTile);
     MOE_CK(launch_gemm(GM_DENSE, g, m, std::min(sms, tiles), s, pdl));
     return MOE_OK;
 }
@@ -272,7 +273,7 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
     if (!logits) {
         float* lg = logits_out ? logits_out : reinterpret_cast<float*>(w8 + L.logits);
         if (!mark()) return MOE_ERR_CUDA;
-        if (T <= 64) {
+        if (T <= 64 && router_small_supported(H)) {
             MOE_CK(launch_router_small(x, static_cast<const bf16*>(d->router_w), T, H, E, lg, nullptr, s, false));
         } else {
             st = run_router_dense(d, x, lg, nullptr, sms, s, err, false);
@@ -323,17 +324,20 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
     int32_t* tiles1 = reinterpret_cast<int32_t*>(w8 + L.tiles1);
     int32_t* tiles2 = reinterpret_cast<int32_t*>(w8 + L.tiles2);
     int32_t* perm = reinterpret_cast<int32_t*>(w8 + L.perm);
+    int* counts = reinterpret_cast<int*>(w8 + L.counts);
+    int* cursor = counts + (E + 2);
     bf16* h = reinterpret_cast<bf16*>(w8 + L.h);
     bf16* hs = reinterpret_cast<bf16*>(w8 + L.hs);
     float* acc = reinterpret_cast<float*>(w8 + L.acc);
     bf16* ys = Is ? reinterpret_cast<bf16*>(w8 + L.ys) : nullptr;
 
     const bool chain = !timed;  // programmatic overlap between consecutive kernels
-    // 2. top-k
+    // 2. top-k (also counts the slots per expert)
+    MOE_CK(cudaMemsetAsync(counts, 0, 2 * (size_t)(E + 2) * sizeof(int), s));
     if (!mark()) return MOE_ERR_CUDA;
     RefineArgs ra = {x, static_cast<const bf16*>(d->router_w), H, logits_rw};
     MOE_CK(launch_topk(logits, false, T, E, K, d->score, d->bias, d->renorm, tw, tid, nullptr, topk_w_out,
-                       topk_ids_out, s, pdl && chain, dense_router ? &ra : nullptr));
+                       topk_ids_out, s, pdl && chain, dense_router ? &ra : nullptr, counts));
     // 3. permutation + tile tables
     const bool swiglu = d->act == MOE_ACT_SWIGLU;
     PermuteArgs pa;
@@ -354,7 +358,7 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
     pa.tiles1 = tiles1;
     pa.tiles2 = tiles2;
     if (!mark()) return MOE_ERR_CUDA;
-    MOE_CK(launch_permute(pa, s, chain));
+    MOE_CK(launch_permute_fast(pa, counts, cursor, s, chain));
 
     // 4. FC1 (+ activation), zeroing acc for FC2
     const uint64_t rows1 = swiglu ? 2ull * I : (uint64_t)I;

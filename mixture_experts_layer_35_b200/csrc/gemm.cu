@@ -12,8 +12,10 @@
 //       the expert's tokens gathered row by row from x with cp.async into the swizzled
 //       layout; epilogue applies SwiGLU / ReLU^2 and stores h (BF16) in permuted order.
 //   FC2: A = W2[e] rows of 128 output features, B = the expert's contiguous h rows
-//       (TMA, 16-row boxes); epilogue scales by the routing weight and adds into the
-//       FP32 accumulator acc[t, :] with red.global.add ("weighted output combination").
+//       (TMA, 16-row boxes); epilogue scales by the routing weight, stages the block in
+//       shared memory and adds it into the FP32 accumulator acc[t, :] with asynchronous
+//       bulk reduce-adds, one 128-byte row segment per token ("weighted output
+//       combination").
 //       The shared expert is one more group whose FC2 output is rounded to BF16 into ys.
 //   DENSE: router logits, A = Wr (128 experts per tile), B = x rows (TMA).
 //
@@ -41,7 +43,10 @@ struct Cfg {
     static constexpr bool kSwiglu = (MODE == GM_FC1_SWIGLU);
     static constexpr int kNA = kSwiglu ? 2 : 1;
     static constexpr int kStageBytes = kNA * A_BYTES + B_BYTES;
-    static constexpr int kStages = kSwiglu ? 4 : 6;
+    static constexpr int kStages = kSwiglu ? 4 : (MODE == GM_FC2 ? 5 : 6);
+    // FC2: per epilogue warp, two [32 tokens][32 features] FP32 staging blocks for the
+    // bulk reduce-add into acc.
+    static constexpr int kEpiBytes = (MODE == GM_FC2) ? 4 * 2 * 32 * 32 * 4 : 0;
     static constexpr int kAccCols = kSwiglu ? 2 * BN : BN;
     static constexpr int kTmemCols = kSwiglu ? 512 : 256;
     static constexpr int kThreads = kGather ? 320 : 192;
@@ -49,7 +54,7 @@ struct Cfg {
     static constexpr int kMaxGroups = MOE_MAX_EXPERTS + 1;
     // dynamic smem: alignment slack, stages, barriers, flags, tile and offset tables
     static constexpr size_t kSmem =
-        1024 + (size_t)kStages * kStageBytes + 256 + (size_t)(kMaxGroups + 1) * 4 * 2 + 64;
+        1024 + (size_t)kStages * kStageBytes + kEpiBytes + 256 + (size_t)(kMaxGroups + 1) * 4 * 2 + 64;
 };
 
 struct TileInfo {
@@ -60,12 +65,12 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmArgs& a, const int* s_
                                                 int tile) {
     TileInfo ti;
     if (a.dense) {
-        const int ntok = cdiv(a.T, BN);
+        const int ntok = cdiv(a.T, kDenseTokenTile);
         ti.g = 0;
         ti.ft = tile / ntok;
         const int tt = tile - ti.ft * ntok;
-        ti.row0 = tt * BN;
-        ti.n = min(BN, a.T - ti.row0);
+        ti.row0 = tt * kDenseTokenTile;
+        ti.n = min(kDenseTokenTile, a.T - ti.row0);
         ti.shared = 0;
         return ti;
     }
@@ -98,7 +103,8 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
     const uint32_t raw_u32 = smem_u32(smem_raw);
     const uint32_t base_u32 = (raw_u32 + 1023u) & ~1023u;
     uint8_t* base = smem_raw + (base_u32 - raw_u32);
-    uint8_t* meta = base + (size_t)C::kStages * C::kStageBytes;
+    float* epi_stage = reinterpret_cast<float*>(base + (size_t)C::kStages * C::kStageBytes);
+    uint8_t* meta = base + (size_t)C::kStages * C::kStageBytes + C::kEpiBytes;
     uint64_t* bars = reinterpret_cast<uint64_t*>(meta);  // full[S], empty[S], tfull[2], tempty[2]
     const uint32_t bar_u32 = smem_u32(bars);
     auto full_bar = [&](int s) { return bar_u32 + 8u * s; };
@@ -145,7 +151,7 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    const int total = a.dense ? a.nfeat_r * cdiv(a.T, BN) : s_tiles[G];
+    const int total = a.dense ? a.nfeat_r * cdiv(a.T, kDenseTokenTile) : s_tiles[G];
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
@@ -234,6 +240,7 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
                 z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
         int tcount = 0;
+        int ebuf = 0;
         for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x, ++tcount) {
             const TileInfo ti = decode_tile(a, s_tiles, s_offs, G, tile);
             const int buf = tcount & 1;
@@ -272,6 +279,10 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
                                 a.ys[(size_t)(ti.row0 + col) * a.feat_s + f] = __float2bfloat16_rn(__uint_as_float(v[j]));
                         }
                     } else {
+                        // Column j of this chunk is token t_j with routing weight w_j.  The
+                        // warp stages w_j * y[f, j] as rows [j][32 features] in shared memory,
+                        // then lane j reduce-adds row j into acc[t_j, f0 .. f0+31] with one
+                        // asynchronous bulk reduction (FP32 add in L2).
                         int my_t = 0;
                         float my_w = 0.0f;
                         const int colm = c0 + lane;
@@ -281,12 +292,23 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
                             my_t = src - kk * a.T;
                             my_w = a.topk_w[(size_t)my_t * a.K + kk];
                         }
+                        float* stg = epi_stage + (size_t)(q * 2 + ebuf) * 32 * 32;
+                        bulk_wait_read<1>();  // the reads of this buffer's previous use are done
+                        __syncwarp();
 #pragma unroll
                         for (int j = 0; j < 32; ++j) {
-                            const int t = __shfl_sync(0xffffffffu, my_t, j);
                             const float w = __shfl_sync(0xffffffffu, my_w, j);
-                            if (c0 + j < ti.n && fok) atomicAdd(a.acc + (size_t)t * a.feat_r + f, w * __uint_as_float(v[j]));
+                            stg[j * 32 + lane] = w * __uint_as_float(v[j]);
                         }
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        const int fbase = ti.ft * BM + q * 32;
+                        const int nf = min(32, a.feat_r - fbase);
+                        if (colm < ti.n && nf > 0)
+                            bulk_reduce_add_f32(a.acc + (size_t)my_t * a.feat_r + fbase, smem_u32(stg + lane * 32),
+                                                (uint32_t)nf * 4u);
+                        bulk_commit();
+                        ebuf ^= 1;
                     }
                 } else {  // GM_DENSE
 #pragma unroll
@@ -304,6 +326,7 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(tempty_bar(buf));
         }
+        if (MODE == GM_FC2) bulk_wait_all<0>();  // every reduce-add issued by this thread has landed
     } else if (C::kGather) {
         // ------------------------------------------------------------ FC1 token gather
         const int p = threadIdx.x - 192;  // 0..127

@@ -36,7 +36,9 @@ struct RefineArgs {
 };
 cudaError_t launch_topk(const void* logits, bool bf16_in, int M, int E, int K, int score, const float* bias,
                         int renorm, float* topk_w, int32_t* topk_ids, int32_t* src_idx, float* w_copy,
-                        int32_t* id_copy, cudaStream_t s, bool pdl, const RefineArgs* refine = nullptr);
+                        int32_t* id_copy, cudaStream_t s, bool pdl, const RefineArgs* refine = nullptr,
+                        int* counts = nullptr);
+bool router_small_supported(int H);
 cudaError_t launch_router_small(const bf16* x, const bf16* wr, int T, int H, int E, float* logits,
                                 float* logits_copy, cudaStream_t s, bool pdl);
 
@@ -82,9 +84,16 @@ struct PermuteArgs {
 };
 size_t permute_smem_bytes(int E);
 cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s, bool pdl);
+// Fused-path permutation: the per-expert counts were accumulated by the top-k kernel;
+// slots are placed with per-expert atomic cursors (order within an expert is not
+// fixed).  `cursor` [E] must be zero on entry.
+cudaError_t launch_permute_fast(const PermuteArgs& a, const int* counts, int* cursor, cudaStream_t s, bool pdl);
 
 // ---------------------------------------------------------------- grouped tcgen05 GEMM
 enum GemmMode { GM_FC1_SWIGLU = 0, GM_FC1_RELU2 = 1, GM_FC2 = 2, GM_DENSE = 3 };
+// Token rows per tile of the dense router GEMM (E is small, so smaller token tiles give
+// the grid more CTAs).
+static constexpr int kDenseTokenTile = 64;
 struct GemmArgs {
     int T, K;            // tokens and top-k (slot decode of perm entries)
     int kdim;            // reduction length (H for FC1 / router, I or I_s for FC2)
@@ -94,7 +103,7 @@ struct GemmArgs {
     int up_r, up_s;        // SwiGLU: row offset of the up half (I, I_s)
     int E;               // routed groups; group E = shared (if has_shared)
     int has_shared;
-    int dense;           // GM_DENSE: one group of T rows, tiles = nfeat_r * ceil(T / 128)
+    int dense;           // GM_DENSE: one group of T rows, tiles = nfeat_r * ceil(T / kDenseTokenTile)
     const int32_t* offsets;  // [E + 1] permuted row offsets of the routed groups
     const int32_t* tiles;    // [G + 1] tile prefix (group-major)
     const int32_t* perm;     // [T*K] source slot indices k*T + t

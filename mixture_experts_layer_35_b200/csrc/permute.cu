@@ -47,6 +47,8 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp, int& tot
     return r;
 }
 
+__device__ void write_tile_tables(const PermuteArgs& a, int my_cnt, int* s_warp);
+
 __global__ void __launch_bounds__(kThreads, 1) permute_kernel(const PermuteArgs a) {
     extern __shared__ int smem[];
     const int E = a.E, M = a.M, K = a.K;
@@ -81,23 +83,7 @@ __global__ void __launch_bounds__(kThreads, 1) permute_kernel(const PermuteArgs 
     const int off = block_exclusive_scan(my_cnt, s_warp, total);
     if (tid < E) a.offsets[tid] = off;
     if (tid == 0) a.offsets[E] = total;
-    if (a.tiles1) {
-        const int G = E + (a.has_shared ? 1 : 0);
-        const int rows = (tid < E) ? my_cnt : (tid == E && a.has_shared ? M : 0);
-        const int ntok = cdiv(rows, a.bn);
-        const bool sh = tid == E;
-        int tot1, tot2;
-        const int p1 = block_exclusive_scan(tid < G ? ntok * (sh ? a.nfeat1_s : a.nfeat1_r) : 0, s_warp, tot1);
-        const int p2 = block_exclusive_scan(tid < G ? ntok * (sh ? a.nfeat2_s : a.nfeat2_r) : 0, s_warp, tot2);
-        if (tid < G) {
-            a.tiles1[tid] = p1;
-            a.tiles2[tid] = p2;
-        }
-        if (tid == 0) {
-            a.tiles1[G] = tot1;
-            a.tiles2[G] = tot2;
-        }
-    }
+    if (a.tiles1) write_tile_tables(a, my_cnt, s_warp);
     if (tid < E) {
         for (int w = 0; w < 32; ++w) hist[w * E + tid] += off;
     }
@@ -122,7 +108,66 @@ __global__ void __launch_bounds__(kThreads, 1) permute_kernel(const PermuteArgs 
     pdl_trigger();
 }
 
+// Tile tables of the grouped GEMMs from the per-expert counts (one thread per group).
+__device__ void write_tile_tables(const PermuteArgs& a, int my_cnt, int* s_warp) {
+    const int tid = threadIdx.x, E = a.E, M = a.M;
+    const int G = E + (a.has_shared ? 1 : 0);
+    const int rows = (tid < E) ? my_cnt : (tid == E && a.has_shared ? M : 0);
+    const int ntok = cdiv(rows, a.bn);
+    const bool sh = tid == E;
+    int tot1, tot2;
+    const int p1 = block_exclusive_scan(tid < G ? ntok * (sh ? a.nfeat1_s : a.nfeat1_r) : 0, s_warp, tot1);
+    const int p2 = block_exclusive_scan(tid < G ? ntok * (sh ? a.nfeat2_s : a.nfeat2_r) : 0, s_warp, tot2);
+    if (tid < G) {
+        a.tiles1[tid] = p1;
+        a.tiles2[tid] = p2;
+    }
+    if (tid == 0) {
+        a.tiles1[G] = tot1;
+        a.tiles2[G] = tot2;
+    }
+}
+
+// Every CTA scans the counts into offsets (E <= 1024 values); CTA 0 also publishes the
+// offsets and the tile tables; each thread then places one slot.
+__global__ void __launch_bounds__(kThreads) permute_fast_kernel(const PermuteArgs a, const int* __restrict__ counts,
+                                                               int* __restrict__ cursor) {
+    __shared__ int s_off[MOE_MAX_EXPERTS];
+    __shared__ int s_warp[33];
+    const int tid = threadIdx.x, E = a.E;
+    pdl_wait();
+    const int my_cnt = (tid < E) ? counts[tid] : 0;
+    int total;
+    const int off = block_exclusive_scan(my_cnt, s_warp, total);
+    if (tid < E) s_off[tid] = off;
+    if (blockIdx.x == 0) {
+        if (tid < E) a.offsets[tid] = off;
+        if (tid == 0) a.offsets[E] = total;
+        if (a.tiles1) write_tile_tables(a, my_cnt, s_warp);
+    }
+    __syncthreads();
+    const long long i = (long long)blockIdx.x * kThreads + tid;
+    if (i < (long long)a.M * a.K) {
+        const int e = a.ids[i];
+        if ((unsigned)e < (unsigned)E) {
+            const int t = (int)(i / a.K), k = (int)(i - (long long)t * a.K);
+            const int pos = s_off[e] + atomicAdd(cursor + e, 1);
+            a.perm[pos] = k * a.M + t;
+            if (a.inv) a.inv[k * a.M + t] = pos;
+        } else {
+            set_dev_error(a.err, MOE_DEVERR_BAD_EXPERT_ID);
+        }
+    }
+    pdl_trigger();
+}
+
 }  // namespace
+
+cudaError_t launch_permute_fast(const PermuteArgs& a, const int* counts, int* cursor, cudaStream_t s, bool pdl) {
+    const long long n = (long long)a.M * a.K;
+    const int grid = (int)std::max<long long>(1, (n + kThreads - 1) / kThreads);
+    return launch_k(permute_fast_kernel, dim3(grid), dim3(kThreads), 0, s, pdl, a, counts, cursor);
+}
 
 size_t permute_smem_bytes(int E) { return (size_t)(33 * E) * sizeof(int); }
 

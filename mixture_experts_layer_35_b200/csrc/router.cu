@@ -46,10 +46,21 @@ __device__ __forceinline__ void refine_row(float (&l)[V], int row, int E, int K,
             m &= m - 1;
             const int ee = src + 32 * c;
             const bf16* wrow = wr + (size_t)ee * H;
-            double acc = 0.0;
-            for (int q = lane; q < nch; q += 32)
-                acc = dot8_f64(ld_nc16(xr + (size_t)q * 8), ld_nc16(wrow + (size_t)q * 8), acc);
-            const float exact = __double2float_rn(warp_sum_f64(acc));
+            // four independent partial sums keep four 16-byte chunks of the row in flight
+            double acc0 = 0.0, acc1 = 0.0, acc2 = 0.0, acc3 = 0.0;
+            int q = lane;
+            for (; q + 96 < nch; q += 128) {
+                const uint4 w0 = ld_nc16(wrow + (size_t)q * 8), w1 = ld_nc16(wrow + (size_t)(q + 32) * 8);
+                const uint4 w2 = ld_nc16(wrow + (size_t)(q + 64) * 8), w3 = ld_nc16(wrow + (size_t)(q + 96) * 8);
+                const uint4 x0 = ld_nc16(xr + (size_t)q * 8), x1 = ld_nc16(xr + (size_t)(q + 32) * 8);
+                const uint4 x2 = ld_nc16(xr + (size_t)(q + 64) * 8), x3 = ld_nc16(xr + (size_t)(q + 96) * 8);
+                acc0 = dot8_f64(x0, w0, acc0);
+                acc1 = dot8_f64(x1, w1, acc1);
+                acc2 = dot8_f64(x2, w2, acc2);
+                acc3 = dot8_f64(x3, w3, acc3);
+            }
+            for (; q < nch; q += 32) acc0 = dot8_f64(ld_nc16(xr + (size_t)q * 8), ld_nc16(wrow + (size_t)q * 8), acc0);
+            const float exact = __double2float_rn(warp_sum_f64((acc0 + acc1) + (acc2 + acc3)));
             if (lane == src) {
                 l[c] = exact;
                 if (logits_rw) logits_rw[(size_t)row * E + ee] = exact;
@@ -64,7 +75,8 @@ __global__ void __launch_bounds__(256) topk_kernel(const void* __restrict__ logi
                                                    float* __restrict__ topk_w, int32_t* __restrict__ topk_ids,
                                                    int32_t* __restrict__ src_idx, float* __restrict__ w_copy,
                                                    int32_t* __restrict__ id_copy, const bf16* __restrict__ x,
-                                                   const bf16* __restrict__ wr, int H, float* logits_rw) {
+                                                   const bf16* __restrict__ wr, int H, float* logits_rw,
+                                                   int* __restrict__ counts) {
     pdl_wait();
     const int lane = threadIdx.x & 31;
     const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -85,6 +97,7 @@ __global__ void __launch_bounds__(256) topk_kernel(const void* __restrict__ logi
             if (src_idx) src_idx[o] = lane * M + row;
             if (w_copy) w_copy[o] = w;
             if (id_copy) id_copy[o] = id;
+            if (counts) atomicAdd(counts + id, 1);
         }
     }
     pdl_trigger();
@@ -92,7 +105,7 @@ __global__ void __launch_bounds__(256) topk_kernel(const void* __restrict__ logi
 
 cudaError_t launch_topk(const void* logits, bool bf16_in, int M, int E, int K, int score, const float* bias,
                         int renorm, float* topk_w, int32_t* topk_ids, int32_t* src_idx, float* w_copy,
-                        int32_t* id_copy, cudaStream_t s, bool pdl, const RefineArgs* refine) {
+                        int32_t* id_copy, cudaStream_t s, bool pdl, const RefineArgs* refine, int* counts) {
     const int rows_per_block = 8;
     dim3 grid(cdiv(M, rows_per_block)), block(32 * rows_per_block);
     const int v = topk_v(E);
@@ -104,11 +117,11 @@ cudaError_t launch_topk(const void* logits, bool bf16_in, int M, int E, int K, i
     if (v == VV) {                                                                                             \
         if (refine)                                                                                            \
             return launch_k(topk_kernel<VV, false, true>, grid, block, 0, s, pdl, logits, M, E, K, score, bias, \
-                            renorm, topk_w, topk_ids, src_idx, w_copy, id_copy, x, wr, H, lrw);                \
+                            renorm, topk_w, topk_ids, src_idx, w_copy, id_copy, x, wr, H, lrw, counts);        \
         return bf16_in ? launch_k(topk_kernel<VV, true, false>, grid, block, 0, s, pdl, logits, M, E, K, score, \
-                                  bias, renorm, topk_w, topk_ids, src_idx, w_copy, id_copy, x, wr, H, lrw)     \
+                                  bias, renorm, topk_w, topk_ids, src_idx, w_copy, id_copy, x, wr, H, lrw, counts) \
                        : launch_k(topk_kernel<VV, false, false>, grid, block, 0, s, pdl, logits, M, E, K, score, \
-                                  bias, renorm, topk_w, topk_ids, src_idx, w_copy, id_copy, x, wr, H, lrw);    \
+                                  bias, renorm, topk_w, topk_ids, src_idx, w_copy, id_copy, x, wr, H, lrw, counts); \
     }
     MOE_L(1) MOE_L(2) MOE_L(4) MOE_L(8) MOE_L(16) MOE_L(32)
 #undef MOE_L
@@ -121,7 +134,7 @@ cudaError_t launch_topk(const void* logits, bool bf16_in, int M, int E, int K, i
 // (x is tiny and stays in L1/L2).  The accumulation is FP64 (BF16 products are exact in
 // double), so the FP32 logit is the correctly rounded dot product except when the exact
 // value lies within ~1e-16 of an FP32 rounding boundary.
-template <int TT>
+template <int VH, int TT>
 __global__ void __launch_bounds__(128) router_logits_small(const bf16* __restrict__ x, const bf16* __restrict__ wr,
                                                            int T, int H, int E, float* __restrict__ logits,
                                                            float* __restrict__ logits_copy) {
@@ -131,22 +144,31 @@ __global__ void __launch_bounds__(128) router_logits_small(const bf16* __restric
     if (e < E) {
         const int nch = H >> 3;  // 16-byte chunks per row
         const bf16* wrow = wr + (size_t)e * H;
+        uint4 w[VH];  // the whole row is loaded at once: one memory latency per row
+#pragma unroll
+        for (int j = 0; j < VH; ++j) {
+            const int c = lane + 32 * j;
+            w[j] = (c < nch) ? ld_stream16(wrow + (size_t)c * 8) : make_uint4(0u, 0u, 0u, 0u);
+        }
         for (int t0 = 0; t0 < T; t0 += TT) {
             double acc[TT];
 #pragma unroll
-            for (int j = 0; j < TT; ++j) acc[j] = 0.0;
-            for (int c = lane; c < nch; c += 32) {
-                const uint4 w = ld_stream16(wrow + (size_t)c * 8);
+            for (int i = 0; i < TT; ++i) acc[i] = 0.0;
 #pragma unroll
-                for (int j = 0; j < TT; ++j)
-                    if (t0 + j < T) acc[j] = dot8_f64(w, ld_nc16(x + (size_t)(t0 + j) * H + (size_t)c * 8), acc[j]);
+            for (int j = 0; j < VH; ++j) {
+                const int c = lane + 32 * j;
+                if (c < nch) {
+#pragma unroll
+                    for (int i = 0; i < TT; ++i)
+                        if (t0 + i < T) acc[i] = dot8_f64(w[j], ld_nc16(x + (size_t)(t0 + i) * H + (size_t)c * 8), acc[i]);
+                }
             }
 #pragma unroll
-            for (int j = 0; j < TT; ++j) {
-                const float v = __double2float_rn(warp_sum_f64(acc[j]));
-                if (lane == 0 && t0 + j < T) {
-                    logits[(size_t)(t0 + j) * E + e] = v;
-                    if (logits_copy) logits_copy[(size_t)(t0 + j) * E + e] = v;
+            for (int i = 0; i < TT; ++i) {
+                const float v = __double2float_rn(warp_sum_f64(acc[i]));
+                if (lane == 0 && t0 + i < T) {
+                    logits[(size_t)(t0 + i) * E + e] = v;
+                    if (logits_copy) logits_copy[(size_t)(t0 + i) * E + e] = v;
                 }
             }
         }
@@ -154,12 +176,23 @@ __global__ void __launch_bounds__(128) router_logits_small(const bf16* __restric
     pdl_trigger();
 }
 
+bool router_small_supported(int H) { return (H >> 3) <= 32 * 16; }
+
 cudaError_t launch_router_small(const bf16* x, const bf16* wr, int T, int H, int E, float* logits,
                                 float* logits_copy, cudaStream_t s, bool pdl) {
     dim3 grid(cdiv(E, 4)), block(128);
-    if (T <= 4) return launch_k(router_logits_small<4>, grid, block, 0, s, pdl, x, wr, T, H, E, logits, logits_copy);
-    if (T <= 8) return launch_k(router_logits_small<8>, grid, block, 0, s, pdl, x, wr, T, H, E, logits, logits_copy);
-    return launch_k(router_logits_small<16>, grid, block, 0, s, pdl, x, wr, T, H, E, logits, logits_copy);
+    const int need = cdiv(H >> 3, 32);
+#define MOE_R(VV)                                                                                               \
+    if (need <= VV) {                                                                                           \
+        if (T <= 2)                                                                                             \
+            return launch_k(router_logits_small<VV, 2>, grid, block, 0, s, pdl, x, wr, T, H, E, logits, logits_copy); \
+        if (T <= 4)                                                                                             \
+            return launch_k(router_logits_small<VV, 4>, grid, block, 0, s, pdl, x, wr, T, H, E, logits, logits_copy); \
+        return launch_k(router_logits_small<VV, 8>, grid, block, 0, s, pdl, x, wr, T, H, E, logits, logits_copy);     \
+    }
+    MOE_R(4) MOE_R(8) MOE_R(12) MOE_R(16)
+#undef MOE_R
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace moe

@@ -12,8 +12,8 @@
 //              w[t,k] * (W2[e_k, f, :] . h[slot]) in FP32 over the slots, rounds to BF16,
 //              adds the BF16 shared-expert output and rounds again ("MTP1 isolated
 //              gather/shared-add closure": routed FP32 accumulation -> BF16 -> shared BF16
-//              add -> BF16), writing the layer output directly.  Before waiting for
-//              fc1 it prefetches its W2 rows into L2.
+//              add -> BF16), writing the layer output directly.  fc1 has already
+//              prefetched the routed experts' W2 into L2 while it streamed W13.
 #include "kernels.cuh"
 #include "router.cuh"
 
@@ -118,6 +118,29 @@ __global__ void __launch_bounds__(256) fc1_small(const SmallArgs a) {
     __syncthreads();
     pdl_trigger();
 
+    // Bring the W2 rows the next kernel needs into L2 while this one streams W13: the
+    // distinct experts' W2 matrices (contiguous [H, I] each) and the shared W2, split
+    // evenly over the CTAs in 32 KB bulk prefetches.
+    {
+        const size_t per = (size_t)H * I * 2;
+        const size_t tot = (size_t)U * per + (size_t)H * a.Is * 2;
+        const size_t lo = tot * blockIdx.x / gridDim.x, hi = tot * (blockIdx.x + 1) / gridDim.x;
+        const size_t lo16 = lo & ~(size_t)15, hi16 = (hi + 15) & ~(size_t)15;
+        for (size_t off = lo16 + (size_t)tid * 32768; off < hi16; off += (size_t)blockDim.x * 32768) {
+            const size_t end = off + 32768 < hi16 ? off + 32768 : hi16;
+            const size_t u = off / per;
+            if (u < (size_t)U) {
+                const size_t uend = (u + 1) * per;
+                const size_t stop = end < uend ? end : uend;
+                bulk_prefetch_l2(reinterpret_cast<const uint8_t*>(a.w2 + (size_t)s_ulist[u] * H * I) + (off - u * per),
+                                 (uint32_t)(stop - off));
+            } else {
+                const size_t so = off - (size_t)U * per;
+                bulk_prefetch_l2(reinterpret_cast<const uint8_t*>(a.ws2) + so, (uint32_t)(end - off));
+            }
+        }
+    }
+
     const int nch = H >> 3;
     const bool swiglu = a.act == MOE_ACT_SWIGLU;
     const long long Nr = (long long)U * I;
@@ -194,28 +217,41 @@ __global__ void __launch_bounds__(256) fc2_small(const SmallArgs a) {
     const int f0 = (int)((long long)blockIdx.x * H / gridDim.x);
     const int f1 = (int)((long long)(blockIdx.x + 1) * H / gridDim.x);
     const int nf = f1 - f0;
-    if (nf > 0) {  // bring this CTA's W2 rows into L2 while fc1 still runs
-        for (int i = tid; i < T * K; i += blockDim.x)
-            bulk_prefetch_l2(a.w2 + ((size_t)s_ids[i] * H + f0) * I, (uint32_t)((size_t)nf * I * 2));
-        if (tid == 0 && Is) bulk_prefetch_l2(a.ws2 + (size_t)f0 * Is, (uint32_t)((size_t)nf * Is * 2));
-    }
-    pdl_wait();
+    pdl_wait();  // h from fc1 (W2 was prefetched into L2 by fc1)
     const int nchI = I >> 3, nchS = Is >> 3;
+    // slots per batch: keep about 16 row chunks of W2 (and as many of h) in flight
+    constexpr int KB = VI <= 2 ? 8 : (VI <= 4 ? 4 : (VI <= 8 ? 2 : 1));
     const int items = T * nf;
     for (int item = warp; item < items; item += nw) {
         const int t = item / nf, f = f0 + (item - t * nf);
         float acc = 0.0f;
-        for (int k = 0; k < K; ++k) {
-            const int e = s_ids[t * K + k];
-            const bf16* row = a.w2 + ((size_t)e * H + f) * I;
-            const bf16* hr = a.h + (size_t)(k * T + t) * I;
-            float part = 0.0f;
+        for (int k0 = 0; k0 < K; k0 += KB) {
+            uint4 wv[KB][VI], hv[KB][VI];
 #pragma unroll
-            for (int j = 0; j < VI; ++j) {
-                const int c = lane + 32 * j;
-                if (c < nchI) part = dot8(ld_stream16(row + (size_t)c * 8), ld_nc16(hr + (size_t)c * 8), part);
+            for (int kb = 0; kb < KB; ++kb) {
+                const int k = k0 + kb;
+                const bf16* row = a.w2 + ((size_t)(k < K ? s_ids[t * K + k] : 0) * H + f) * I;
+                const bf16* hr = a.h + (size_t)((k < K ? k : 0) * T + t) * I;
+#pragma unroll
+                for (int j = 0; j < VI; ++j) {
+                    const int c = lane + 32 * j;
+                    if (k < K && c < nchI) {
+                        wv[kb][j] = ld_nc16(row + (size_t)c * 8);
+                        hv[kb][j] = ld_nc16(hr + (size_t)c * 8);
+                    }
+                }
             }
-            acc = fmaf(s_w[t * K + k], part, acc);
+#pragma unroll
+            for (int kb = 0; kb < KB; ++kb) {
+                const int k = k0 + kb;
+                if (k < K) {
+                    float part = 0.0f;
+#pragma unroll
+                    for (int j = 0; j < VI; ++j)
+                        if (lane + 32 * j < nchI) part = dot8(wv[kb][j], hv[kb][j], part);
+                    acc = fmaf(s_w[t * K + k], part, acc);
+                }
+            }
         }
         const float routed = warp_sum(acc);
         float ys = 0.0f;
@@ -224,7 +260,7 @@ __global__ void __launch_bounds__(256) fc2_small(const SmallArgs a) {
             const bf16* hr = a.hs + (size_t)t * Is;
             float part = 0.0f;
             for (int c = lane; c < nchS; c += 32)
-                part = dot8(ld_stream16(row + (size_t)c * 8), ld_nc16(hr + (size_t)c * 8), part);
+                part = dot8(ld_nc16(row + (size_t)c * 8), ld_nc16(hr + (size_t)c * 8), part);
             ys = warp_sum(part);
         }
         if (lane == 0) {
