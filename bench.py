@@ -36,6 +36,7 @@ sys.path.insert(0, ROOT)
 from mixture_experts_layer_35_b200 import inputs as gen  # noqa: E402
 
 L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2: written between timed steps
+METRIC = "fused MoE layer \u00b5s & tokens/s vs T=1..8192, % HBM/tensor roofline, 1\u00d7B200"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -144,6 +145,7 @@ def accounting(shape, T: int, U: int, router: bool, Is: int):
     k = {}
     k["router"] = {"bytes": E * H * 2 + T * H * 2 + T * E * 4, "flops": 2 * T * E * H}
     k["topk"] = {"bytes": T * E * 4 + T * K * 8, "flops": 0}
+    k["route"] = {"bytes": T * E * 4 + T * K * 8, "flops": 0}
     k["permute"] = {"bytes": T * K * 4 * 2, "flops": 0}
     k["fc1"] = {"bytes": U * rows1 * H * 2 + rows1s * H * 2 + T * H * 2 + h_bytes,
                 "flops": 2 * T * K * rows1 * H + 2 * T * rows1s * H}
@@ -158,7 +160,7 @@ def accounting(shape, T: int, U: int, router: bool, Is: int):
 
 def kernel_names(path: str, router: bool):
     names = ["router"] if router else []
-    return names + (["fc1", "fc2"] if path == "small" else ["topk", "permute", "fc1", "fc2", "finalize"])
+    return names + (["route", "fc1", "fc2"] if path == "small" else ["topk", "permute", "fc1", "fc2", "finalize"])
 
 
 def roofline_of(acc: dict, dur_s: float, peaks: dict):
@@ -298,7 +300,7 @@ def run_ours(args, rank, local, world):
     dist_init(world, "nccl")
     shape = gen.SHORT[args.config]
     peaks, peaks_src = load_peaks()
-    b = Bench(shape, args.T, device, seed=args.seed + rank, routing=args.routing)
+    b = Bench(shape, args.T, device, seed=args.seed + rank, routing=args.routing, path=args.path)
     per, clk = b.timed(args.steps, args.warmup, world, clocks=True)
     local_ms = float(sum(per))
     total_ms = max_over_ranks(local_ms, world, device)
@@ -323,7 +325,7 @@ def run_ours(args, rank, local, world):
     e2e_value = world * args.T * args.steps / (e2e_total / 1e3)
 
     line = {
-        "metric": "fused MoE layer tokens/s (one full layer forward per step)",
+        "metric": METRIC,
         "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic (seeded generator, random-init weights of the layer's shape)",
@@ -367,7 +369,7 @@ def sweep(args, device, peaks):
     for cfg, T in plan:
         shape = gen.SHORT[cfg]
         try:
-            b = Bench(shape, T, device, seed=1, routing="router")
+            b = Bench(shape, T, device, seed=1, routing="router", path=args.path)
             per, _ = b.timed(8, 2)
             med = statistics.median(per)
             U = b.distinct_experts()
@@ -406,7 +408,7 @@ def run_reference(args, rank, local, world):
             times.append(dt)
     tot = sum(times)
     value = sample * args.steps / tot
-    line = {"impl": "reference", "metric": "fused MoE layer tokens/s (one full layer forward per step)",
+    line = {"impl": "reference", "metric": METRIC,
             "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": tot / args.steps * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f64", "data": "synthetic (seeded generator)",
@@ -427,6 +429,8 @@ def main(argv=None):
     p.add_argument("--config", choices=sorted(gen.SHORT), default="qwen36")
     p.add_argument("--T", type=int, default=4096)
     p.add_argument("--routing", choices=["router", "zipf"], default="router")
+    p.add_argument("--path", choices=["auto", "small", "large"], default="auto",
+                   help="force an execution path (selector studies); auto = the library's choice")
     p.add_argument("--seed", type=int, default=0)
     p.add_argument("--no-sweep", action="store_true")
     p.add_argument("--sweep-all", action="store_true")

@@ -14,7 +14,7 @@ bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) 
 
 // Workspace carve-up of moe_fused_forward, 256-byte aligned regions after the header.
 struct WsLayout {
-    size_t logits, topk_w, topk_ids, offsets, tiles1, tiles2, counts, perm, h, hs, acc, ys, total;
+    size_t logits, route, topk_w, topk_ids, offsets, tiles1, tiles2, counts, perm, h, hs, acc, ys, total;
 };
 WsLayout layout(const moe_layer_desc* d) {
     const size_t T = (size_t)d->T, E = (size_t)d->E, K = (size_t)d->top_k, H = (size_t)d->H, I = (size_t)d->I,
@@ -27,6 +27,7 @@ WsLayout layout(const moe_layer_desc* d) {
         return r;
     };
     L.logits = take(T * E * 4);
+    L.route = take(sizeof(RouteTable));
     L.topk_w = take(T * K * 4);
     L.topk_ids = take(T * K * 4);
     L.offsets = take((E + 2) * 4);
@@ -212,7 +213,8 @@ moe_status_t moe_permute(const int32_t* topk_ids, int M, int K, int E, int32_t* 
     a.perm = perm;
     a.inv = inv;
     a.err = &static_cast<WsHeader*>(ws)->err;
-    a.bn = 128;
+    a.bn1 = kFc1TokenTile;
+    a.bn2 = kFc2TokenTile;
     if (launch_permute(a, (cudaStream_t)stream, false) != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_OK;
 }
@@ -230,7 +232,7 @@ int moe_select_path(const moe_layer_desc* d) {
 int moe_fused_forward_launches(const moe_layer_desc* d) {
     if (validate_desc(d) != MOE_OK || d->T == 0) return 0;
     const int router = d->router_logits ? 0 : 1;
-    if (resolve_path(d) == MOE_PATH_SMALL) return router + 2;
+    if (resolve_path(d) == MOE_PATH_SMALL) return router + 3;  // route table, fc1, fc2
     return router + 5;  // topk, permute, fc1, fc2, finalize
 }
 
@@ -274,7 +276,7 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
         float* lg = logits_out ? logits_out : reinterpret_cast<float*>(w8 + L.logits);
         if (!mark()) return MOE_ERR_CUDA;
         if (T <= 64 && router_small_supported(H)) {
-            MOE_CK(launch_router_small(x, static_cast<const bf16*>(d->router_w), T, H, E, lg, nullptr, s, false));
+            MOE_CK(launch_router_small(x, static_cast<const bf16*>(d->router_w), T, H, E, lg, nullptr, err, s, false));
         } else {
             st = run_router_dense(d, x, lg, nullptr, sms, s, err, false);
             if (st != MOE_OK) return st;
@@ -288,6 +290,10 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
     }
 
     if (path == MOE_PATH_SMALL) {
+        RouteTable* rt = reinterpret_cast<RouteTable*>(w8 + L.route);
+        if (!mark()) return MOE_ERR_CUDA;
+        MOE_CK(launch_route_small(logits, T, E, K, d->score, d->bias, d->renorm, rt, topk_w_out, topk_ids_out, s,
+                                  pdl && !timed));
         SmallArgs a;
         std::memset(&a, 0, sizeof(a));
         a.T = T;
@@ -299,20 +305,17 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
         a.score = d->score;
         a.renorm = d->renorm;
         a.Is = Is;
-        a.logits = logits;
-        a.bias = d->bias;
+        a.rt = rt;
         a.x = x;
         a.w13 = static_cast<const bf16*>(d->w13);
         a.w2 = static_cast<const bf16*>(d->w2);
         a.ws13 = static_cast<const bf16*>(d->ws13);
         a.ws2 = static_cast<const bf16*>(d->ws2);
-        a.w_out = topk_w_out;
-        a.id_out = topk_ids_out;
         a.h = reinterpret_cast<bf16*>(w8 + L.h);
         a.hs = reinterpret_cast<bf16*>(w8 + L.hs);
         a.out = out;
         const std::function<bool()> mark_fn = mark;
-        MOE_CK(launch_small(a, sms, s, pdl, timed ? &mark_fn : nullptr));
+        MOE_CK(launch_small(a, sms, s, true, timed ? &mark_fn : nullptr));
         if (!mark()) return MOE_ERR_CUDA;
         return MOE_OK;
     }
@@ -350,7 +353,8 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
     pa.perm = perm;
     pa.err = err;
     pa.has_shared = Is > 0;
-    pa.bn = 128;
+    pa.bn1 = kFc1TokenTile;
+    pa.bn2 = kFc2TokenTile;
     pa.nfeat1_r = cdiv(I, 128);
     pa.nfeat1_s = cdiv(Is, 128);
     pa.nfeat2_r = cdiv(H, 128);

@@ -14,7 +14,7 @@
 //   FC2: A = W2[e] rows of 128 output features, B = the expert's contiguous h rows
 //       (TMA, 16-row boxes); epilogue scales by the routing weight, stages the block in
 //       shared memory and adds it into the FP32 accumulator acc[t, :] with asynchronous
-//       bulk reduce-adds, one 128-byte row segment per token ("weighted output
+//       bulk reduce-adds, one 512-byte row (128 features) per token ("weighted output
 //       combination").
 //       The shared expert is one more group whose FC2 output is rounded to BF16 into ys.
 //   DENSE: router logits, A = Wr (128 experts per tile), B = x rows (TMA).
@@ -23,7 +23,8 @@
 //   warp 0      TMA producer (weights; FC2/DENSE token rows)
 //   warp 1      TMEM allocator and single-thread MMA issuer
 //   warps 2-5   epilogue: tcgen05.ld of the accumulator (warp w reads TMEM lanes of
-//               quarter w % 4), activation / scaling, stores
+//               quarter w % 4), activation / scaling, stores; FC2 has eight epilogue
+//               warps (2-9), the second four taking the odd 32-token column chunks
 //   warps 6-9   FC1 only: cp.async gather of token rows of x
 // Shared memory holds a ring of stages (full/empty mbarriers); TMEM holds two
 // accumulator buffers so the epilogue of one tile overlaps the mainloop of the next.
@@ -32,9 +33,8 @@
 namespace moe {
 namespace {
 
-constexpr int BM = 128, BN = 128, BK = 64;
+constexpr int BM = 128, BK = 64;
 constexpr int A_BYTES = BM * BK * 2;  // 16 KB
-constexpr int B_BYTES = BN * BK * 2;  // 16 KB
 constexpr int BBOX = 16;              // token rows per TMA box of the B operand
 
 template <int MODE>
@@ -42,14 +42,22 @@ struct Cfg {
     static constexpr bool kGather = (MODE == GM_FC1_SWIGLU || MODE == GM_FC1_RELU2);
     static constexpr bool kSwiglu = (MODE == GM_FC1_SWIGLU);
     static constexpr int kNA = kSwiglu ? 2 : 1;
-    static constexpr int kStageBytes = kNA * A_BYTES + B_BYTES;
-    static constexpr int kStages = kSwiglu ? 4 : (MODE == GM_FC2 ? 5 : 6);
-    // FC2: per epilogue warp, two [32 tokens][32 features] FP32 staging blocks for the
-    // bulk reduce-add into acc.
-    static constexpr int kEpiBytes = (MODE == GM_FC2) ? 4 * 2 * 32 * 32 * 4 : 0;
-    static constexpr int kAccCols = kSwiglu ? 2 * BN : BN;
-    static constexpr int kTmemCols = kSwiglu ? 512 : 256;
-    static constexpr int kThreads = kGather ? 320 : 192;
+    // Token rows per tile (MMA N): FC2 takes up to 256 so that an expert's W2 tile is
+    // streamed once for all its tokens at prefill sizes; FC1 keeps 128 so that its gate
+    // and up accumulators stay double-buffered in TMEM.
+    static constexpr int kBN = (MODE == GM_FC2) ? 256 : 128;
+    static constexpr int kBBytes = kBN * BK * 2;
+    static constexpr int kStageBytes = kNA * A_BYTES + kBBytes;
+    static constexpr int kStages = kSwiglu ? 4 : (MODE == GM_FC2 ? 3 : 6);
+    // Epilogue warps: FC2's epilogue (staging + bulk reduce) is heavier than its short
+    // mainloop, so it gets two warps per TMEM lane quarter, splitting the token columns.
+    static constexpr int kEpiWarps = (MODE == GM_FC2) ? 8 : 4;
+    // FC2: per half of the epilogue warps, two [32 tokens][128 features] FP32 staging
+    // blocks for the bulk reduce-add into acc.
+    static constexpr int kEpiBytes = (MODE == GM_FC2) ? 2 * 2 * 32 * 128 * 4 : 0;
+    static constexpr int kAccCols = kSwiglu ? 2 * kBN : kBN;
+    static constexpr int kTmemCols = (2 * kAccCols) >= 512 ? 512 : 256;
+    static constexpr int kThreads = 64 + 32 * kEpiWarps + (kGather ? 128 : 0);
     static constexpr int kLag = 2;
     static constexpr int kMaxGroups = MOE_MAX_EXPERTS + 1;
     // dynamic smem: alignment slack, stages, barriers, flags, tile and offset tables
@@ -61,6 +69,7 @@ struct TileInfo {
     int g, ft, n, row0, shared;
 };
 
+template <int BN>
 __device__ __forceinline__ TileInfo decode_tile(const GemmArgs& a, const int* s_tiles, const int* s_offs, int G,
                                                 int tile) {
     TileInfo ti;
@@ -126,7 +135,7 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(tfull_bar(b), 1);
-            mbar_init(tempty_bar(b), 4);
+            mbar_init(tempty_bar(b), C::kEpiWarps);
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -152,13 +161,18 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     const int total = a.dense ? a.nfeat_r * cdiv(a.T, kDenseTokenTile) : s_tiles[G];
+    // Tiles are dealt round-robin over the persistent CTAs: at any moment the CTAs work on
+    // neighbouring tiles of the group-major list (one expert's feature and token tiles),
+    // which share that expert's weight rows and token rows in L2, and tiles of unequal
+    // cost (ragged token tails) spread evenly.
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
+            const uint64_t wpol = l2_policy_evict_first();
             int it = 0;
             for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
-                const TileInfo ti = decode_tile(a, s_tiles, s_offs, G, tile);
+                const TileInfo ti = decode_tile<C::kBN>(a, s_tiles, s_offs, G, tile);
                 const bool sh = ti.shared;
                 const CUtensorMap* ta = sh ? &tm_a_s : &tm_a_r;
                 const CUtensorMap* tb = sh ? &tm_b_s : &tm_b_r;
@@ -176,6 +190,8 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
                     if (sh || a.dense) {
                         tma_load_2d(st, ta, full_bar(s), kb * BK, frow);
                         if (C::kSwiglu) tma_load_2d(st + A_BYTES, ta, full_bar(s), kb * BK, a.up_s + frow);
+                    } else if (MODE == GM_FC2) {  // weights streamed once: evict first
+                        tma_load_3d_hint(st, ta, full_bar(s), kb * BK, frow, ti.g, wpol);
                     } else {
                         tma_load_3d(st, ta, full_bar(s), kb * BK, frow, ti.g);
                         if (C::kSwiglu) tma_load_3d(st + A_BYTES, ta, full_bar(s), kb * BK, a.up_r + frow, ti.g);
@@ -194,7 +210,7 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
         if (lane == 0) {
             int it = 0, tcount = 0;
             for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x, ++tcount) {
-                const TileInfo ti = decode_tile(a, s_tiles, s_offs, G, tile);
+                const TileInfo ti = decode_tile<C::kBN>(a, s_tiles, s_offs, G, tile);
                 const int kd = ti.shared ? a.kdim_s : a.kdim;
                 const int nk = cdiv(kd, BK);
                 const int npad = cdiv(ti.n, 16) * 16;
@@ -204,7 +220,7 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
                 if (!mbar_wait(tempty_bar(buf), tph ^ 1u, abort_flag, a.err)) break;
                 tc_fence_after();
                 const uint32_t d0 = tmem_base + (uint32_t)(buf * C::kAccCols);
-                const uint32_t d1 = d0 + BN;
+                const uint32_t d1 = d0 + C::kBN;
                 bool ok = true;
                 for (int kb = 0; kb < nk; ++kb, ++it) {
                     const int s = it % C::kStages;
@@ -229,33 +245,64 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
                 tc_commit(tfull_bar(buf));
             }
         }
-    } else if (warp < 6) {
+    } else if (warp < 2 + C::kEpiWarps) {
         // ------------------------------------------------------------ epilogue
-        const int q = warp & 3;
-        const int et = threadIdx.x - 64;  // 0..127
+        const int q = warp & 3;                     // TMEM lane quarter of this warp
+        const int half = (warp - 2) >> 2;          // FC2: which token columns (chunk parity)
+        const int nhalf = C::kEpiWarps / 4;
+        const int et = threadIdx.x - 64;
         if (a.zero_ptr) {
             float4* z = reinterpret_cast<float4*>(a.zero_ptr);
             const size_t n4 = a.zero_n / 4;
-            for (size_t i = (size_t)blockIdx.x * 128 + et; i < n4; i += (size_t)gridDim.x * 128)
+            const int ne = 32 * C::kEpiWarps;
+            for (size_t i = (size_t)blockIdx.x * ne + et; i < n4; i += (size_t)gridDim.x * ne)
                 z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
         int tcount = 0;
         int ebuf = 0;
-        for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x, ++tcount) {
-            const TileInfo ti = decode_tile(a, s_tiles, s_offs, G, tile);
+        // (the abort flag is checked through the per-tile wait and vote below, so that the
+        // epilogue warps always take the same number of tiles)
+        constexpr int kChunks = C::kBN / (32 * (C::kEpiWarps / 4));
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++tcount) {
+            const TileInfo ti = decode_tile<C::kBN>(a, s_tiles, s_offs, G, tile);
             const int buf = tcount & 1;
             const uint32_t tph = (uint32_t)(tcount >> 1) & 1u;
-            if (!mbar_wait(tfull_bar(buf), tph, abort_flag, a.err)) break;
+            // FC2: token and routing weight of each column this thread will scale, loaded
+            // before the accumulator is ready (hidden behind the tile's mainloop).
+            int mt[kChunks];
+            float mw[kChunks];
+#pragma unroll
+            for (int ci = 0; ci < kChunks; ++ci) {
+                mt[ci] = 0;
+                mw[ci] = 0.0f;
+                const int colm = 32 * half + 32 * nhalf * ci + lane;
+                if (MODE == GM_FC2 && !ti.shared && colm < ti.n) {
+                    const int src = a.perm[ti.row0 + colm];
+                    const int kk = src / a.T;
+                    mt[ci] = src - kk * a.T;
+                    mw[ci] = a.topk_w[(size_t)mt[ci] * a.K + kk];
+                }
+            }
+            const bool waited = mbar_wait(tfull_bar(buf), tph, abort_flag, a.err);
+            if (MODE == GM_FC2) {
+                // the FC2 epilogue warps meet at named barriers below: leave together or not at all
+                if (named_barrier_or(1 + half, 128, !waited || *abort_flag)) break;
+            } else if (!waited) {
+                break;
+            }
             tc_fence_after();
             const int f = ti.ft * BM + q * 32 + lane;
             const int feat = ti.shared ? a.feat_s : a.feat_r;
             const bool fok = f < feat;
             const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * C::kAccCols);
-            for (int c0 = 0; c0 < ti.n; c0 += 32) {
+#pragma unroll
+            for (int ci = 0; ci < kChunks; ++ci) {
+                const int c0 = 32 * half + 32 * nhalf * ci;
+                if (c0 >= ti.n) break;
                 uint32_t v[32];
                 tmem_ld32(tb + c0, v);
                 uint32_t u[32];
-                if (C::kSwiglu) tmem_ld32(tb + BN + c0, u);
+                if (C::kSwiglu) tmem_ld32(tb + C::kBN + c0, u);
                 tmem_ld_wait();
                 if (C::kGather) {
                     bf16* dst = ti.shared ? a.hs : a.h;
@@ -280,33 +327,27 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
                         }
                     } else {
                         // Column j of this chunk is token t_j with routing weight w_j.  The
-                        // warp stages w_j * y[f, j] as rows [j][32 features] in shared memory,
-                        // then lane j reduce-adds row j into acc[t_j, f0 .. f0+31] with one
-                        // asynchronous bulk reduction (FP32 add in L2).
-                        int my_t = 0;
-                        float my_w = 0.0f;
-                        const int colm = c0 + lane;
-                        if (colm < ti.n) {
-                            const int src = a.perm[ti.row0 + colm];
-                            const int kk = src / a.T;
-                            my_t = src - kk * a.T;
-                            my_w = a.topk_w[(size_t)my_t * a.K + kk];
-                        }
-                        float* stg = epi_stage + (size_t)(q * 2 + ebuf) * 32 * 32;
-                        bulk_wait_read<1>();  // the reads of this buffer's previous use are done
-                        __syncwarp();
+                        // four epilogue warps of this half stage w_j * y[f, j] as rows
+                        // [j][128 features] in shared memory; then one thread per row
+                        // reduce-adds the whole 512-byte row into acc[t_j, f0 .. f0+127] with
+                        // one asynchronous bulk reduction (FP32 add in L2).
+                        float* stg = epi_stage + (size_t)(half * 2 + ebuf) * 32 * 128;
+                        bulk_wait_read<1>();           // my reduces from this buffer's last use have read it
+                        named_barrier(1 + half, 128);  // ... and everybody else's
 #pragma unroll
                         for (int j = 0; j < 32; ++j) {
-                            const float w = __shfl_sync(0xffffffffu, my_w, j);
-                            stg[j * 32 + lane] = w * __uint_as_float(v[j]);
+                            const float w = __shfl_sync(0xffffffffu, mw[ci], j);
+                            stg[j * 128 + q * 32 + lane] = w * __uint_as_float(v[j]);
                         }
                         fence_proxy_async_smem();
-                        __syncwarp();
-                        const int fbase = ti.ft * BM + q * 32;
-                        const int nf = min(32, a.feat_r - fbase);
-                        if (colm < ti.n && nf > 0)
-                            bulk_reduce_add_f32(a.acc + (size_t)my_t * a.feat_r + fbase, smem_u32(stg + lane * 32),
-                                                (uint32_t)nf * 4u);
+                        named_barrier(1 + half, 128);
+                        const int r = q * 8 + (lane & 7);  // row issued by this thread
+                        const int t_r = __shfl_sync(0xffffffffu, mt[ci], r);
+                        const int fb = ti.ft * BM;
+                        const int nfe = min(BM, a.feat_r - fb);
+                        if (lane < 8 && c0 + r < ti.n && nfe > 0)
+                            bulk_reduce_add_f32(a.acc + (size_t)t_r * a.feat_r + fb, smem_u32(stg + r * 128),
+                                                (uint32_t)nfe * 4u);
                         bulk_commit();
                         ebuf ^= 1;
                     }
@@ -333,7 +374,7 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
         const int chunk = p & 7, rsub = p >> 3;
         int it = 0;
         for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
-            const TileInfo ti = decode_tile(a, s_tiles, s_offs, G, tile);
+            const TileInfo ti = decode_tile<C::kBN>(a, s_tiles, s_offs, G, tile);
             const int kd = ti.shared ? a.kdim_s : a.kdim;
             const int nk = cdiv(kd, BK);
             const int npad = cdiv(ti.n, 16) * 16;

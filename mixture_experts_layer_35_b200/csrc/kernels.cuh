@@ -40,28 +40,40 @@ cudaError_t launch_topk(const void* logits, bool bf16_in, int M, int E, int K, i
                         int* counts = nullptr);
 bool router_small_supported(int H);
 cudaError_t launch_router_small(const bf16* x, const bf16* wr, int T, int H, int E, float* logits,
-                                float* logits_copy, cudaStream_t s, bool pdl);
+                                float* logits_copy, int* err, cudaStream_t s, bool pdl);
 
 // ---------------------------------------------------------------- few-token path
 static constexpr int kSmallMaxT = 16;
+static constexpr int kSmallMaxSlots = kSmallMaxT * MOE_MAX_TOPK;
+// Routing of the few-token path, built once by route_small_kernel: the distinct experts
+// in ascending order (ulist), and for each the slots k*T + t it serves
+// (utok[uoff[u] .. uoff[u+1])), plus every slot's expert and weight (index t*K + k).
+struct RouteTable {
+    int U;
+    int pad[31];
+    int ulist[kSmallMaxSlots];
+    int uoff[kSmallMaxSlots + 1];
+    int utok[kSmallMaxSlots];
+    int ids[kSmallMaxSlots];
+    float w[kSmallMaxSlots];
+};
+cudaError_t launch_route_small(const float* logits, int T, int E, int K, int score, const float* bias, int renorm,
+                               RouteTable* rt, float* w_out, int32_t* id_out, cudaStream_t s, bool pdl);
 struct SmallArgs {
     int T, H, I, E, K, act, score, renorm, Is;
-    const float* logits;  // [T, E]
-    const float* bias;    // [E] or null
+    const RouteTable* rt;
     const bf16* x;
     const bf16* w13;
     const bf16* w2;
     const bf16* ws13;
     const bf16* ws2;
-    float* w_out;      // [T, K] caller output or null
-    int32_t* id_out;   // [T, K] caller output or null
     bf16* h;           // [T*K, I], row = slot k*T + t
     bf16* hs;          // [T, Is]
     bf16* out;         // [T, H]
 };
 bool small_path_supported(int T, int H, int I, int Is);
-// `mark` (optional) records a timing event before each of the two kernels; when it is
-// given the kernels are launched without programmatic overlap.
+// `mark` (optional) records a timing event before each of the two streaming kernels;
+// when it is given the kernels are launched without programmatic overlap.
 cudaError_t launch_small(const SmallArgs& a, int num_sms, cudaStream_t s, bool pdl_first,
                          const std::function<bool()>* mark);
 
@@ -77,7 +89,7 @@ struct PermuteArgs {
     int* err;
     // grouped-GEMM tile tables (null when not wanted)
     int has_shared;      // adds group E with M rows
-    int bn;              // token rows per tile
+    int bn1, bn2;        // token rows per tile of the FC1 / FC2 GEMMs
     int nfeat1_r, nfeat1_s, nfeat2_r, nfeat2_s;
     int32_t* tiles1;     // [G + 1] exclusive prefix of FC1 tiles over groups
     int32_t* tiles2;     // [G + 1] exclusive prefix of FC2 tiles over groups
@@ -92,8 +104,10 @@ cudaError_t launch_permute_fast(const PermuteArgs& a, const int* counts, int* cu
 // ---------------------------------------------------------------- grouped tcgen05 GEMM
 enum GemmMode { GM_FC1_SWIGLU = 0, GM_FC1_RELU2 = 1, GM_FC2 = 2, GM_DENSE = 3 };
 // Token rows per tile of the dense router GEMM (E is small, so smaller token tiles give
-// the grid more CTAs).
+// the grid more CTAs), and of the grouped FC1 / FC2 GEMMs.
 static constexpr int kDenseTokenTile = 64;
+static constexpr int kFc1TokenTile = 128;
+static constexpr int kFc2TokenTile = 256;
 struct GemmArgs {
     int T, K;            // tokens and top-k (slot decode of perm entries)
     int kdim;            // reduction length (H for FC1 / router, I or I_s for FC2)

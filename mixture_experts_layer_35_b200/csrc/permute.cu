@@ -113,11 +113,10 @@ __device__ void write_tile_tables(const PermuteArgs& a, int my_cnt, int* s_warp)
     const int tid = threadIdx.x, E = a.E, M = a.M;
     const int G = E + (a.has_shared ? 1 : 0);
     const int rows = (tid < E) ? my_cnt : (tid == E && a.has_shared ? M : 0);
-    const int ntok = cdiv(rows, a.bn);
     const bool sh = tid == E;
     int tot1, tot2;
-    const int p1 = block_exclusive_scan(tid < G ? ntok * (sh ? a.nfeat1_s : a.nfeat1_r) : 0, s_warp, tot1);
-    const int p2 = block_exclusive_scan(tid < G ? ntok * (sh ? a.nfeat2_s : a.nfeat2_r) : 0, s_warp, tot2);
+    const int p1 = block_exclusive_scan(tid < G ? cdiv(rows, a.bn1) * (sh ? a.nfeat1_s : a.nfeat1_r) : 0, s_warp, tot1);
+    const int p2 = block_exclusive_scan(tid < G ? cdiv(rows, a.bn2) * (sh ? a.nfeat2_s : a.nfeat2_r) : 0, s_warp, tot2);
     if (tid < G) {
         a.tiles1[tid] = p1;
         a.tiles2[tid] = p2;

@@ -1,74 +1,27 @@
-// router.cu -- router logits for few tokens (weight streaming) and the warp-per-row
-// router top-k kernel behind moe_router_topk and the large-token path.
+// router.cu -- router logits for few tokens, the warp-per-row router top-k (moe_router_topk
+// and the many-token path), and the route table of the few-token path.
 #include "kernels.cuh"
 #include "router.cuh"
 
 namespace moe {
 
-// ---------------------------------------------------------------- top-k, one warp per row
-// With `refine` (logits from the tensor-core router, FP32 accumulation in the MMA's own
-// order): a first selection on those logits; then every expert whose key lies within
-// `kRefineWindow` (relative) of the K-th key -- the selected ones included -- gets its
-// logit recomputed as an FP64 dot product rounded once to FP32, written back, and the
-// selection and weights are redone.  An expert outside the window cannot enter the top
-// K as long as the tensor-core logit error stays below half the window (it is ~1e-6
-// absolute on these workloads against a window of 2e-3), so ids and weights follow the
-// correctly rounded logits.
-static constexpr float kRefineWindow = 2e-3f;
+// Tensor-core router logits carry an FP32 accumulation error of ~1e-6 on these
+// workloads; the routing window assumes at most this (two orders of magnitude above).
+static constexpr float kTcLogitErr = 2e-4f;
 
-template <int V>
-__device__ __forceinline__ void refine_row(float (&l)[V], int row, int E, int K, int score, const float* bias,
-                                           int renorm, int lane, const bf16* x, const bf16* wr, int H,
-                                           float* logits_rw) {
-    int id;
-    float w, lg;
-    warp_topk_row<V>(l, E, K, score, bias, renorm, lane, id, w, lg);
-    // K-th key of the first selection
-    const int idK = __shfl_sync(0xffffffffu, id, K - 1);
-    const float lK = __shfl_sync(0xffffffffu, lg, K - 1);
-    float kK = (score == MOE_SCORE_SIGMOID) ? sigmoid_f32_rn(lK) : lK;
-    if (bias) kK = __fadd_rn(kK, bias[idK]);
-    const float win = kRefineWindow * fmaxf(1.0f, fabsf(kK)) * (score == MOE_SCORE_SIGMOID ? 0.25f : 1.0f);
-    const bf16* xr = x + (size_t)row * H;
-    const int nch = H >> 3;
-#pragma unroll
-    for (int c = 0; c < V; ++c) {
-        const int e = lane + 32 * c;
-        bool cand = false;
-        if (e < E) {
-            float k = (score == MOE_SCORE_SIGMOID) ? sigmoid_f32_rn(l[c]) : l[c];
-            if (bias) k = __fadd_rn(k, bias[e]);
-            cand = !(k < kK - win);  // also true for NaN
-        }
-        unsigned m = __ballot_sync(0xffffffffu, cand);
-        while (m) {
-            const int src = __ffs(m) - 1;
-            m &= m - 1;
-            const int ee = src + 32 * c;
-            const bf16* wrow = wr + (size_t)ee * H;
-            // four independent partial sums keep four 16-byte chunks of the row in flight
-            double acc0 = 0.0, acc1 = 0.0, acc2 = 0.0, acc3 = 0.0;
-            int q = lane;
-            for (; q + 96 < nch; q += 128) {
-                const uint4 w0 = ld_nc16(wrow + (size_t)q * 8), w1 = ld_nc16(wrow + (size_t)(q + 32) * 8);
-                const uint4 w2 = ld_nc16(wrow + (size_t)(q + 64) * 8), w3 = ld_nc16(wrow + (size_t)(q + 96) * 8);
-                const uint4 x0 = ld_nc16(xr + (size_t)q * 8), x1 = ld_nc16(xr + (size_t)(q + 32) * 8);
-                const uint4 x2 = ld_nc16(xr + (size_t)(q + 64) * 8), x3 = ld_nc16(xr + (size_t)(q + 96) * 8);
-                acc0 = dot8_f64(x0, w0, acc0);
-                acc1 = dot8_f64(x1, w1, acc1);
-                acc2 = dot8_f64(x2, w2, acc2);
-                acc3 = dot8_f64(x3, w3, acc3);
-            }
-            for (; q < nch; q += 32) acc0 = dot8_f64(ld_nc16(xr + (size_t)q * 8), ld_nc16(wrow + (size_t)q * 8), acc0);
-            const float exact = __double2float_rn(warp_sum_f64((acc0 + acc1) + (acc2 + acc3)));
-            if (lane == src) {
-                l[c] = exact;
-                if (logits_rw) logits_rw[(size_t)row * E + ee] = exact;
-            }
-        }
+struct RowRefine {
+    const bf16* xr;
+    const bf16* wr;
+    int H, E, row, lane;
+    float* logits_rw;
+    __device__ float operator()(int e) const {
+        const float v = warp_dot_exact(xr, wr + (size_t)e * H, H, lane);
+        if (logits_rw && lane == 0) logits_rw[(size_t)row * E + e] = v;
+        return v;
     }
-}
+};
 
+// ---------------------------------------------------------------- top-k, one warp per row
 template <int V, bool BF16_IN, bool REFINE>
 __global__ void __launch_bounds__(256) topk_kernel(const void* __restrict__ logits, int M, int E, int K, int score,
                                                    const float* __restrict__ bias, int renorm,
@@ -86,10 +39,14 @@ __global__ void __launch_bounds__(256) topk_kernel(const void* __restrict__ logi
             load_row_bf16<V>(static_cast<const uint16_t*>(logits) + (size_t)row * E, E, lane, l);
         else
             load_row_f32<V>(static_cast<const float*>(logits) + (size_t)row * E, E, lane, l);
-        if (REFINE) refine_row<V>(l, row, E, K, score, bias, renorm, lane, x, wr, H, logits_rw);
         int id;
         float w, lg;
-        warp_topk_row<V>(l, E, K, score, bias, renorm, lane, id, w, lg);
+        if (REFINE) {
+            const RowRefine rf{x + (size_t)row * H, wr, H, E, row, lane, logits_rw};
+            warp_route_row<V>(l, E, K, score, bias, renorm, lane, kTcLogitErr, rf, id, w, lg);
+        } else {
+            warp_route_row<V>(l, E, K, score, bias, renorm, lane, 0.0f, NoRefine{}, id, w, lg);
+        }
         if (lane < K) {
             const size_t o = (size_t)row * K + lane;
             topk_w[o] = w;
@@ -129,48 +86,87 @@ cudaError_t launch_topk(const void* logits, bool bf16_in, int M, int E, int K, i
 }
 
 // ---------------------------------------------------------------- router logits, few tokens
-// l[t, e] = x[t,:] . Wr[e,:].  One warp per expert row: the lanes stream the row in
-// 16-byte chunks once (HBM), and dot each chunk with the matching chunk of every token
-// (x is tiny and stays in L1/L2).  The accumulation is FP64 (BF16 products are exact in
-// double), so the FP32 logit is the correctly rounded dot product except when the exact
-// value lies within ~1e-16 of an FP32 rounding boundary.
-template <int VH, int TT>
-__global__ void __launch_bounds__(128) router_logits_small(const bf16* __restrict__ x, const bf16* __restrict__ wr,
-                                                           int T, int H, int E, float* __restrict__ logits,
-                                                           float* __restrict__ logits_copy) {
-    pdl_wait();
-    const int lane = threadIdx.x & 31;
-    const int e = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    if (e < E) {
-        const int nch = H >> 3;  // 16-byte chunks per row
-        const bf16* wrow = wr + (size_t)e * H;
-        uint4 w[VH];  // the whole row is loaded at once: one memory latency per row
+// l[t, e] = x[t,:] . Wr[e,:], correctly rounded (Sum2 error-free accumulation of the exact
+// BF16 products).  Two warps per CTA, one expert row per warp held in registers (one
+// memory latency per row); the tokens, 16 at a time, are staged in shared memory; each
+// warp runs four independent Sum2 chains (two tokens x even/odd chunks).
+static constexpr int kRouterTokBlock = 16;
+
+template <int VH>
+__global__ void __launch_bounds__(64) router_logits_small(const bf16* __restrict__ x, const bf16* __restrict__ wr,
+                                                          int T, int H, int E, float* __restrict__ logits,
+                                                          float* __restrict__ logits_copy, int* err) {
+    extern __shared__ uint4 xs[];  // [kRouterTokBlock][H / 8]
+    __shared__ __align__(8) uint64_t s_bar;
+    __shared__ int s_abort;
+    const int tid = threadIdx.x, lane = tid & 31;
+    const uint32_t bar = smem_u32(&s_bar);
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        s_abort = 0;
+        fence_mbar_init();
+    }
+    const int e = blockIdx.x * (blockDim.x >> 5) + (tid >> 5);
+    const int nch = H >> 3;
+    uint4 w[VH];
 #pragma unroll
-        for (int j = 0; j < VH; ++j) {
-            const int c = lane + 32 * j;
-            w[j] = (c < nch) ? ld_stream16(wrow + (size_t)c * 8) : make_uint4(0u, 0u, 0u, 0u);
+    for (int j = 0; j < VH; ++j) {
+        const int c = lane + 32 * j;
+        w[j] = (e < E && c < nch) ? ld_stream16(wr + (size_t)e * H + (size_t)c * 8) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    pdl_wait();  // x may come from the previous kernel
+    uint32_t phase = 0;
+    for (int t0 = 0; t0 < T; t0 += kRouterTokBlock) {
+        const int nt = min(kRouterTokBlock, T - t0);
+        __syncthreads();  // every warp is done with the previous block (and sees the barrier init)
+        if (tid == 0) {   // the token block in one bulk copy (rows are 16-byte multiples)
+            const uint32_t bytes = (uint32_t)nt * H * 2;
+            fence_proxy_async_smem();
+            mbar_expect_tx(bar, bytes);
+            bulk_copy_g2s(smem_u32(xs), x + (size_t)t0 * H, bytes, bar);
         }
-        for (int t0 = 0; t0 < T; t0 += TT) {
-            double acc[TT];
-#pragma unroll
-            for (int i = 0; i < TT; ++i) acc[i] = 0.0;
+        const bool ok = mbar_wait(bar, phase, &s_abort, err);
+        phase ^= 1u;
+        if (__syncthreads_or(!ok)) break;  // a wait that gave up ends every warp together
+        if (e >= E) continue;
+        for (int t = 0; t < nt; t += 2) {
+            const bool two = t + 1 < nt;
+            Sum2 a0 = {0.f, 0.f}, a1 = {0.f, 0.f}, b0 = {0.f, 0.f}, b1 = {0.f, 0.f};
 #pragma unroll
             for (int j = 0; j < VH; ++j) {
                 const int c = lane + 32 * j;
                 if (c < nch) {
-#pragma unroll
-                    for (int i = 0; i < TT; ++i)
-                        if (t0 + i < T) acc[i] = dot8_f64(w[j], ld_nc16(x + (size_t)(t0 + i) * H + (size_t)c * 8), acc[i]);
+                    const uint4 xa = xs[t * nch + c];
+                    if (j & 1) sum2_dot8(a1, xa, w[j]);
+                    else sum2_dot8(a0, xa, w[j]);
+                    if (two) {
+                        const uint4 xb = xs[(t + 1) * nch + c];
+                        if (j & 1) sum2_dot8(b1, xb, w[j]);
+                        else sum2_dot8(b0, xb, w[j]);
+                    }
                 }
             }
-#pragma unroll
-            for (int i = 0; i < TT; ++i) {
-                const float v = __double2float_rn(warp_sum_f64(acc[i]));
-                if (lane == 0 && t0 + i < T) {
-                    logits[(size_t)(t0 + i) * E + e] = v;
-                    if (logits_copy) logits_copy[(size_t)(t0 + i) * E + e] = v;
+            float q;
+            two_sum(a0.s, a1.s, a0.s, q);
+            a0.c = __fadd_rn(__fadd_rn(a0.c, a1.c), q);
+            two_sum(b0.s, b1.s, b0.s, q);
+            b0.c = __fadd_rn(__fadd_rn(b0.c, b1.c), q);
+            const float va = sum2_warp_finish(a0);
+            const float vb = sum2_warp_finish(b0);
+            if (lane == 0) {
+                logits[(size_t)(t0 + t) * E + e] = va;
+                if (logits_copy) logits_copy[(size_t)(t0 + t) * E + e] = va;
+                if (two) {
+                    logits[(size_t)(t0 + t + 1) * E + e] = vb;
+                    if (logits_copy) logits_copy[(size_t)(t0 + t + 1) * E + e] = vb;
                 }
             }
+        }
+    }
+    __syncthreads();
+    if (s_abort) {  // a wait gave up: let the bulk copy in flight land before the CTA retires
+        const uint64_t t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 50000ull) {
         }
     }
     pdl_trigger();
@@ -179,19 +175,126 @@ __global__ void __launch_bounds__(128) router_logits_small(const bf16* __restric
 bool router_small_supported(int H) { return (H >> 3) <= 32 * 16; }
 
 cudaError_t launch_router_small(const bf16* x, const bf16* wr, int T, int H, int E, float* logits,
-                                float* logits_copy, cudaStream_t s, bool pdl) {
-    dim3 grid(cdiv(E, 4)), block(128);
+                                float* logits_copy, int* err, cudaStream_t s, bool pdl) {
+    dim3 grid(cdiv(E, 2)), block(64);
+    const size_t smem = (size_t)kRouterTokBlock * H * 2;
     const int need = cdiv(H >> 3, 32);
-#define MOE_R(VV)                                                                                               \
-    if (need <= VV) {                                                                                           \
-        if (T <= 2)                                                                                             \
-            return launch_k(router_logits_small<VV, 2>, grid, block, 0, s, pdl, x, wr, T, H, E, logits, logits_copy); \
-        if (T <= 4)                                                                                             \
-            return launch_k(router_logits_small<VV, 4>, grid, block, 0, s, pdl, x, wr, T, H, E, logits, logits_copy); \
-        return launch_k(router_logits_small<VV, 8>, grid, block, 0, s, pdl, x, wr, T, H, E, logits, logits_copy);     \
+#define MOE_R(VV)                                                                                                \
+    if (need <= VV) {                                                                                            \
+        cudaError_t st = cudaFuncSetAttribute(router_logits_small<VV>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                                               (int)smem);                                                       \
+        if (st != cudaSuccess) return st;                                                                        \
+        return launch_k(router_logits_small<VV>, grid, block, smem, s, pdl, x, wr, T, H, E, logits, logits_copy, err); \
     }
     MOE_R(4) MOE_R(8) MOE_R(12) MOE_R(16)
 #undef MOE_R
+    return cudaErrorInvalidValue;
+}
+
+// ---------------------------------------------------------------- route table, few tokens
+// One CTA, one warp per token row: route each row, then list the distinct experts in
+// ascending order with the slots (k*T + t) each one serves, for the streaming kernels.
+// Everything is built in shared memory and written out once.
+template <int V>
+__global__ void __launch_bounds__(32 * kSmallMaxT) route_small_kernel(const float* __restrict__ logits, int T, int E,
+                                                                      int K, int score, const float* __restrict__ bias,
+                                                                      int renorm, RouteTable* __restrict__ rt,
+                                                                      float* __restrict__ w_out,
+                                                                      int32_t* __restrict__ id_out) {
+    __shared__ int s_ids[kSmallMaxSlots];
+    __shared__ int s_uidx[MOE_MAX_EXPERTS];
+    __shared__ int s_ulist[kSmallMaxSlots];
+    __shared__ int s_uoff[kSmallMaxSlots + 1];
+    __shared__ int s_wcnt[32], s_wbase[32];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+    const int TK = T * K;
+    for (int e = tid; e < E; e += blockDim.x) s_uidx[e] = 0;
+    pdl_wait();
+    for (int t = warp; t < T; t += nw) {
+        float l[V];
+        load_row_f32<V>(logits + (size_t)t * E, E, lane, l);
+        int id;
+        float w, lg;
+        warp_route_row<V>(l, E, K, score, bias, renorm, lane, 0.0f, NoRefine{}, id, w, lg);
+        if (lane < K) {
+            s_ids[t * K + lane] = id;
+            rt->ids[t * K + lane] = id;
+            rt->w[t * K + lane] = w;
+            if (w_out) w_out[(size_t)t * K + lane] = w;
+            if (id_out) id_out[(size_t)t * K + lane] = id;
+        }
+    }
+    __syncthreads();
+    for (int i = tid; i < TK; i += blockDim.x) atomicAdd(&s_uidx[s_ids[i]], 1);  // slots per expert
+    __syncthreads();
+    const int nchunk = cdiv(E, 32);
+    for (int j = warp; j < nchunk; j += nw) {
+        const int e = 32 * j + lane;
+        const unsigned m = __ballot_sync(0xffffffffu, e < E && s_uidx[e] > 0);
+        if (lane == 0) s_wcnt[j] = __popc(m);
+    }
+    __syncthreads();
+    if (warp == 0) {
+        const int v = (lane < nchunk) ? s_wcnt[lane] : 0;
+        int incl = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int n = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += n;
+        }
+        if (lane < nchunk) s_wbase[lane] = incl - v;
+    }
+    __syncthreads();
+    for (int j = warp; j < nchunk; j += nw) {  // compact the experts, ascending id
+        const int e = 32 * j + lane;
+        const bool f = e < E && s_uidx[e] > 0;
+        const unsigned m = __ballot_sync(0xffffffffu, f);
+        if (f) s_ulist[s_wbase[j] + __popc(m & ((1u << lane) - 1u))] = e;
+    }
+    __syncthreads();
+    const int U = s_wbase[nchunk - 1] + s_wcnt[nchunk - 1];
+    if (warp == 0) {  // offsets of each expert's slot list
+        int run = 0;
+        for (int u0 = 0; u0 < U; u0 += 32) {
+            const int u = u0 + lane;
+            const int v = (u < U) ? s_uidx[s_ulist[u]] : 0;
+            int incl = v;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int n = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += n;
+            }
+            if (u < U) s_uoff[u] = run + incl - v;
+            run += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) s_uoff[U] = run;
+    }
+    __syncthreads();
+    for (int u = tid; u < U; u += blockDim.x) {  // one thread per expert: its slots, ascending token
+        const int e = s_ulist[u];
+        int pos = s_uoff[u];
+        rt->ulist[u] = e;
+        rt->uoff[u] = pos;
+        for (int t = 0; t < T; ++t)
+            for (int k = 0; k < K; ++k)
+                if (s_ids[t * K + k] == e) rt->utok[pos++] = k * T + t;
+    }
+    if (tid == 0) {
+        rt->uoff[U] = s_uoff[U];
+        rt->U = U;
+    }
+    pdl_trigger();
+}
+
+cudaError_t launch_route_small(const float* logits, int T, int E, int K, int score, const float* bias, int renorm,
+                               RouteTable* rt, float* w_out, int32_t* id_out, cudaStream_t s, bool pdl) {
+    const int v = topk_v(E);
+    dim3 grid(1), block(32 * std::max(1, std::min(T, kSmallMaxT)));
+#define MOE_RT(VV) \
+    if (v == VV)   \
+        return launch_k(route_small_kernel<VV>, grid, block, 0, s, pdl, logits, T, E, K, score, bias, renorm, rt, w_out, id_out);
+    MOE_RT(1) MOE_RT(2) MOE_RT(4) MOE_RT(8) MOE_RT(16) MOE_RT(32)
+#undef MOE_RT
     return cudaErrorInvalidValue;
 }
 

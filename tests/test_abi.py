@@ -97,7 +97,7 @@ def test_zero_tokens_is_a_noop():
 def test_path_selection_and_launch_counts():
     d = _desc(T=4)
     assert moe.select_path(d) == "small"
-    assert moe.launches(d) == 3
+    assert moe.launches(d) == 4
     d = _desc(T=4096)
     assert moe.select_path(d) == "large"
     assert moe.launches(d) == 6

@@ -98,6 +98,20 @@ def test_full_shapes_decode_all_rows(shape, T):
     _check(shape, d, "auto")
 
 
+@pytest.mark.parametrize("shape,T", [(gen.QWEN36, 16), (gen.NEMOTRON, 16), (gen.LARGE_E, 16), (gen.NEMOTRON, 9),
+                                     (gen.LARGE_E, 11)])
+def test_full_shapes_small_path_max_tokens(shape, T):
+    """The streaming path at its largest token counts, where x takes most of the shared
+    memory and the stage ring is shortest."""
+    d = _util.device_layer(shape, T, seed=40 + T)
+    _check(shape, d, "small")
+    layer = moe.MoELayer(shape, _util.weights_of(d), path="small")
+    o1 = layer.forward(d["x"])
+    o2 = layer.forward(d["x"])
+    torch.cuda.synchronize()
+    assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
+
+
 @pytest.mark.parametrize("shape,T,routing,nrows", [
     (gen.QWEN36, 4096, "router", 24), (gen.QWEN36, 2048, "zipf", 24), (gen.QWEN36, 8192, "router", 12),
     (gen.NEMOTRON, 1024, "router", 8), (gen.NEMOTRON, 4096, "zipf", 6), (gen.LARGE_E, 256, "router", 16),
