@@ -163,6 +163,16 @@ def kernel_names(path: str, router: bool):
     return names + (["route", "fc1", "fc2"] if path == "small" else ["topk", "permute", "fc1", "fc2", "finalize"])
 
 
+# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu
+# capture of the default workload (seed 0, one GPU), keyed by (config, T, routing, kernel).
+# The capture and its command are summarised in profiles/; an entry is removed whenever
+# its kernel changes, so that a stale count is never reported.
+NCU_TRAFFIC = {
+    ("qwen36", 4096, "router", "fc1"): 1.251730e9 + 65.964032e6,
+    ("qwen36", 4096, "router", "fc2"): 0.635051e9 + 12.244736e6,
+}
+
+
 def roofline_of(acc: dict, dur_s: float, peaks: dict):
     t_hbm = acc["bytes"] / (peaks["hbm_gbs"] * 1e9)
     t_tc = acc["flops"] / (peaks["bf16_tflops"] * 1e12)
@@ -317,7 +327,8 @@ def run_ours(args, rank, local, world):
     roof = roofline_of(acc["kernels"][dom_name], kt[dom] / 1e3, peaks)
     roof["kernel"] = f"{dom_name} ({b.path} path)"
     roof["timing"] = b.kernel_timing
-    roof["traffic"] = None
+    roof["traffic"] = (NCU_TRAFFIC.get((args.config, args.T, args.routing, dom_name))
+                       if args.seed == 0 and b.path == "large" else None)
     roof["peak_source"] = f"of {peaks_src}"
     layer_roof = roofline_of(acc["layer"], ms_step / 1e3, peaks)
     e2e_ms, bi, bo = b.e2e(args.steps, args.warmup)
