@@ -87,10 +87,12 @@ cudaError_t launch_topk(const void* logits, bool bf16_in, int M, int E, int K, i
 
 // ---------------------------------------------------------------- router logits, few tokens
 // l[t, e] = x[t,:] . Wr[e,:], correctly rounded (Sum2 error-free accumulation of the exact
-// BF16 products).  Two warps per CTA, one expert row per warp held in registers (one
-// memory latency per row); the tokens, 16 at a time, are staged in shared memory; each
-// warp runs four independent Sum2 chains (two tokens x even/odd chunks).
-static constexpr int kRouterTokBlock = 16;
+// BF16 products).  CTA (i, g): two warps, one expert row each (experts 2i, 2i+1) held in
+// registers (one memory latency per row), and token group g of kRouterTokBlock tokens,
+// staged in shared memory by one bulk copy.  Each warp runs four independent Sum2 chains
+// (two tokens x even/odd chunks).  Splitting the tokens over the grid keeps the chains
+// short: the Sum2 arithmetic, not memory, would otherwise set the time at T = 16..64.
+static constexpr int kRouterTokBlock = 4;
 
 template <int VH>
 __global__ void __launch_bounds__(64) router_logits_small(const bf16* __restrict__ x, const bf16* __restrict__ wr,
@@ -115,20 +117,16 @@ __global__ void __launch_bounds__(64) router_logits_small(const bf16* __restrict
         w[j] = (e < E && c < nch) ? ld_stream16(wr + (size_t)e * H + (size_t)c * 8) : make_uint4(0u, 0u, 0u, 0u);
     }
     pdl_wait();  // x may come from the previous kernel
-    uint32_t phase = 0;
-    for (int t0 = 0; t0 < T; t0 += kRouterTokBlock) {
-        const int nt = min(kRouterTokBlock, T - t0);
-        __syncthreads();  // every warp is done with the previous block (and sees the barrier init)
-        if (tid == 0) {   // the token block in one bulk copy (rows are 16-byte multiples)
-            const uint32_t bytes = (uint32_t)nt * H * 2;
-            fence_proxy_async_smem();
-            mbar_expect_tx(bar, bytes);
-            bulk_copy_g2s(smem_u32(xs), x + (size_t)t0 * H, bytes, bar);
-        }
-        const bool ok = mbar_wait(bar, phase, &s_abort, err);
-        phase ^= 1u;
-        if (__syncthreads_or(!ok)) break;  // a wait that gave up ends every warp together
-        if (e >= E) continue;
+    const int t0 = blockIdx.y * kRouterTokBlock;
+    const int nt = min(kRouterTokBlock, T - t0);
+    __syncthreads();  // the barrier init is visible
+    if (tid == 0) {   // the token group in one bulk copy (rows are 16-byte multiples)
+        const uint32_t bytes = (uint32_t)nt * H * 2;
+        mbar_expect_tx(bar, bytes);
+        bulk_copy_g2s(smem_u32(xs), x + (size_t)t0 * H, bytes, bar);
+    }
+    const bool ok = mbar_wait(bar, 0, &s_abort, err);
+    if (ok && e < E) {
         for (int t = 0; t < nt; t += 2) {
             const bool two = t + 1 < nt;
             Sum2 a0 = {0.f, 0.f}, a1 = {0.f, 0.f}, b0 = {0.f, 0.f}, b1 = {0.f, 0.f};
@@ -165,8 +163,8 @@ __global__ void __launch_bounds__(64) router_logits_small(const bf16* __restrict
     }
     __syncthreads();
     if (s_abort) {  // a wait gave up: let the bulk copy in flight land before the CTA retires
-        const uint64_t t0 = globaltimer_ns();
-        while (globaltimer_ns() - t0 < 50000ull) {
+        const uint64_t ts = globaltimer_ns();
+        while (globaltimer_ns() - ts < 50000ull) {
         }
     }
     pdl_trigger();
@@ -176,7 +174,7 @@ bool router_small_supported(int H) { return (H >> 3) <= 32 * 16; }
 
 cudaError_t launch_router_small(const bf16* x, const bf16* wr, int T, int H, int E, float* logits,
                                 float* logits_copy, int* err, cudaStream_t s, bool pdl) {
-    dim3 grid(cdiv(E, 2)), block(64);
+    dim3 grid(cdiv(E, 2), cdiv(T, kRouterTokBlock)), block(64);
     const size_t smem = (size_t)kRouterTokBlock * H * 2;
     const int need = cdiv(H >> 3, 32);
 #define MOE_R(VV)                                                                                                \
