@@ -58,6 +58,8 @@ struct Cfg {
     static constexpr int kAccCols = kSwiglu ? 2 * kBN : kBN;
     static constexpr int kTmemCols = (2 * kAccCols) >= 512 ? 512 : 256;
     static constexpr int kThreads = 64 + 32 * kEpiWarps + (kGather ? 128 : 0);
+    // FC1 gather: stages of token rows in flight before the gather warps signal the oldest
+    // one.  (Measured: a lag of 3 or one warp per stage both leave the MMA waiting longer.)
     static constexpr int kLag = 2;
     static constexpr int kMaxGroups = MOE_MAX_EXPERTS + 1;
     // dynamic smem: alignment slack, stages, barriers, flags, tile and offset tables
@@ -260,6 +262,7 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
         }
         int tcount = 0;
         int ebuf = 0;
+        const uint64_t acc_pol = l2_policy_evict_last();
         // (the abort flag is checked through the per-tile wait and vote below, so that the
         // epilogue warps always take the same number of tiles)
         constexpr int kChunks = C::kBN / (32 * (C::kEpiWarps / 4));
@@ -345,9 +348,9 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
                         const int t_r = __shfl_sync(0xffffffffu, mt[ci], r);
                         const int fb = ti.ft * BM;
                         const int nfe = min(BM, a.feat_r - fb);
-                        if (lane < 8 && c0 + r < ti.n && nfe > 0)
-                            bulk_reduce_add_f32(a.acc + (size_t)t_r * a.feat_r + fb, smem_u32(stg + r * 128),
-                                                (uint32_t)nfe * 4u);
+                        if (lane < 8 && c0 + r < ti.n && nfe > 0)  // acc stays in L2 across the K adds
+                            bulk_reduce_add_f32_hint(a.acc + (size_t)t_r * a.feat_r + fb, smem_u32(stg + r * 128),
+                                                     (uint32_t)nfe * 4u, acc_pol);
                         bulk_commit();
                         ebuf ^= 1;
                     }

@@ -22,17 +22,21 @@ struct RowRefine {
 };
 
 // ---------------------------------------------------------------- top-k, one warp per row
+static constexpr int kTopkRowsPerBlock = 4;  // small blocks: the SM fills up to its register limit
+
 template <int V, bool BF16_IN, bool REFINE>
-__global__ void __launch_bounds__(256) topk_kernel(const void* __restrict__ logits, int M, int E, int K, int score,
+__global__ void __launch_bounds__(32 * kTopkRowsPerBlock) topk_kernel(const void* __restrict__ logits, int M, int E, int K, int score,
                                                    const float* __restrict__ bias, int renorm,
                                                    float* __restrict__ topk_w, int32_t* __restrict__ topk_ids,
                                                    int32_t* __restrict__ src_idx, float* __restrict__ w_copy,
                                                    int32_t* __restrict__ id_copy, const bf16* __restrict__ x,
                                                    const bf16* __restrict__ wr, int H, float* logits_rw,
                                                    int* __restrict__ counts) {
+    __shared__ float s_wbuf[kTopkRowsPerBlock][32];
     pdl_wait();
     const int lane = threadIdx.x & 31;
     const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    float* wbuf = s_wbuf[threadIdx.x >> 5];
     if (row < M) {
         float l[V];
         if (BF16_IN)
@@ -43,9 +47,9 @@ __global__ void __launch_bounds__(256) topk_kernel(const void* __restrict__ logi
         float w, lg;
         if (REFINE) {
             const RowRefine rf{x + (size_t)row * H, wr, H, E, row, lane, logits_rw};
-            warp_route_row<V>(l, E, K, score, bias, renorm, lane, kTcLogitErr, rf, id, w, lg);
+            warp_route_row<V>(l, E, K, score, bias, renorm, lane, kTcLogitErr, rf, wbuf, id, w, lg);
         } else {
-            warp_route_row<V>(l, E, K, score, bias, renorm, lane, 0.0f, NoRefine{}, id, w, lg);
+            warp_route_row<V>(l, E, K, score, bias, renorm, lane, 0.0f, NoRefine{}, wbuf, id, w, lg);
         }
         if (lane < K) {
             const size_t o = (size_t)row * K + lane;
@@ -63,8 +67,7 @@ __global__ void __launch_bounds__(256) topk_kernel(const void* __restrict__ logi
 cudaError_t launch_topk(const void* logits, bool bf16_in, int M, int E, int K, int score, const float* bias,
                         int renorm, float* topk_w, int32_t* topk_ids, int32_t* src_idx, float* w_copy,
                         int32_t* id_copy, cudaStream_t s, bool pdl, const RefineArgs* refine, int* counts) {
-    const int rows_per_block = 8;
-    dim3 grid(cdiv(M, rows_per_block)), block(32 * rows_per_block);
+    dim3 grid(cdiv(M, kTopkRowsPerBlock)), block(32 * kTopkRowsPerBlock);
     const int v = topk_v(E);
     const bf16* x = refine ? refine->x : nullptr;
     const bf16* wr = refine ? refine->wr : nullptr;
@@ -204,6 +207,7 @@ __global__ void __launch_bounds__(32 * kSmallMaxT) route_small_kernel(const floa
     __shared__ int s_ulist[kSmallMaxSlots];
     __shared__ int s_uoff[kSmallMaxSlots + 1];
     __shared__ int s_wcnt[32], s_wbase[32];
+    __shared__ float s_wbuf[kSmallMaxT][32];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
     const int TK = T * K;
     for (int e = tid; e < E; e += blockDim.x) s_uidx[e] = 0;
@@ -213,7 +217,7 @@ __global__ void __launch_bounds__(32 * kSmallMaxT) route_small_kernel(const floa
         load_row_f32<V>(logits + (size_t)t * E, E, lane, l);
         int id;
         float w, lg;
-        warp_route_row<V>(l, E, K, score, bias, renorm, lane, 0.0f, NoRefine{}, id, w, lg);
+        warp_route_row<V>(l, E, K, score, bias, renorm, lane, 0.0f, NoRefine{}, s_wbuf[warp], id, w, lg);
         if (lane < K) {
             s_ids[t * K + lane] = id;
             rt->ids[t * K + lane] = id;

@@ -8,9 +8,10 @@
 //
 // Layout: lane l of the warp owns experts e = l + 32 c, c = 0..V-1 (coalesced loads of
 // the row).  A selection takes K rounds; each round reduces every lane's best remaining
-// (key, id) across the warp with XOR shuffles 16, 8, 4, 2, 1 under the total order (key
-// desc, id asc), so every lane ends with the same winner, which its owner drops.  Lane k
-// keeps slot k.
+// entry across the warp under the total order (key desc, id asc) -- the maximum
+// order-preserving key code, then the minimum id among the lanes holding it, two
+// hardware warp reductions -- so every lane sees the same winner, which its owner drops.
+// Lane k keeps slot k.
 //
 // Exact values only where they decide something.  Keys are first screened in cheap FP32
 // (a fast sigmoid; logits that may carry an accumulation error `eps_l`), the K-th
@@ -33,10 +34,6 @@ __device__ __noinline__ float sigmoid_f32_rn(float l) { return __double2float_rn
 __device__ __noinline__ double exp_f64(double v) { return exp(v); }
 // Screening sigmoid: a few ulp from the correctly rounded value.
 __device__ __forceinline__ float sigmoid_fast(float l) { return __frcp_rn(1.0f + __expf(-l)); }
-
-__device__ __forceinline__ bool key_better(float ka, int ia, float kb, int ib) {
-    return ka > kb || (ka == kb && ia < ib);
-}
 
 // ---------------------------------------------------------------- error-free dot product
 // Sum2 of Ogita, Rump and Oishi ("Accurate sum and dot product", SIAM J. Sci. Comput.
@@ -109,65 +106,81 @@ __device__ __forceinline__ uint32_t key_code(float k) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// K rounds over the lane-strided keys.  Each round takes every lane's best remaining
-// expert under (key desc, id asc) and reduces across the warp with two hardware
-// reductions: the maximum key code, then the minimum id among the lanes holding it.
-// Returns the id of slot `lane` (lanes < K) and the K-th key in every lane.
-template <int V>
-__device__ __forceinline__ int warp_select(const float (&key)[V], int E, int K, int lane, float& kth) {
+// Inverse of key_code (zero decodes as +0).
+__device__ __forceinline__ float key_decode(uint32_t code) {
+    return __uint_as_float((code & 0x80000000u) ? (code & 0x7fffffffu) : ~code);
+}
+
+// One entry of a lane's selection cache: key code (0 = none: real keys never map to 0),
+// chunk index, and two payload values that the selection hands to the slot's lane.
+struct SelEntry {
+    uint32_t code;
+    int j;
+    float pa, pb;
+};
+
+// K rounds over the lane-strided keys under (key desc, id asc).  Each lane keeps its
+// three best remaining entries.  A round reduces the lanes' heads across the warp with
+// two hardware reductions (the maximum code, then the minimum id among the lanes holding
+// it); the winner's payload goes to lane k by shuffle.  The winning lane pops its head
+// and rescans its keys only when its cache runs dry, so a round costs a few instructions
+// instead of a scan of all V keys.
+// Returns the id of slot `lane` (lanes < K), its payload (PAYLOAD), and the K-th key.
+template <int V, bool PAYLOAD>
+__device__ __forceinline__ int warp_select(const float (&key)[V], const float (&pa)[V], const float (&pb)[V], int E,
+                                           int K, int lane, float& kth, float& out_a, float& out_b) {
     uint32_t avail = 0;
 #pragma unroll
     for (int c = 0; c < V; ++c)
         if (lane + 32 * c < E) avail |= 1u << c;
-    int my = 0;
-    kth = 0.0f;
-    for (int k = 0; k < K; ++k) {
-        float bk = __int_as_float(0xff800000);
-        int bi = 0x7fffffff;
+    SelEntry e1, e2, e3;
+    auto rescan = [&]() {
+        e1 = e2 = e3 = SelEntry{0u, 0, 0.0f, 0.0f};
 #pragma unroll
         for (int c = 0; c < V; ++c) {
             if ((avail >> c) & 1u) {
-                const int e = lane + 32 * c;
-                if (key_better(key[c], e, bk, bi)) {
-                    bk = key[c];
-                    bi = e;
+                // ids ascend with c within a lane: on equal codes the earlier entry ranks first
+                const SelEntry n{key_code(key[c]), c, PAYLOAD ? pa[c] : 0.0f, PAYLOAD ? pb[c] : 0.0f};
+                if (n.code > e1.code) {
+                    e3 = e2;
+                    e2 = e1;
+                    e1 = n;
+                } else if (n.code > e2.code) {
+                    e3 = e2;
+                    e2 = n;
+                } else if (n.code > e3.code) {
+                    e3 = n;
                 }
             }
         }
-        const uint32_t code = (bi == 0x7fffffff) ? 0u : key_code(bk);
-        const uint32_t best = __reduce_max_sync(0xffffffffu, code);
-        const int win = (int)__reduce_min_sync(0xffffffffu, (code == best) ? (uint32_t)bi : 0x7fffffffu);
-        if (lane == (win & 31)) avail &= ~(1u << (win >> 5));
+    };
+    rescan();
+    int my = 0;
+    out_a = out_b = 0.0f;
+    kth = 0.0f;
+    for (int k = 0; k < K; ++k) {
+        const uint32_t best = __reduce_max_sync(0xffffffffu, e1.code);
+        const uint32_t mine = (e1.code != 0u && e1.code == best) ? (uint32_t)(lane + 32 * e1.j) : 0x7fffffffu;
+        const int win = (int)__reduce_min_sync(0xffffffffu, mine);
+        if (PAYLOAD) {
+            const float va = __shfl_sync(0xffffffffu, e1.pa, win & 31);
+            const float vb = __shfl_sync(0xffffffffu, e1.pb, win & 31);
+            if (lane == k) {
+                out_a = va;
+                out_b = vb;
+            }
+        }
         if (lane == k) my = win;
-        if (k == K - 1) kth = __shfl_sync(0xffffffffu, bk, win & 31);
-    }
-    return my;
-}
-
-// Value of expert `id` (uniform across the warp) from its owner lane.
-template <int V>
-__device__ __forceinline__ float warp_fetch(const float (&v)[V], int id) {
-    const int cw = id >> 5;
-    float r = v[0];
-#pragma unroll
-    for (int c = 1; c < V; ++c)
-        if (c == cw) r = v[c];
-    return __shfl_sync(0xffffffffu, r, id & 31);
-}
-
-// Position of the n-th (0-based) set bit of m; n < popc(m).
-__device__ __forceinline__ int nth_set_bit(unsigned m, int n) {
-    int p = 0;
-#pragma unroll
-    for (int w = 16; w >= 1; w >>= 1) {
-        const int lo = __popc(m & ((1u << w) - 1u));
-        if (n >= lo) {
-            n -= lo;
-            m >>= w;
-            p += w;
+        if (k == K - 1) kth = key_decode(best);
+        if (lane == (win & 31)) {
+            avail &= ~(1u << (win >> 5));
+            e1 = e2;
+            e2 = e3;
+            e3.code = 0u;
+            if (e1.code == 0u && avail) rescan();
         }
     }
-    return p;
+    return my;
 }
 
 struct NoRefine {
@@ -175,13 +188,18 @@ struct NoRefine {
 };
 
 // Screening + exact values for the candidates.  On entry key[] holds the screening keys;
-// on exit the keys of every candidate are exact (and refined logits are in l).
+// on exit the keys of every candidate are exact (and refined logits are in l), and for
+// sigmoid scores sx[] holds each candidate's correctly rounded sigmoid.  The experts the
+// final selection takes are always candidates: each of the K screened best has an exact
+// key at least kth - win/2, above the exact key of anything outside the window.
+// wbuf: 32 floats of shared memory owned by this warp.
 template <int V, class Refine>
-__device__ __forceinline__ void route_refine_keys(float (&l)[V], float (&key)[V], int E, int K, bool sig,
-                                                  const float* bias, int lane, float eps_l, const Refine& refine) {
+__device__ __forceinline__ void route_refine_keys(float (&l)[V], float (&key)[V], float (&sx)[V], int E, int K,
+                                                  bool sig, const float* bias, int lane, float eps_l,
+                                                  const Refine& refine, float* wbuf) {
     const float NEG_INF = __int_as_float(0xff800000);
-    float kth;
-    warp_select<V>(key, E, K, lane, kth);
+    float kth, ua, ub;
+    warp_select<V, false>(key, key, key, E, K, lane, kth, ua, ub);
     // Window: screening error of a key (logit error, sigmoid slope <= 1/4, fast-sigmoid
     // error, key rounding), doubled because both sides of a comparison carry it.
     const float mag = fmaxf(1.0f, fabsf(kth));
@@ -213,47 +231,45 @@ __device__ __forceinline__ void route_refine_keys(float (&l)[V], float (&key)[V]
         }
     }
     if (!sig) return;
-    // Sigmoid keys: the candidates are packed onto consecutive lanes so that the FP64
-    // sigmoid runs once per 32 candidates rather than once per chunk holding one.
+    // Sigmoid keys: the candidates' logits are packed into the warp's buffer, each lane
+    // evaluates one FP64 sigmoid, and the results go back to the owners -- one pass per 32
+    // candidates.
     const unsigned lt = (1u << lane) - 1u;
     for (int r0 = 0; r0 < ncand; r0 += 32) {
-        const int j = r0 + lane;  // candidate evaluated by this lane
-        float lv = 0.0f;
 #pragma unroll
         for (int c = 0; c < V; ++c) {
-            const int rel = j - base[c];
-            const bool mine = rel >= 0 && rel < __popc(mc[c]);
-            const float v = __shfl_sync(0xffffffffu, l[c], mine ? nth_set_bit(mc[c], rel) : 0);
-            if (mine) lv = v;
+            const int pos = base[c] + __popc(mc[c] & lt) - r0;
+            if (((mc[c] >> lane) & 1u) && pos >= 0 && pos < 32) wbuf[pos] = l[c];
         }
-        const float sv = (j < ncand) ? sigmoid_f32_rn(lv) : 0.0f;
+        __syncwarp();
+        const float lv = wbuf[lane];
+        const float sv = (r0 + lane < ncand) ? sigmoid_f32_rn(lv) : 0.0f;
+        __syncwarp();
+        wbuf[lane] = sv;
+        __syncwarp();
 #pragma unroll
         for (int c = 0; c < V; ++c) {
-            const int pos = base[c] + __popc(mc[c] & lt) - r0;  // this lane's candidate, this round
-            const bool here = ((mc[c] >> lane) & 1u) && pos >= 0 && pos < 32;
-            const float got = __shfl_sync(0xffffffffu, sv, here ? pos : 0);
-            if (here) {
-                float k = got;
+            const int pos = base[c] + __popc(mc[c] & lt) - r0;
+            if (((mc[c] >> lane) & 1u) && pos >= 0 && pos < 32) {
+                const float sg = wbuf[pos];
+                sx[c] = sg;
+                float k = sg;
                 if (bias) k = __fadd_rn(k, bias[lane + 32 * c]);
                 key[c] = (k != k) ? NEG_INF : k;
             }
         }
+        __syncwarp();
     }
 }
 
-// Weights of the selected experts from exact values (lanes k < K hold slot k).
+// Weights of the selected experts from exact values: lane k < K holds slot k's logit
+// sel_l and (sigmoid scores) its correctly rounded sigmoid sel_s.
 template <int V>
 __device__ __forceinline__ void finish_route_row(const float (&l)[V], int E, int K, bool sig, int renorm, int lane,
-                                                 int out_id, float& out_w, float& out_l) {
+                                                 float sel_l, float sel_s, float& out_w) {
     const float NEG_INF = __int_as_float(0xff800000);
-    out_l = 0.0f;
-    for (int k = 0; k < K; ++k) {
-        const int id = __shfl_sync(0xffffffffu, out_id, k);
-        const float v = warp_fetch<V>(l, id);
-        if (lane == k) out_l = v;
-    }
     if (sig) {
-        const float s = (lane < K) ? sigmoid_f32_rn(out_l) : 0.0f;
+        const float s = (lane < K) ? sel_s : 0.0f;
         double sum = 0.0;
         for (int k = 0; k < K; ++k) sum += (double)__shfl_sync(0xffffffffu, s, k);
         out_w = renorm ? __double2float_rn((double)s / sum) : s;
@@ -264,7 +280,7 @@ __device__ __forceinline__ void finish_route_row(const float (&l)[V], int E, int
             if (lane + 32 * c < E && l[c] == l[c]) lmax = fmaxf(lmax, l[c]);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) lmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
-        const double ex = (lane < K) ? exp_f64((double)out_l - (double)lmax) : 0.0;
+        const double ex = (lane < K) ? exp_f64((double)sel_l - (double)lmax) : 0.0;
         double sum = 0.0;
         if (renorm) {
             for (int k = 0; k < K; ++k) sum += __shfl_sync(0xffffffffu, ex, k);
@@ -283,18 +299,21 @@ __device__ __forceinline__ void finish_route_row(const float (&l)[V], int E, int
 // One routing row.  l[c]: logit of expert lane + 32c (any value for e >= E), exact when
 // eps_l == 0, otherwise within eps_l (absolute) of the exact FP32 value and re-evaluated
 // with refine(e) (warp-collective) where it matters; refined logits are written back
-// into l.  Outputs on lanes k < K: slot k's expert id, weight and exact logit.
+// into l.  wbuf: 32 floats of shared memory owned by this warp.  Outputs on lanes k < K:
+// slot k's expert id, weight and exact logit.
 template <int V, class Refine>
 __device__ __forceinline__ void warp_route_row(float (&l)[V], int E, int K, int score, const float* bias, int renorm,
-                                               int lane, float eps_l, const Refine& refine, int& out_id, float& out_w,
-                                               float& out_l) {
+                                               int lane, float eps_l, const Refine& refine, float* wbuf, int& out_id,
+                                               float& out_w, float& out_l) {
     const float NEG_INF = __int_as_float(0xff800000);
     const bool sig = score == MOE_SCORE_SIGMOID;
     float key[V];
+    float sx[V];  // exact sigmoid of the candidates (sigmoid scores only)
 #pragma unroll
     for (int c = 0; c < V; ++c) {
         const int e = lane + 32 * c;
         key[c] = NEG_INF;
+        sx[c] = 0.0f;
         if (e < E) {
             const float lv = l[c];
             float k = sig ? sigmoid_fast(lv) : lv;
@@ -302,14 +321,11 @@ __device__ __forceinline__ void warp_route_row(float (&l)[V], int E, int K, int 
             key[c] = (k != k) ? NEG_INF : k;
         }
     }
-    float kth;
-    if (!sig && eps_l == 0.0f) {  // exact logits keyed directly: the screening keys are the keys
-        out_id = warp_select<V>(key, E, K, lane, kth);
-    } else {
-        route_refine_keys<V>(l, key, E, K, sig, bias, lane, eps_l, refine);
-        out_id = warp_select<V>(key, E, K, lane, kth);
-    }
-    finish_route_row<V>(l, E, K, sig, renorm, lane, out_id, out_w, out_l);
+    // exact logits keyed directly (softmax, eps 0): the screening keys are the keys
+    if (sig || eps_l > 0.0f) route_refine_keys<V>(l, key, sx, E, K, sig, bias, lane, eps_l, refine, wbuf);
+    float kth, sel_s;
+    out_id = warp_select<V, true>(key, l, sx, E, K, lane, kth, out_l, sel_s);
+    finish_route_row<V>(l, E, K, sig, renorm, lane, out_l, sel_s, out_w);
 }
 
 // Load one row of FP32 logits in the lane-strided layout.
