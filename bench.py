@@ -397,6 +397,107 @@ def sweep(args, device, peaks):
     return rows
 
 
+# ---------------------------------------------------------------- router top-k alone
+ROUTER_E, ROUTER_K = 256, 10
+
+
+def run_router_topk(args, rank, local, world):
+    """The router-top-k-only workload: moe_router_topk on BF16 logits [M, 256] (M = --T),
+    sigmoid scores, an FP32 selection bias ~ N(0, 0.5), top-10, renormalised, with ~10 %
+    of rows holding a designed exact tie.  One step is one call over all M rows."""
+    import mixture_experts_layer_35_b200.moe as moe
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    dist_init(world, "nccl")
+    peaks, peaks_src = load_peaks()
+    M, E, K = args.T, ROUTER_E, ROUTER_K
+    case = gen.make_router_case(M, E, K, seed=args.seed + rank, bias_mode="random")
+    lg = case["logits"].to(device)
+    bias = case["bias"].to(device)
+    outs = tuple(torch.empty((M, K), dtype=dt, device=device) for dt in (torch.float32, torch.int32, torch.int32))
+    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.Stream(device)
+    call = lambda x=lg: moe.router_topk(x, K, "sigmoid", bias, True, stream=stream, out=outs)  # noqa: E731
+    call()
+    torch.cuda.synchronize(device)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        call()
+    torch.cuda.synchronize(device)
+    for _ in range(args.warmup):
+        flush_buf.fill_(1)
+        graph.replay()
+    torch.cuda.synchronize(device)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier(world, device)
+    torch.cuda.synchronize(device)
+    sampler = ClockSampler(device.index)
+    for a, b in evs:
+        flush_buf.fill_(1)
+        a.record()
+        graph.replay()
+        b.record()
+    torch.cuda.synchronize(device)
+    clk = sampler.stop()
+    barrier(world, device)
+    per = [a.elapsed_time(b) for a, b in evs]
+    total_ms = max_over_ranks(float(sum(per)), world, device)
+    ms_step = total_ms / args.steps
+    value = world * M * args.steps / (total_ms / 1e3)
+    acc = {"bytes": M * E * 2 + E * 4 + M * K * 12, "flops": 0}
+    roof = roofline_of(acc, ms_step / 1e3, peaks)
+    roof.update({"kernel": "topk_kernel", "timing": "CUDA-graph replay, one launch per step", "traffic": None,
+                 "peak_source": f"of {peaks_src}"})
+    # end to end: pinned host logits in, weights and ids out, through the public call
+    lg_host = case["logits"].pin_memory()
+    w_host = torch.empty((M, K), dtype=torch.float32).pin_memory()
+    id_host = torch.empty((M, K), dtype=torch.int32).pin_memory()
+    lg_dev = torch.empty_like(lg)
+    e2e_ms = []
+    for i in range(args.warmup + args.steps):
+        flush_buf.fill_(1)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        lg_dev.copy_(lg_host, non_blocking=True)
+        moe.router_topk(lg_dev, K, "sigmoid", bias, True, out=outs)
+        w_host.copy_(outs[0], non_blocking=True)
+        id_host.copy_(outs[1], non_blocking=True)
+        b.record()
+        torch.cuda.synchronize(device)
+        if i >= args.warmup:
+            e2e_ms.append(a.elapsed_time(b))
+    e2e_total = max_over_ranks(float(sum(e2e_ms)), world, device)
+    line = {
+        "metric": METRIC, "value": value, "unit": "rows/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded generator, designed ties)",
+        "config": {"workload": f"router-top-k-only BF16 logits [{M},{E}] top-{K} sigmoid+bias renorm",
+                   "rows_per_step": M, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write)"},
+        "roofline": roof,
+        "e2e": {"value": world * M * args.steps / (e2e_total / 1e3), "unit": "rows/s",
+                "h2d_bytes_per_step": M * E * 2, "d2h_bytes_per_step": M * K * 8},
+        "gpu_launches": args.steps, "clocks": clk,
+        "us_per_step_p10_p50_p90": [float(np.percentile(per, q)) * 1e3 for q in (10, 50, 90)],
+    }
+    if rank == 0 and world == 1 and not args.no_cpu:
+        import oracle
+        hl = gen.bf16_bits(case["logits"])
+        hb = case["bias"].numpy()
+        t0, n = time.perf_counter(), 0
+        while n < M and time.perf_counter() - t0 < args.cpu_budget:
+            oracle.topk(hl[n:n + 64], K, "sigmoid", hb, True, logits_bf16=True)
+            n += min(64, M - n)
+        dt = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": n / dt, "unit": "rows/s", "cores": 1, "kind": "oracle",
+                                "sample": f"{n} rows of the same logits in {dt:.2f} s (single-threaded C)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    barrier(world, device)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
 # ---------------------------------------------------------------- reference arm (CPU oracle)
 def run_reference(args, rank, local, world):
     if rank != 0:
@@ -437,6 +538,8 @@ def main(argv=None):
     p.add_argument("--steps", type=int, default=100)
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", choices=["layer", "router_topk"], default="layer",
+                   help="layer: moe_fused_forward on --config; router_topk: moe_router_topk alone, M = --T rows")
     p.add_argument("--config", choices=sorted(gen.SHORT), default="qwen36")
     p.add_argument("--T", type=int, default=4096)
     p.add_argument("--routing", choices=["router", "zipf"], default="router")
@@ -453,6 +556,8 @@ def main(argv=None):
     rank, local, world = dist_env()
     if args.impl == "reference":
         run_reference(args, rank, local, world)
+    elif args.workload == "router_topk":
+        run_router_topk(args, rank, local, world)
     else:
         run_ours(args, rank, local, world)
 

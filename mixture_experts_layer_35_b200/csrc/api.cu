@@ -66,9 +66,19 @@ moe_status_t validate_desc(const moe_layer_desc* d) {
 // Token-count rule of MOE_PATH_AUTO.  The streaming path reads each routed expert once
 // and wins while the experts see few tokens; the tensor-core path wins once its MMA
 // work per weight byte pays for the tile machinery.
+// Path selector.  The streaming path saves the many-token path's extra kernels (top-k +
+// permute + finalize against one route-table kernel), but streams weights on the CUDA
+// cores more slowly than TMA + tcgen05 does, so it wins only while the weight bytes of
+// the call are small.  The threshold sits in the measured crossover on B200: the
+// streaming path was ahead at 100.7 MB of touched expert weights (Qwen3.6-shaped T = 2)
+// and behind at 108 MB (large-E-shaped T = 1, with its shared expert) and above.
+static constexpr double kSmallPathMaxBytes = 104e6;
 int auto_path(const moe_layer_desc* d) {
     if (!small_path_supported(d->T, d->H, d->I, d->I_shared)) return MOE_PATH_LARGE;
-    return d->T <= 8 ? MOE_PATH_SMALL : MOE_PATH_LARGE;
+    const double m = d->act == MOE_ACT_SWIGLU ? 3.0 : 2.0;
+    const double experts = (double)std::min(d->T * d->top_k, d->E);
+    const double bytes = experts * m * d->H * d->I * 2.0 + m * d->H * (double)d->I_shared * 2.0;
+    return bytes <= kSmallPathMaxBytes ? MOE_PATH_SMALL : MOE_PATH_LARGE;
 }
 int resolve_path(const moe_layer_desc* d) {
     if (d->path == MOE_PATH_AUTO) return auto_path(d);
@@ -131,7 +141,7 @@ moe_status_t run_router_dense(const moe_layer_desc* d, const bf16* x, float* log
     m.a_s = m.a_r;
     m.b_s = m.b_r;
     const int tiles = g.nfeat_r * cdiv(d->T, kDenseTokenTile);
-    MOE_CK(launch_gemm(GM_DENSE, g, m, std::min(sms, tiles), s, pdl));
+    MOE_CK(launch_gemm(GM_DENSE, 0, g, m, std::min(sms, tiles), s, pdl));
     return MOE_OK;
 }
 
@@ -213,8 +223,6 @@ moe_status_t moe_permute(const int32_t* topk_ids, int M, int K, int E, int32_t* 
     a.perm = perm;
     a.inv = inv;
     a.err = &static_cast<WsHeader*>(ws)->err;
-    a.bn1 = kFc1TokenTile;
-    a.bn2 = kFc2TokenTile;
     if (launch_permute(a, (cudaStream_t)stream, false) != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_OK;
 }
@@ -353,8 +361,10 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
     pa.perm = perm;
     pa.err = err;
     pa.has_shared = Is > 0;
-    pa.bn1 = kFc1TokenTile;
-    pa.bn2 = kFc2TokenTile;
+    const int fc1_mode = swiglu ? GM_FC1_SWIGLU : GM_FC1_RELU2;
+    const int bn1 = gemm_token_tile(fc1_mode, T, K, E), bn2 = gemm_token_tile(GM_FC2, T, K, E);
+    pa.bn1 = bn1;
+    pa.bn2 = bn2;
     pa.nfeat1_r = cdiv(I, 128);
     pa.nfeat1_s = cdiv(Is, 128);
     pa.nfeat2_r = cdiv(H, 128);
@@ -402,7 +412,7 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
     g1.zero_n = (size_t)T * H;
     g1.err = err;
     if (!mark()) return MOE_ERR_CUDA;
-    MOE_CK(launch_gemm(swiglu ? GM_FC1_SWIGLU : GM_FC1_RELU2, g1, m1, sms, s, chain));
+    MOE_CK(launch_gemm(fc1_mode, bn1, g1, m1, sms, s, chain));
 
     // 5. FC2 + weighted scatter-add (shared expert -> ys)
     GemmMaps m2;
@@ -427,7 +437,7 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
     g2.zero_ptr = nullptr;
     g2.zero_n = 0;
     if (!mark()) return MOE_ERR_CUDA;
-    MOE_CK(launch_gemm(GM_FC2, g2, m2, sms, s, chain));
+    MOE_CK(launch_gemm(GM_FC2, bn2, g2, m2, sms, s, chain));
 
     // 6. finalize
     if (!mark()) return MOE_ERR_CUDA;

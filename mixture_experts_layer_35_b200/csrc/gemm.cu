@@ -37,34 +37,57 @@ constexpr int BM = 128, BK = 64;
 constexpr int A_BYTES = BM * BK * 2;  // 16 KB
 constexpr int BBOX = 16;              // token rows per TMA box of the B operand
 
+// Token rows per tile (MMA N) of each mode at prefill sizes: FC2 takes up to 256 so that
+// an expert's W2 tile is streamed once for all its tokens; FC1 keeps 128 so that its gate
+// and up accumulators stay double-buffered in TMEM.  When every expert has at most 32
+// rows (T <= 32) both use 32-row tiles, whose smaller token stages leave room for a
+// deeper weight ring.
 template <int MODE>
+constexpr int default_bn() {
+    return MODE == GM_FC2 ? 256 : 128;
+}
+
+template <int MODE, int BN>
 struct Cfg {
     static constexpr bool kGather = (MODE == GM_FC1_SWIGLU || MODE == GM_FC1_RELU2);
     static constexpr bool kSwiglu = (MODE == GM_FC1_SWIGLU);
     static constexpr int kNA = kSwiglu ? 2 : 1;
-    // Token rows per tile (MMA N): FC2 takes up to 256 so that an expert's W2 tile is
-    // streamed once for all its tokens at prefill sizes; FC1 keeps 128 so that its gate
-    // and up accumulators stay double-buffered in TMEM.
-    static constexpr int kBN = (MODE == GM_FC2) ? 256 : 128;
+    static constexpr int kBN = BN;
     static constexpr int kBBytes = kBN * BK * 2;
     static constexpr int kStageBytes = kNA * A_BYTES + kBBytes;
-    static constexpr int kStages = kSwiglu ? 4 : (MODE == GM_FC2 ? 3 : 6);
     // Epilogue warps: FC2's epilogue (staging + bulk reduce) is heavier than its short
-    // mainloop, so it gets two warps per TMEM lane quarter, splitting the token columns.
-    static constexpr int kEpiWarps = (MODE == GM_FC2) ? 8 : 4;
+    // mainloop, so with wide tiles it gets two warps per TMEM lane quarter, splitting the
+    // token columns.
+    static constexpr int kEpiWarps = (MODE == GM_FC2 && BN > 32) ? 8 : 4;
     // FC2: per half of the epilogue warps, two [32 tokens][128 features] FP32 staging
     // blocks for the bulk reduce-add into acc.
-    static constexpr int kEpiBytes = (MODE == GM_FC2) ? 2 * 2 * 32 * 128 * 4 : 0;
+    static constexpr int kEpiBytes = (MODE == GM_FC2) ? (kEpiWarps / 4) * 2 * 32 * 128 * 4 : 0;
     static constexpr int kAccCols = kSwiglu ? 2 * kBN : kBN;
-    static constexpr int kTmemCols = (2 * kAccCols) >= 512 ? 512 : 256;
+    // Two accumulator buffers (the epilogue of one tile overlaps the next mainloop) when
+    // they fit TMEM's 512 columns; a 256-token SwiGLU tile (gate + up = 512 columns) has one.
+    static constexpr int kAccBufs = (2 * kAccCols) <= 512 ? 2 : 1;
+    static constexpr int kTmemCols =
+        (kAccBufs * kAccCols) > 256 ? 512 : ((kAccBufs * kAccCols) > 128 ? 256 : 128);
+    static_assert(kAccCols <= 512, "accumulator exceeds TMEM");
     static constexpr int kThreads = 64 + 32 * kEpiWarps + (kGather ? 128 : 0);
     // FC1 gather: stages of token rows in flight before the gather warps signal the oldest
-    // one.  (Measured: a lag of 3 or one warp per stage both leave the MMA waiting longer.)
-    static constexpr int kLag = 2;
+    // one.  It must stay at most kStages - 2: the gather can only issue stage j + lag once
+    // the MMA has freed that slot, so with lag = kStages - 1 the signal for stage j waits
+    // for the MMA to finish stage j - 1 and every stage starts late (measured: lag 3 of 4
+    // stages, and lag 2 of 3, both stall; one warp per stage is slower too).
+    static constexpr int kLagMax = 2;
     static constexpr int kMaxGroups = MOE_MAX_EXPERTS + 1;
+    static constexpr size_t kMeta = 256 + (size_t)(kMaxGroups + 1) * 4 * 2 + 64;
+    // As many stages as the 227 KB of shared memory hold (at most 12: the barrier block).
+    static constexpr int kStages =
+        (int)((227 * 1024 - 1024 - kMeta - kEpiBytes) / kStageBytes) < 12
+            ? (int)((227 * 1024 - 1024 - kMeta - kEpiBytes) / kStageBytes)
+            : 12;
     // dynamic smem: alignment slack, stages, barriers, flags, tile and offset tables
-    static constexpr size_t kSmem =
-        1024 + (size_t)kStages * kStageBytes + kEpiBytes + 256 + (size_t)(kMaxGroups + 1) * 4 * 2 + 64;
+    static constexpr size_t kSmem = 1024 + (size_t)kStages * kStageBytes + kEpiBytes + kMeta;
+    static constexpr int kLag = (kStages - 2) < kLagMax ? (kStages - 2) : kLagMax;
+    static_assert(kStages >= 3, "ring too shallow");
+    static_assert(8 * (2 * kStages + 4) + 8 <= 256, "barrier block");
 };
 
 struct TileInfo {
@@ -105,11 +128,11 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmArgs& a, const int* s_
     return ti;
 }
 
-template <int MODE>
-__global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
+template <int MODE, int BN>
+__global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
     gemm_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ CUtensorMap tm_a_s,
                 const __grid_constant__ CUtensorMap tm_b_r, const __grid_constant__ CUtensorMap tm_b_s) {
-    using C = Cfg<MODE>;
+    using C = Cfg<MODE, BN>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_u32 = smem_u32(smem_raw);
     const uint32_t base_u32 = (raw_u32 + 1023u) & ~1023u;
@@ -217,8 +240,8 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
                 const int nk = cdiv(kd, BK);
                 const int npad = cdiv(ti.n, 16) * 16;
                 const uint32_t idesc = idesc_bf16_f32(BM, npad);
-                const int buf = tcount & 1;
-                const uint32_t tph = (uint32_t)(tcount >> 1) & 1u;
+                const int buf = tcount % C::kAccBufs;
+                const uint32_t tph = (uint32_t)(tcount / C::kAccBufs) & 1u;
                 if (!mbar_wait(tempty_bar(buf), tph ^ 1u, abort_flag, a.err)) break;
                 tc_fence_after();
                 const uint32_t d0 = tmem_base + (uint32_t)(buf * C::kAccCols);
@@ -268,8 +291,8 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
         constexpr int kChunks = C::kBN / (32 * (C::kEpiWarps / 4));
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++tcount) {
             const TileInfo ti = decode_tile<C::kBN>(a, s_tiles, s_offs, G, tile);
-            const int buf = tcount & 1;
-            const uint32_t tph = (uint32_t)(tcount >> 1) & 1u;
+            const int buf = tcount % C::kAccBufs;
+            const uint32_t tph = (uint32_t)(tcount / C::kAccBufs) & 1u;
             // FC2: token and routing weight of each column this thread will scale, loaded
             // before the accumulator is ready (hidden behind the tile's mainloop).
             int mt[kChunks];
@@ -381,9 +404,9 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
             const int kd = ti.shared ? a.kdim_s : a.kdim;
             const int nk = cdiv(kd, BK);
             const int npad = cdiv(ti.n, 16) * 16;
-            int tok[8];
+            int tok[C::kBN / 16];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
+            for (int j = 0; j < C::kBN / 16; ++j) {
                 const int r = rsub + 16 * j;
                 tok[j] = -1;
                 if (r < ti.n) tok[j] = ti.shared ? ti.row0 + r : (a.perm[ti.row0 + r] % a.T);
@@ -399,7 +422,7 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
                 const uint32_t bs = base_u32 + (uint32_t)s * C::kStageBytes + C::kNA * A_BYTES;
                 const int kcol = kb * BK + chunk * 8;
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
+                for (int j = 0; j < C::kBN / 16; ++j) {
                     const int r = rsub + 16 * j;
                     if (r < npad) {
                         const uint32_t dst = bs + (uint32_t)r * 128u + ((uint32_t)(chunk ^ (r & 7)) << 4);
@@ -464,29 +487,49 @@ __global__ void __launch_bounds__(256) finalize_kernel(const float* __restrict__
 
 }  // namespace
 
-size_t gemm_smem_bytes(int mode) {
-    switch (mode) {
-        case GM_FC1_SWIGLU: return Cfg<GM_FC1_SWIGLU>::kSmem;
-        case GM_FC1_RELU2: return Cfg<GM_FC1_RELU2>::kSmem;
-        case GM_FC2: return Cfg<GM_FC2>::kSmem;
-        default: return Cfg<GM_DENSE>::kSmem;
-    }
-}
-
-template <int MODE>
+template <int MODE, int BN>
 static cudaError_t launch_mode(const GemmArgs& a, const GemmMaps& m, int grid, cudaStream_t s, bool pdl) {
-    using C = Cfg<MODE>;
-    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
+    using C = Cfg<MODE, BN>;
+    cudaError_t e =
+        cudaFuncSetAttribute(gemm_kernel<MODE, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
     if (e != cudaSuccess) return e;
-    return launch_k(gemm_kernel<MODE>, dim3(grid), dim3(C::kThreads), C::kSmem, s, pdl, a, m.a_r, m.a_s, m.b_r, m.b_s);
+    return launch_k(gemm_kernel<MODE, BN>, dim3(grid), dim3(C::kThreads), C::kSmem, s, pdl, a, m.a_r, m.a_s, m.b_r,
+                    m.b_s);
 }
 
-cudaError_t launch_gemm(int mode, const GemmArgs& a, const GemmMaps& m, int grid, cudaStream_t s, bool pdl) {
+int gemm_token_tile(int mode, int T, int K, int E) {
+    if (mode == GM_DENSE) return default_bn<GM_DENSE>();
+    if (T <= 32) return 32;  // no expert has more rows than a tile
+    const double rows = (double)T * K / E;  // average rows per expert
+    if (mode == GM_FC2) return rows <= 64.0 ? 128 : 256;  // measured: 256 ahead from ~128 rows
+    // FC1: a tile re-streams the expert's weight slice, so an expert just over a tile's
+    // width costs a second, nearly empty tile; 256-token tiles keep most experts at one.
+    // Not for SwiGLU: its 256-token stage (64 KB) leaves room for only 3 stages, and the
+    // bytes in flight per SM, not the tile count, set the time (measured: 128 is ahead at
+    // 128 and 256 rows per expert).
+    if (mode == GM_FC1_SWIGLU) return rows <= 48.0 ? 64 : 128;
+    return rows <= 48.0 ? 64 : (rows <= 96.0 ? 128 : 256);
+}
+
+cudaError_t launch_gemm(int mode, int bn, const GemmArgs& a, const GemmMaps& m, int grid, cudaStream_t s, bool pdl) {
     switch (mode) {
-        case GM_FC1_SWIGLU: return launch_mode<GM_FC1_SWIGLU>(a, m, grid, s, pdl);
-        case GM_FC1_RELU2: return launch_mode<GM_FC1_RELU2>(a, m, grid, s, pdl);
-        case GM_FC2: return launch_mode<GM_FC2>(a, m, grid, s, pdl);
-        case GM_DENSE: return launch_mode<GM_DENSE>(a, m, grid, s, pdl);
+        case GM_FC1_SWIGLU:
+            if (bn == 32) return launch_mode<GM_FC1_SWIGLU, 32>(a, m, grid, s, pdl);
+            if (bn == 64) return launch_mode<GM_FC1_SWIGLU, 64>(a, m, grid, s, pdl);
+            if (bn == 128) return launch_mode<GM_FC1_SWIGLU, 128>(a, m, grid, s, pdl);
+            break;
+        case GM_FC1_RELU2:
+            if (bn == 32) return launch_mode<GM_FC1_RELU2, 32>(a, m, grid, s, pdl);
+            if (bn == 64) return launch_mode<GM_FC1_RELU2, 64>(a, m, grid, s, pdl);
+            if (bn == 128) return launch_mode<GM_FC1_RELU2, 128>(a, m, grid, s, pdl);
+            if (bn == 256) return launch_mode<GM_FC1_RELU2, 256>(a, m, grid, s, pdl);
+            break;
+        case GM_FC2:
+            if (bn == 32) return launch_mode<GM_FC2, 32>(a, m, grid, s, pdl);
+            if (bn == 128) return launch_mode<GM_FC2, 128>(a, m, grid, s, pdl);
+            if (bn == 256) return launch_mode<GM_FC2, 256>(a, m, grid, s, pdl);
+            break;
+        case GM_DENSE: return launch_mode<GM_DENSE, default_bn<GM_DENSE>()>(a, m, grid, s, pdl);
     }
     return cudaErrorInvalidValue;
 }

@@ -104,10 +104,8 @@ cudaError_t launch_permute_fast(const PermuteArgs& a, const int* counts, int* cu
 // ---------------------------------------------------------------- grouped tcgen05 GEMM
 enum GemmMode { GM_FC1_SWIGLU = 0, GM_FC1_RELU2 = 1, GM_FC2 = 2, GM_DENSE = 3 };
 // Token rows per tile of the dense router GEMM (E is small, so smaller token tiles give
-// the grid more CTAs), and of the grouped FC1 / FC2 GEMMs.
+// the grid more CTAs).  The grouped FC1 / FC2 GEMMs take gemm_token_tile(mode, T).
 static constexpr int kDenseTokenTile = 64;
-static constexpr int kFc1TokenTile = 128;
-static constexpr int kFc2TokenTile = 256;
 struct GemmArgs {
     int T, K;            // tokens and top-k (slot decode of perm entries)
     int kdim;            // reduction length (H for FC1 / router, I or I_s for FC2)
@@ -139,9 +137,13 @@ struct GemmMaps {
     CUtensorMap b_r;  // FC2: h [T*K, I]; DENSE: x [T, H] (16-row boxes)
     CUtensorMap b_s;  // FC2: hs [T, I_s]
 };
-cudaError_t launch_gemm(int mode, const GemmArgs& a, const GemmMaps& m, int grid, cudaStream_t s, bool pdl);
-size_t gemm_smem_bytes(int mode);
-int gemm_max_tiles_hint(int mode);
+// Token rows per tile of a grouped GEMM for a call over T tokens, top-k K and E experts:
+// 32 when T <= 32 (no expert can have more rows), else by the average rows per expert
+// (FC1: 64 up to 48 rows, else 128, and 256 above 96 for ReLU^2; FC2: 128 up to 64
+// rows, else 256).  Narrow tiles leave shared memory for a deeper
+// weight ring.  The permute kernel's tile tables must use the same value as the launch.
+int gemm_token_tile(int mode, int T, int K, int E);
+cudaError_t launch_gemm(int mode, int bn, const GemmArgs& a, const GemmMaps& m, int grid, cudaStream_t s, bool pdl);
 
 // finalize: out = bf16(bf16(acc) + ys) or bf16(acc)
 cudaError_t launch_finalize(const float* acc, const bf16* ys, bf16* out, size_t n, int num_sms, cudaStream_t s,

@@ -97,13 +97,17 @@ def _check(st: int, where: str):
 
 
 def router_topk(logits: torch.Tensor, top_k: int, score: str = "sigmoid", bias: Optional[torch.Tensor] = None,
-                renorm: bool = True, stream=None):
-    """Router top-k on [M, E] BF16 or FP32 device logits -> (weights f32, ids i32, src i32)."""
+                renorm: bool = True, stream=None, out=None):
+    """Router top-k on [M, E] BF16 or FP32 device logits -> (weights f32, ids i32, src i32).
+    ``out``: optional preallocated (weights, ids, src) tensors of shape [M, top_k]."""
     M, E = logits.shape
     dev = logits.device
-    w = torch.empty((M, top_k), dtype=torch.float32, device=dev)
-    ids = torch.empty((M, top_k), dtype=torch.int32, device=dev)
-    src = torch.empty((M, top_k), dtype=torch.int32, device=dev)
+    if out is not None:
+        w, ids, src = out
+    else:
+        w = torch.empty((M, top_k), dtype=torch.float32, device=dev)
+        ids = torch.empty((M, top_k), dtype=torch.int32, device=dev)
+        src = torch.empty((M, top_k), dtype=torch.int32, device=dev)
     dt = DT_BF16 if logits.dtype == torch.bfloat16 else DT_FP32
     st = _lib.moe_router_topk(_ptr(logits), dt, M, E, top_k, SCORE[score], _ptr(bias), int(renorm),
                               _ptr(w), _ptr(ids), _ptr(src), _stream(stream))

@@ -7,6 +7,7 @@ import re
 import pytest
 
 import mixture_experts_layer_35_b200.moe as moe
+from mixture_experts_layer_35_b200 import inputs as gen
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -106,6 +107,16 @@ def test_path_selection_and_launch_counts():
     d = _desc(T=64, path="small")
     assert moe.select_path(d) == "small"
     assert _fwd(d, ws=FAKE * 8, ws_bytes=moe.workspace_size(d)) == moe.MOE_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("shape,T,path", [
+    ("qwen36", 1, "small"), ("qwen36", 2, "small"), ("qwen36", 4, "large"), ("qwen36", 16, "large"),
+    ("nemotron", 1, "large"), ("large_e", 1, "large"), ("tiny", 4, "small"), ("tiny", 16, "small")])
+def test_selector_follows_touched_weight_bytes(shape, T, path):
+    """The streaming path is chosen while the call's expert weights are at most 104 MB."""
+    s = gen.SHORT[shape]
+    d = _desc(T=T, H=s.H, I=s.I, E=s.E, top_k=s.K, act=s.act, score=s.score, I_shared=s.I_shared)
+    assert moe.select_path(d) == path
 
 
 def test_router_topk_and_permute_validation():
