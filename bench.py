@@ -79,23 +79,59 @@ def load_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region: a
-    thread issues one-shot queries back to back until stopped (a streaming nvidia-smi
-    killed at the end loses its buffered output)."""
+    """SM clocks and clock-event (throttle) reasons sampled during the timed region by a
+    polling thread: NVML every 2 ms on the GPU matched by PCI bus id, else one-shot
+    nvidia-smi queries back to back."""
 
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
     REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+    NVML_BITS = (0x8, 0x40, 0x20, 0x4)  # the same reasons as NVML clock-event bits
 
     def __init__(self, gpu_index: int):
         import threading
         self.idx = gpu_index
         self.rows = []
         self.raw = []
+        self.source = "nvidia-smi"
+        self._nvml = self._nvml_handle(gpu_index)
         self._stop = threading.Event()
         self._t = threading.Thread(target=self._loop, daemon=True)
         self._t.start()
+
+    @staticmethod
+    def _nvml_handle(gpu_index):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(gpu_index)
+        except Exception:  # no NVML binding: fall back to nvidia-smi
+            return None
+        try:
+            return pynvml, pynvml.nvmlDeviceGetHandleByUUID("GPU-" + str(props.uuid))
+        except Exception:
+            pass
+        try:
+            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return None
+
+    def _query_nvml(self):
+        nv, h = self._nvml
+        try:
+            sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+            mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+            pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+            getr = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                nv.nvmlDeviceGetCurrentClocksThrottleReasons
+            bits = getr(h)
+        except Exception:
+            return False
+        act = ["Active" if bits & b else "Not Active" for b in self.NVML_BITS]
+        self.rows.append([str(sm), str(mx), f"{pw:.1f}", hex(bits)] + act)
+        return True
 
     def _query(self):
         try:
@@ -111,7 +147,11 @@ class ClockSampler:
 
     def _loop(self):
         while not self._stop.is_set():
-            self._query()
+            if self._nvml is not None and self._query_nvml():
+                self.source = "nvml"
+                time.sleep(0.002)
+            else:
+                self._query()
 
     def stop(self):
         self._stop.set()
@@ -129,7 +169,7 @@ class ClockSampler:
         mx = [v for v in (num(r[1]) for r in self.rows) if v is not None]
         reasons = sorted({n for r in self.rows for n, v in zip(self.REASONS, r[4:8]) if v == "Active"})
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(self.rows)}
+                "reasons": reasons, "samples": len(self.rows), "source": self.source}
 
 
 # ---------------------------------------------------------------- algorithmic accounting

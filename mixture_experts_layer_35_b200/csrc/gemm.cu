@@ -44,7 +44,7 @@ constexpr int BBOX = 16;              // token rows per TMA box of the B operand
 // deeper weight ring.
 template <int MODE>
 constexpr int default_bn() {
-    return MODE == GM_FC2 ? 256 : 128;
+    return MODE == GM_FC2 ? 256 : (MODE == GM_DENSE ? kDenseTokenTile : 128);
 }
 
 template <int MODE, int BN>
@@ -59,9 +59,10 @@ struct Cfg {
     // mainloop, so with wide tiles it gets two warps per TMEM lane quarter, splitting the
     // token columns.
     static constexpr int kEpiWarps = (MODE == GM_FC2 && BN > 32) ? 8 : 4;
-    // FC2: per half of the epilogue warps, two [32 tokens][128 features] FP32 staging
-    // blocks for the bulk reduce-add into acc.
-    static constexpr int kEpiBytes = (MODE == GM_FC2) ? (kEpiWarps / 4) * 2 * 32 * 128 * 4 : 0;
+    // FC2: per half of the epilogue warps, two [16 tokens][128 features] FP32 staging
+    // blocks (double buffer) for the bulk reduce-add into acc.
+    static constexpr int kEpiRows = 16;
+    static constexpr int kEpiBytes = (MODE == GM_FC2) ? (kEpiWarps / 4) * 2 * kEpiRows * 128 * 4 : 0;
     static constexpr int kAccCols = kSwiglu ? 2 * kBN : kBN;
     // Two accumulator buffers (the epilogue of one tile overlaps the next mainloop) when
     // they fit TMEM's 512 columns; a 256-token SwiGLU tile (gate + up = 512 columns) has one.
@@ -92,13 +93,14 @@ struct Cfg {
 
 struct TileInfo {
     int g, ft, n, row0, shared;
+    int nk;  // k-blocks of this tile
 };
 
 template <int BN>
 __device__ __forceinline__ TileInfo decode_tile(const GemmArgs& a, const int* s_tiles, const int* s_offs, int G,
                                                 int tile) {
     TileInfo ti;
-    if (a.dense) {
+    if (a.dense) {  // tile = (feature tile, token tile), token tile fastest
         const int ntok = cdiv(a.T, kDenseTokenTile);
         ti.g = 0;
         ti.ft = tile / ntok;
@@ -106,6 +108,7 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmArgs& a, const int* s_
         ti.row0 = tt * kDenseTokenTile;
         ti.n = min(kDenseTokenTile, a.T - ti.row0);
         ti.shared = 0;
+        ti.nk = cdiv(a.kdim, BK);
         return ti;
     }
     int lo = 0, hi = G;
@@ -125,6 +128,7 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmArgs& a, const int* s_
     ti.row0 = (sh ? 0 : s_offs[g]) + tt * BN;
     ti.n = min(BN, rows - tt * BN);
     ti.shared = sh;
+    ti.nk = cdiv(sh ? a.kdim_s : a.kdim, BK);
     return ti;
 }
 
@@ -201,12 +205,10 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
                 const bool sh = ti.shared;
                 const CUtensorMap* ta = sh ? &tm_a_s : &tm_a_r;
                 const CUtensorMap* tb = sh ? &tm_b_s : &tm_b_r;
-                const int kd = sh ? a.kdim_s : a.kdim;
-                const int nk = cdiv(kd, BK);
                 const int frow = ti.ft * BM;
                 const int nbox = cdiv(ti.n, BBOX);
                 const uint32_t bytes = C::kNA * A_BYTES + (C::kGather ? 0u : (uint32_t)nbox * BBOX * BK * 2);
-                for (int kb = 0; kb < nk; ++kb, ++it) {
+                for (int kb = 0; kb < ti.nk; ++kb, ++it) {
                     const int s = it % C::kStages;
                     const uint32_t ph = (uint32_t)(it / C::kStages) & 1u;
                     if (!mbar_wait(empty_bar(s), ph ^ 1u, abort_flag, a.err)) break;
@@ -236,8 +238,7 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
             int it = 0, tcount = 0;
             for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x, ++tcount) {
                 const TileInfo ti = decode_tile<C::kBN>(a, s_tiles, s_offs, G, tile);
-                const int kd = ti.shared ? a.kdim_s : a.kdim;
-                const int nk = cdiv(kd, BK);
+                const int nk = ti.nk;
                 const int npad = cdiv(ti.n, 16) * 16;
                 const uint32_t idesc = idesc_bf16_f32(BM, npad);
                 const int buf = tcount % C::kAccBufs;
@@ -352,30 +353,36 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
                                 a.ys[(size_t)(ti.row0 + col) * a.feat_s + f] = __float2bfloat16_rn(__uint_as_float(v[j]));
                         }
                     } else {
-                        // Column j of this chunk is token t_j with routing weight w_j.  The
-                        // four epilogue warps of this half stage w_j * y[f, j] as rows
-                        // [j][128 features] in shared memory; then one thread per row
-                        // reduce-adds the whole 512-byte row into acc[t_j, f0 .. f0+127] with
-                        // one asynchronous bulk reduction (FP32 add in L2).
-                        float* stg = epi_stage + (size_t)(half * 2 + ebuf) * 32 * 128;
-                        bulk_wait_read<1>();           // my reduces from this buffer's last use have read it
-                        named_barrier(1 + half, 128);  // ... and everybody else's
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            const float w = __shfl_sync(0xffffffffu, mw[ci], j);
-                            stg[j * 128 + q * 32 + lane] = w * __uint_as_float(v[j]);
-                        }
-                        fence_proxy_async_smem();
-                        named_barrier(1 + half, 128);
-                        const int r = q * 8 + (lane & 7);  // row issued by this thread
-                        const int t_r = __shfl_sync(0xffffffffu, mt[ci], r);
+                        // Column j of this chunk is token t_j with routing weight w_j.  In two
+                        // passes of 16 columns, the four epilogue warps of this half stage
+                        // w_j * y[f, j] as rows [j][128 features] in shared memory; then one
+                        // thread per row reduce-adds the whole 512-byte row into
+                        // acc[t_j, f0 .. f0+127] with one asynchronous bulk reduction (FP32
+                        // add in L2).
                         const int fb = ti.ft * BM;
                         const int nfe = min(BM, a.feat_r - fb);
-                        if (lane < 8 && c0 + r < ti.n && nfe > 0)  // acc stays in L2 across the K adds
-                            bulk_reduce_add_f32_hint(a.acc + (size_t)t_r * a.feat_r + fb, smem_u32(stg + r * 128),
-                                                     (uint32_t)nfe * 4u, acc_pol);
-                        bulk_commit();
-                        ebuf ^= 1;
+#pragma unroll
+                        for (int ps = 0; ps < 32 / C::kEpiRows; ++ps) {
+                            float* stg = epi_stage + (size_t)(half * 2 + ebuf) * C::kEpiRows * 128;
+                            bulk_wait_read<1>();           // my reduces from this buffer's last use have read it
+                            named_barrier(1 + half, 128);  // ... and everybody else's
+#pragma unroll
+                            for (int jj = 0; jj < C::kEpiRows; ++jj) {
+                                const int j = ps * C::kEpiRows + jj;
+                                const float w = __shfl_sync(0xffffffffu, mw[ci], j);
+                                stg[jj * 128 + q * 32 + lane] = w * __uint_as_float(v[j]);
+                            }
+                            fence_proxy_async_smem();
+                            named_barrier(1 + half, 128);
+                            const int r = q * (C::kEpiRows / 4) + (lane & (C::kEpiRows / 4 - 1));  // my row
+                            const int t_r = __shfl_sync(0xffffffffu, mt[ci], ps * C::kEpiRows + r);
+                            if (lane < C::kEpiRows / 4 && c0 + ps * C::kEpiRows + r < ti.n && nfe > 0)
+                                // acc stays in L2 across the K adds
+                                bulk_reduce_add_f32_hint(a.acc + (size_t)t_r * a.feat_r + fb,
+                                                         smem_u32(stg + r * 128), (uint32_t)nfe * 4u, acc_pol);
+                            bulk_commit();
+                            ebuf ^= 1;
+                        }
                     }
                 } else {  // GM_DENSE
 #pragma unroll
@@ -501,7 +508,9 @@ int gemm_token_tile(int mode, int T, int K, int E) {
     if (mode == GM_DENSE) return default_bn<GM_DENSE>();
     if (T <= 32) return 32;  // no expert has more rows than a tile
     const double rows = (double)T * K / E;  // average rows per expert
-    if (mode == GM_FC2) return rows <= 64.0 ? 128 : 256;  // measured: 256 ahead from ~128 rows
+    // FC2: a tile that covers an expert's rows streams its W2 slice once; 192 still holds
+    // almost every expert at ~128 rows and leaves room for a 4th stage.
+    if (mode == GM_FC2) return rows <= 64.0 ? 128 : (rows <= 150.0 ? 192 : 256);
     // FC1: a tile re-streams the expert's weight slice, so an expert just over a tile's
     // width costs a second, nearly empty tile; 256-token tiles keep most experts at one.
     // Not for SwiGLU: its 256-token stage (64 KB) leaves room for only 3 stages, and the
@@ -527,6 +536,7 @@ cudaError_t launch_gemm(int mode, int bn, const GemmArgs& a, const GemmMaps& m, 
         case GM_FC2:
             if (bn == 32) return launch_mode<GM_FC2, 32>(a, m, grid, s, pdl);
             if (bn == 128) return launch_mode<GM_FC2, 128>(a, m, grid, s, pdl);
+            if (bn == 192) return launch_mode<GM_FC2, 192>(a, m, grid, s, pdl);
             if (bn == 256) return launch_mode<GM_FC2, 256>(a, m, grid, s, pdl);
             break;
         case GM_DENSE: return launch_mode<GM_DENSE, default_bn<GM_DENSE>()>(a, m, grid, s, pdl);

@@ -103,8 +103,9 @@ cudaError_t launch_permute_fast(const PermuteArgs& a, const int* counts, int* cu
 
 // ---------------------------------------------------------------- grouped tcgen05 GEMM
 enum GemmMode { GM_FC1_SWIGLU = 0, GM_FC1_RELU2 = 1, GM_FC2 = 2, GM_DENSE = 3 };
-// Token rows per tile of the dense router GEMM (E is small, so smaller token tiles give
-// the grid more CTAs).  The grouped FC1 / FC2 GEMMs take gemm_token_tile(mode, T).
+// Token rows per tile of the dense router GEMM (E is small, so narrow token tiles give the
+// grid its width; measured: 256-token tiles with split-K and FP32 atomics into the logits
+// were 3x slower).  The grouped FC1 / FC2 GEMMs take gemm_token_tile(mode, T, K, E).
 static constexpr int kDenseTokenTile = 64;
 struct GemmArgs {
     int T, K;            // tokens and top-k (slot decode of perm entries)
