@@ -208,8 +208,8 @@ def kernel_names(path: str, router: bool):
 # The capture and its command are summarised in profiles/; an entry is removed whenever
 # its kernel changes, so that a stale count is never reported.
 NCU_TRAFFIC = {
-    ("qwen36", 4096, "router", "fc1"): 1.251730e9 + 65.964032e6,
-    ("qwen36", 4096, "router", "fc2"): 0.635051e9 + 12.244736e6,
+    ("qwen36", 4096, "router", "fc1"): 1.259206e9 + 65.595392e6,
+    ("qwen36", 4096, "router", "fc2"): 0.634541e9 + 10.745600e6,
 }
 
 
