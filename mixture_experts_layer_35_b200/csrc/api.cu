@@ -241,7 +241,7 @@ int moe_fused_forward_launches(const moe_layer_desc* d) {
     if (validate_desc(d) != MOE_OK || d->T == 0) return 0;
     const int router = d->router_logits ? 0 : 1;
     if (resolve_path(d) == MOE_PATH_SMALL) return router + 3;  // route table, fc1, fc2
-    return router + 5;  // topk, permute, fc1, fc2, finalize
+    return router + 5;                                          // topk, permute, fc1, fc2, finalize
 }
 
 static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, void* out_, float* topk_w_out,
@@ -343,6 +343,9 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
     bf16* ys = Is ? reinterpret_cast<bf16*>(w8 + L.ys) : nullptr;
 
     const bool chain = !timed;  // programmatic overlap between consecutive kernels
+    const bool swiglu = d->act == MOE_ACT_SWIGLU;
+    const int fc1_mode = swiglu ? GM_FC1_SWIGLU : GM_FC1_RELU2;
+    const int bn1 = gemm_token_tile(fc1_mode, T, K, E), bn2 = gemm_token_tile(GM_FC2, T, K, E);
     // 2. top-k (also counts the slots per expert)
     MOE_CK(cudaMemsetAsync(counts, 0, 2 * (size_t)(E + 2) * sizeof(int), s));
     if (!mark()) return MOE_ERR_CUDA;
@@ -350,7 +353,6 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
     MOE_CK(launch_topk(logits, false, T, E, K, d->score, d->bias, d->renorm, tw, tid, nullptr, topk_w_out,
                        topk_ids_out, s, pdl && chain, dense_router ? &ra : nullptr, counts));
     // 3. permutation + tile tables
-    const bool swiglu = d->act == MOE_ACT_SWIGLU;
     PermuteArgs pa;
     std::memset(&pa, 0, sizeof(pa));
     pa.ids = tid;
@@ -361,8 +363,6 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
     pa.perm = perm;
     pa.err = err;
     pa.has_shared = Is > 0;
-    const int fc1_mode = swiglu ? GM_FC1_SWIGLU : GM_FC1_RELU2;
-    const int bn1 = gemm_token_tile(fc1_mode, T, K, E), bn2 = gemm_token_tile(GM_FC2, T, K, E);
     pa.bn1 = bn1;
     pa.bn2 = bn2;
     pa.nfeat1_r = cdiv(I, 128);

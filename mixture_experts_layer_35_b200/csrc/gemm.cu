@@ -289,7 +289,8 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
         const uint64_t acc_pol = l2_policy_evict_last();
         // (the abort flag is checked through the per-tile wait and vote below, so that the
         // epilogue warps always take the same number of tiles)
-        constexpr int kChunks = C::kBN / (32 * (C::kEpiWarps / 4));
+        // 32-token chunks per half of the epilogue warps (the last may lie past the tile)
+        constexpr int kChunks = (C::kBN + 32 * (C::kEpiWarps / 4) - 1) / (32 * (C::kEpiWarps / 4));
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++tcount) {
             const TileInfo ti = decode_tile<C::kBN>(a, s_tiles, s_offs, G, tile);
             const int buf = tcount % C::kAccBufs;
@@ -508,8 +509,9 @@ int gemm_token_tile(int mode, int T, int K, int E) {
     if (mode == GM_DENSE) return default_bn<GM_DENSE>();
     if (T <= 32) return 32;  // no expert has more rows than a tile
     const double rows = (double)T * K / E;  // average rows per expert
-    // FC2: a tile that covers an expert's rows streams its W2 slice once; 192 still holds
-    // almost every expert at ~128 rows and leaves room for a 4th stage.
+    // FC2: a tile that covers an expert's rows streams its W2 slice once, and FC2 is bound
+    // by the bytes its ring keeps in flight: 192 holds almost every expert of ~128 rows
+    // and leaves room for 4 stages.
     if (mode == GM_FC2) return rows <= 64.0 ? 128 : (rows <= 150.0 ? 192 : 256);
     // FC1: a tile re-streams the expert's weight slice, so an expert just over a tile's
     // width costs a second, nearly empty tile; 256-token tiles keep most experts at one.

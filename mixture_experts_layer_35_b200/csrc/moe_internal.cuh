@@ -59,6 +59,18 @@ __device__ __forceinline__ double dot8_f64(const uint4& a, const uint4& b, doubl
     return acc;
 }
 
+// Eight exact BF16 products formed in FP32, accumulated in FP64.
+__device__ __forceinline__ double dot8_f64p(const uint4& a, const uint4& b, double acc) {
+    acc += (double)__fmul_rn(bf16lo(a.x), bf16lo(b.x));
+    acc += (double)__fmul_rn(bf16hi(a.x), bf16hi(b.x));
+    acc += (double)__fmul_rn(bf16lo(a.y), bf16lo(b.y));
+    acc += (double)__fmul_rn(bf16hi(a.y), bf16hi(b.y));
+    acc += (double)__fmul_rn(bf16lo(a.z), bf16lo(b.z));
+    acc += (double)__fmul_rn(bf16hi(a.z), bf16hi(b.z));
+    acc += (double)__fmul_rn(bf16lo(a.w), bf16lo(b.w));
+    acc += (double)__fmul_rn(bf16hi(a.w), bf16hi(b.w));
+    return acc;
+}
 __device__ __forceinline__ double warp_sum_f64(double v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

@@ -5,8 +5,9 @@
 
 namespace moe {
 
-// Tensor-core router logits carry an FP32 accumulation error of ~1e-6 on these
-// workloads; the routing window assumes at most this (two orders of magnitude above).
+// Tensor-core router logits carry the MMA's FP32 accumulation error: at most 1.4e-5 on
+// the T = 4096 workloads (|l| < 5, measured against the exact logits); the routing window
+// assumes at most 2e-4.
 static constexpr float kTcLogitErr = 2e-4f;
 
 struct RowRefine {
@@ -89,12 +90,13 @@ cudaError_t launch_topk(const void* logits, bool bf16_in, int M, int E, int K, i
 }
 
 // ---------------------------------------------------------------- router logits, few tokens
-// l[t, e] = x[t,:] . Wr[e,:], correctly rounded (Sum2 error-free accumulation of the exact
-// BF16 products).  CTA (i, g): two warps, one expert row each (experts 2i, 2i+1) held in
-// registers (one memory latency per row), and token group g of kRouterTokBlock tokens,
-// staged in shared memory by one bulk copy.  Each warp runs four independent Sum2 chains
-// (two tokens x even/odd chunks).  Splitting the tokens over the grid keeps the chains
-// short: the Sum2 arithmetic, not memory, would otherwise set the time at T = 16..64.
+// l[t, e] = x[t,:] . Wr[e,:]: each BF16 x BF16 product is exact in FP32 and is summed in
+// FP64, rounded once to FP32 (the oracle's definition; see warp_dot_exact).  CTA (i, g):
+// two warps, one expert row each (experts 2i, 2i+1) held in registers (one memory latency
+// per row), and token group g of kRouterTokBlock tokens, staged in shared memory by one
+// bulk copy.  Each warp runs four independent FP64 chains (two tokens x even/odd chunks).
+// Splitting the tokens over the grid keeps the chains short: the arithmetic, not memory,
+// would otherwise set the time at T = 16..64.
 static constexpr int kRouterTokBlock = 4;
 
 template <int VH>
@@ -132,28 +134,23 @@ __global__ void __launch_bounds__(64) router_logits_small(const bf16* __restrict
     if (ok && e < E) {
         for (int t = 0; t < nt; t += 2) {
             const bool two = t + 1 < nt;
-            Sum2 a0 = {0.f, 0.f}, a1 = {0.f, 0.f}, b0 = {0.f, 0.f}, b1 = {0.f, 0.f};
+            double a0 = 0.0, a1 = 0.0, b0 = 0.0, b1 = 0.0;
 #pragma unroll
             for (int j = 0; j < VH; ++j) {
                 const int c = lane + 32 * j;
                 if (c < nch) {
                     const uint4 xa = xs[t * nch + c];
-                    if (j & 1) sum2_dot8(a1, xa, w[j]);
-                    else sum2_dot8(a0, xa, w[j]);
+                    if (j & 1) a1 = dot8_f64p(xa, w[j], a1);
+                    else a0 = dot8_f64p(xa, w[j], a0);
                     if (two) {
                         const uint4 xb = xs[(t + 1) * nch + c];
-                        if (j & 1) sum2_dot8(b1, xb, w[j]);
-                        else sum2_dot8(b0, xb, w[j]);
+                        if (j & 1) b1 = dot8_f64p(xb, w[j], b1);
+                        else b0 = dot8_f64p(xb, w[j], b0);
                     }
                 }
             }
-            float q;
-            two_sum(a0.s, a1.s, a0.s, q);
-            a0.c = __fadd_rn(__fadd_rn(a0.c, a1.c), q);
-            two_sum(b0.s, b1.s, b0.s, q);
-            b0.c = __fadd_rn(__fadd_rn(b0.c, b1.c), q);
-            const float va = sum2_warp_finish(a0);
-            const float vb = sum2_warp_finish(b0);
+            const float va = __double2float_rn(warp_sum_f64(a0 + a1));
+            const float vb = __double2float_rn(warp_sum_f64(b0 + b1));
             if (lane == 0) {
                 logits[(size_t)(t0 + t) * E + e] = va;
                 if (logits_copy) logits_copy[(size_t)(t0 + t) * E + e] = va;

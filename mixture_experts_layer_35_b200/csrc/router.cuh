@@ -16,7 +16,7 @@
 // Exact values only where they decide something.  Keys are first screened in cheap FP32
 // (a fast sigmoid; logits that may carry an accumulation error `eps_l`), the K-th
 // screened key fixes a window, and only the experts inside it -- the K selected ones and
-// any close competitor -- get exact values: the logit re-evaluated by an error-free dot
+// any close competitor -- get exact values: the logit re-evaluated by an exact dot
 // product when it was approximate (`refine`), and the correctly rounded sigmoid
 // (evaluated in FP64 on those few lanes).  An expert outside the window is below every
 // selected one even after the screening errors, so the final selection over the mixed
@@ -35,66 +35,26 @@ __device__ __noinline__ double exp_f64(double v) { return exp(v); }
 // Screening sigmoid: a few ulp from the correctly rounded value.
 __device__ __forceinline__ float sigmoid_fast(float l) { return __frcp_rn(1.0f + __expf(-l)); }
 
-// ---------------------------------------------------------------- error-free dot product
-// Sum2 of Ogita, Rump and Oishi ("Accurate sum and dot product", SIAM J. Sci. Comput.
-// 26(6), 2005): each BF16 x BF16 product is exact in FP32 (8-bit significands); the
-// running sum takes it with Knuth's TwoSum, whose rounding error is exact and collected
-// in a second FP32 term.  The pair (s, c) carries the sum with about twice FP32's
-// precision; s + c rounded once is the correctly rounded dot product except within
-// ~1e-12 (relative) of an FP32 rounding midpoint.
-__device__ __forceinline__ void two_sum(float a, float b, float& s, float& e) {
-    s = __fadd_rn(a, b);
-    const float bb = __fsub_rn(s, a);
-    e = __fadd_rn(__fsub_rn(a, __fsub_rn(s, bb)), __fsub_rn(b, bb));
-}
-struct Sum2 {
-    float s, c;
-};
-__device__ __forceinline__ void sum2_add(Sum2& a, float p) {
-    float q;
-    two_sum(a.s, p, a.s, q);
-    a.c = __fadd_rn(a.c, q);
-}
-__device__ __forceinline__ void sum2_dot8(Sum2& a, const uint4& x, const uint4& w) {
-    sum2_add(a, __fmul_rn(bf16lo(x.x), bf16lo(w.x)));
-    sum2_add(a, __fmul_rn(bf16hi(x.x), bf16hi(w.x)));
-    sum2_add(a, __fmul_rn(bf16lo(x.y), bf16lo(w.y)));
-    sum2_add(a, __fmul_rn(bf16hi(x.y), bf16hi(w.y)));
-    sum2_add(a, __fmul_rn(bf16lo(x.z), bf16lo(w.z)));
-    sum2_add(a, __fmul_rn(bf16hi(x.z), bf16hi(w.z)));
-    sum2_add(a, __fmul_rn(bf16lo(x.w), bf16lo(w.w)));
-    sum2_add(a, __fmul_rn(bf16hi(x.w), bf16hi(w.w)));
-}
-// Combine the lanes' pairs with TwoSum; every lane ends with the same bits (TwoSum's
-// error term is unique, and the remaining adds are commutative pairs).
-__device__ __forceinline__ float sum2_warp_finish(Sum2 a) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        const float s2 = __shfl_xor_sync(0xffffffffu, a.s, o);
-        const float c2 = __shfl_xor_sync(0xffffffffu, a.c, o);
-        float q;
-        two_sum(a.s, s2, a.s, q);
-        a.c = __fadd_rn(__fadd_rn(a.c, c2), q);
-    }
-    return __fadd_rn(a.s, a.c);
-}
-// Warp-collective correctly rounded dot product of two BF16 rows of length H (H % 8 == 0).
+// ---------------------------------------------------------------- exact dot product
+// Warp-collective dot product of two BF16 rows of length H (H % 8 == 0), rounded once to
+// FP32.  Each BF16 x BF16 product is exact in FP32 and is accumulated in FP64 (error about
+// H * 2^-53 * sum|p|, far below half an FP32 ulp of the result except within that distance
+// of a rounding midpoint, where the oracle's own FP64 sum has the same blind spot).  FP64
+// runs at half the FP32 rate here, so one conversion and one add per product cost less
+// than a compensated (TwoSum) FP32 accumulation, which measured slower.
 __device__ __noinline__ float warp_dot_exact(const bf16* __restrict__ a, const bf16* __restrict__ b, int H,
                                                 int lane) {
     const int nch = H >> 3;
-    Sum2 acc0 = {0.f, 0.f}, acc1 = {0.f, 0.f};
+    double acc0 = 0.0, acc1 = 0.0;
     int q = lane;
     for (; q + 32 < nch; q += 64) {
         const uint4 a0 = ld_nc16(a + (size_t)q * 8), b0 = ld_nc16(b + (size_t)q * 8);
         const uint4 a1 = ld_nc16(a + (size_t)(q + 32) * 8), b1 = ld_nc16(b + (size_t)(q + 32) * 8);
-        sum2_dot8(acc0, a0, b0);
-        sum2_dot8(acc1, a1, b1);
+        acc0 = dot8_f64p(a0, b0, acc0);
+        acc1 = dot8_f64p(a1, b1, acc1);
     }
-    if (q < nch) sum2_dot8(acc0, ld_nc16(a + (size_t)q * 8), ld_nc16(b + (size_t)q * 8));
-    float e;
-    two_sum(acc0.s, acc1.s, acc0.s, e);
-    acc0.c = __fadd_rn(__fadd_rn(acc0.c, acc1.c), e);
-    return sum2_warp_finish(acc0);
+    if (q < nch) acc0 = dot8_f64p(ld_nc16(a + (size_t)q * 8), ld_nc16(b + (size_t)q * 8), acc0);
+    return __double2float_rn(warp_sum_f64(acc0 + acc1));
 }
 
 // ---------------------------------------------------------------- selection

@@ -104,6 +104,7 @@ def test_path_selection_and_launch_counts():
     assert moe.launches(d) == 6
     d = _desc(T=4, path="large")
     assert moe.select_path(d) == "large"
+    assert moe.launches(d) == 6
     d = _desc(T=64, path="small")
     assert moe.select_path(d) == "small"
     assert _fwd(d, ws=FAKE * 8, ws_bytes=moe.workspace_size(d)) == moe.MOE_ERR_UNSUPPORTED
