@@ -12,9 +12,9 @@
 //       the expert's tokens gathered row by row from x with cp.async into the swizzled
 //       layout; epilogue applies SwiGLU / ReLU^2 and stores h (BF16) in permuted order.
 //   FC2: A = W2[e] rows of 128 output features, B = the expert's contiguous h rows
-//       (TMA, 16-row boxes); epilogue scales by the routing weight, stages the block in
-//       shared memory and adds it into the FP32 accumulator acc[t, :] with asynchronous
-//       bulk reduce-adds, one 512-byte row (128 features) per token ("weighted output
+//       (TMA, 16-row boxes); epilogue scales by the routing weight, transposes 4x4 blocks
+//       within groups of 4 lanes and adds into the FP32 accumulator acc[t, :] with 16-byte
+//       vector reductions, 4 consecutive features of one token per lane ("weighted output
 //       combination").
 //       The shared expert is one more group whose FC2 output is rounded to BF16 into ys.
 //   DENSE: router logits, A = Wr (128 experts per tile), B = x rows (TMA).
@@ -59,10 +59,7 @@ struct Cfg {
     // mainloop, so with wide tiles it gets two warps per TMEM lane quarter, splitting the
     // token columns.
     static constexpr int kEpiWarps = (MODE == GM_FC2 && BN > 32) ? 8 : 4;
-    // FC2: per half of the epilogue warps, two [16 tokens][128 features] FP32 staging
-    // blocks (double buffer) for the bulk reduce-add into acc.
-    static constexpr int kEpiRows = 16;
-    static constexpr int kEpiBytes = (MODE == GM_FC2) ? (kEpiWarps / 4) * 2 * kEpiRows * 128 * 4 : 0;
+    static constexpr int kEpiBytes = 0;  // epilogues work from registers
     static constexpr int kAccCols = kSwiglu ? 2 * kBN : kBN;
     // Two accumulator buffers (the epilogue of one tile overlaps the next mainloop) when
     // they fit TMEM's 512 columns; a 256-token SwiGLU tile (gate + up = 512 columns) has one.
@@ -141,7 +138,6 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
     const uint32_t raw_u32 = smem_u32(smem_raw);
     const uint32_t base_u32 = (raw_u32 + 1023u) & ~1023u;
     uint8_t* base = smem_raw + (base_u32 - raw_u32);
-    float* epi_stage = reinterpret_cast<float*>(base + (size_t)C::kStages * C::kStageBytes);
     uint8_t* meta = base + (size_t)C::kStages * C::kStageBytes + C::kEpiBytes;
     uint64_t* bars = reinterpret_cast<uint64_t*>(meta);  // full[S], empty[S], tfull[2], tempty[2]
     const uint32_t bar_u32 = smem_u32(bars);
@@ -285,8 +281,6 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
                 z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
         int tcount = 0;
-        int ebuf = 0;
-        const uint64_t acc_pol = l2_policy_evict_last();
         // (the abort flag is checked through the per-tile wait and vote below, so that the
         // epilogue warps always take the same number of tiles)
         // 32-token chunks per half of the epilogue warps (the last may lie past the tile)
@@ -312,12 +306,7 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
                 }
             }
             const bool waited = mbar_wait(tfull_bar(buf), tph, abort_flag, a.err);
-            if (MODE == GM_FC2) {
-                // the FC2 epilogue warps meet at named barriers below: leave together or not at all
-                if (named_barrier_or(1 + half, 128, !waited || *abort_flag)) break;
-            } else if (!waited) {
-                break;
-            }
+            if (!waited) break;
             tc_fence_after();
             const int f = ti.ft * BM + q * 32 + lane;
             const int feat = ti.shared ? a.feat_s : a.feat_r;
@@ -354,35 +343,44 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
                                 a.ys[(size_t)(ti.row0 + col) * a.feat_s + f] = __float2bfloat16_rn(__uint_as_float(v[j]));
                         }
                     } else {
-                        // Column j of this chunk is token t_j with routing weight w_j.  In two
-                        // passes of 16 columns, the four epilogue warps of this half stage
-                        // w_j * y[f, j] as rows [j][128 features] in shared memory; then one
-                        // thread per row reduce-adds the whole 512-byte row into
-                        // acc[t_j, f0 .. f0+127] with one asynchronous bulk reduction (FP32
-                        // add in L2).
-                        const int fb = ti.ft * BM;
-                        const int nfe = min(BM, a.feat_r - fb);
+                        // Column j of this chunk is token t_j with routing weight w_j; lane l
+                        // holds feature f0 + l.  Each block of 4 columns is transposed within
+                        // groups of 4 lanes (two XOR-shuffle stages), after which lane 4g+i
+                        // holds features f0+4g .. f0+4g+3 of token t_{j0+i} and adds them into
+                        // acc with one 16-byte vector reduction (FP32 add in L2).  No shared
+                        // memory is staged, so the ring keeps it for weights.
+                        const int i4 = lane & 3;
+                        const bool fok4 = f - i4 + 3 < a.feat_r;  // features of my group (feat_r % 8 == 0)
 #pragma unroll
-                        for (int ps = 0; ps < 32 / C::kEpiRows; ++ps) {
-                            float* stg = epi_stage + (size_t)(half * 2 + ebuf) * C::kEpiRows * 128;
-                            bulk_wait_read<1>();           // my reduces from this buffer's last use have read it
-                            named_barrier(1 + half, 128);  // ... and everybody else's
+                        for (int j0 = 0; j0 < 32; j0 += 4) {
+                            float r[4];
 #pragma unroll
-                            for (int jj = 0; jj < C::kEpiRows; ++jj) {
-                                const int j = ps * C::kEpiRows + jj;
-                                const float w = __shfl_sync(0xffffffffu, mw[ci], j);
-                                stg[jj * 128 + q * 32 + lane] = w * __uint_as_float(v[j]);
+                            for (int jj = 0; jj < 4; ++jj)
+                                r[jj] = __shfl_sync(0xffffffffu, mw[ci], j0 + jj) * __uint_as_float(v[j0 + jj]);
+                            // r[jj] = w_j * y[feature of this lane, token j0 + jj]; 4x4 transpose
+                            float t0 = (i4 & 1) ? r[0] : r[1], t1 = (i4 & 1) ? r[2] : r[3];
+                            t0 = __shfl_xor_sync(0xffffffffu, t0, 1);
+                            t1 = __shfl_xor_sync(0xffffffffu, t1, 1);
+                            if (i4 & 1) {
+                                r[0] = t0;
+                                r[2] = t1;
+                            } else {
+                                r[1] = t0;
+                                r[3] = t1;
                             }
-                            fence_proxy_async_smem();
-                            named_barrier(1 + half, 128);
-                            const int r = q * (C::kEpiRows / 4) + (lane & (C::kEpiRows / 4 - 1));  // my row
-                            const int t_r = __shfl_sync(0xffffffffu, mt[ci], ps * C::kEpiRows + r);
-                            if (lane < C::kEpiRows / 4 && c0 + ps * C::kEpiRows + r < ti.n && nfe > 0)
-                                // acc stays in L2 across the K adds
-                                bulk_reduce_add_f32_hint(a.acc + (size_t)t_r * a.feat_r + fb,
-                                                         smem_u32(stg + r * 128), (uint32_t)nfe * 4u, acc_pol);
-                            bulk_commit();
-                            ebuf ^= 1;
+                            float u0 = (i4 & 2) ? r[0] : r[2], u1 = (i4 & 2) ? r[1] : r[3];
+                            u0 = __shfl_xor_sync(0xffffffffu, u0, 2);
+                            u1 = __shfl_xor_sync(0xffffffffu, u1, 2);
+                            if (i4 & 2) {
+                                r[0] = u0;
+                                r[1] = u1;
+                            } else {
+                                r[2] = u0;
+                                r[3] = u1;
+                            }
+                            const int tok = __shfl_sync(0xffffffffu, mt[ci], j0 + i4);
+                            if (c0 + j0 + i4 < ti.n && fok4)
+                                red_add_v4_f32(a.acc + (size_t)tok * a.feat_r + (f - i4), r[0], r[1], r[2], r[3]);
                         }
                     }
                 } else {  // GM_DENSE
@@ -401,7 +399,6 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(tempty_bar(buf));
         }
-        if (MODE == GM_FC2) bulk_wait_all<0>();  // every reduce-add issued by this thread has landed
     } else if (C::kGather) {
         // ------------------------------------------------------------ FC1 token gather
         const int p = threadIdx.x - 192;  // 0..127

@@ -253,6 +253,11 @@ __device__ __forceinline__ void bulk_reduce_add_f32_hint(float* gdst, uint32_t s
                  "r"(ssrc), "r"(bytes), "l"(pol)
                  : "memory");
 }
+// 16-byte vector reduction (FP32 add) into global memory; p 16-byte aligned.
+__device__ __forceinline__ void red_add_v4_f32(float* p, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void bulk_wait_read() {
