@@ -381,6 +381,7 @@ def run_ours(args, rank, local, world):
     e2e_total = max_over_ranks(float(sum(e2e_ms)), world, device)
     e2e_value = world * args.T * args.steps / (e2e_total / 1e3)
 
+    dev_err = b.moe.get_error(b.ws)
     line = {
         "metric": METRIC,
         "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -396,6 +397,7 @@ def run_ours(args, rank, local, world):
         "kernel_ms": {n: round(float(v), 5) for n, v in zip(names, kt)},
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo},
         "gpu_launches": b.launches * args.steps,
+        "device_error": dev_err,
         "clocks": clk,
         "us_per_step_p10_p50_p90": [float(np.percentile(per, q)) * 1e3 for q in (10, 50, 90)],
     }
@@ -425,6 +427,7 @@ def sweep(args, device, peaks):
     cache = {}
     for cfg, T in plan:
         shape = gen.SHORT[cfg]
+        print(f"sweep: {cfg} T={T}", file=sys.stderr, flush=True)
         try:
             b = Bench(shape, T, device, seed=1, routing="router", path=args.path)
             per, _ = b.timed(8, 2)
@@ -434,7 +437,8 @@ def sweep(args, device, peaks):
             rf = roofline_of(acc, med / 1e3, peaks)
             rows.append({"config": cfg, "T": T, "path": b.path, "us": med * 1e3, "tokens_per_s": T / (med / 1e3),
                          "distinct_experts": U, "bound": rf["bound"], "frac_of_roofline": rf["frac"],
-                         "achieved": rf["achieved"], "unit": rf["unit"]})
+                         "achieved": rf["achieved"], "unit": rf["unit"],
+                         "device_error": b.moe.get_error(b.ws)})
             del b
         except Exception as e:  # report, keep sweeping
             rows.append({"config": cfg, "T": T, "error": str(e)[:200]})

@@ -58,6 +58,7 @@ typedef enum { MOE_PATH_AUTO = 0, MOE_PATH_SMALL = 1, MOE_PATH_LARGE = 2 } moe_p
 /* Device error codes written to the workspace error word. */
 #define MOE_DEVERR_BAD_EXPERT_ID 0x1   /* an expert id outside [0, E) reached the permute */
 #define MOE_DEVERR_WAIT_TIMEOUT 0x2    /* a bounded device-side wait gave up */
+#define MOE_DEVERR_BAD_INDEX 0x4       /* a computed row/slot index fell outside its buffer; the access was skipped */
 
 /* Limits of this build. */
 #define MOE_MAX_EXPERTS 1024

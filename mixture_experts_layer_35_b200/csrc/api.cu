@@ -275,6 +275,12 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
     const int T = d->T, H = d->H, I = d->I, E = d->E, K = d->top_k, Is = d->I_shared;
     const int sms = num_sms();
 
+    // 0. the many-token path's slot counters start at zero.  Cleared before the first
+    // kernel, so that every kernel launched with programmatic overlap follows a kernel
+    // (a memset between two kernels would leave the second one's overlap undefined).
+    if (path == MOE_PATH_LARGE)
+        MOE_CK(cudaMemsetAsync(w8 + L.counts, 0, 2 * (size_t)(E + 2) * sizeof(int), s));
+
     // 1. router logits
     const float* logits = d->router_logits;
     bool pdl = false;
@@ -346,8 +352,7 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
     const bool swiglu = d->act == MOE_ACT_SWIGLU;
     const int fc1_mode = swiglu ? GM_FC1_SWIGLU : GM_FC1_RELU2;
     const int bn1 = gemm_token_tile(fc1_mode, T, K, E), bn2 = gemm_token_tile(GM_FC2, T, K, E);
-    // 2. top-k (also counts the slots per expert)
-    MOE_CK(cudaMemsetAsync(counts, 0, 2 * (size_t)(E + 2) * sizeof(int), s));
+    // 2. top-k (also counts the slots per expert; the counters were cleared in step 0)
     if (!mark()) return MOE_ERR_CUDA;
     RefineArgs ra = {x, static_cast<const bf16*>(d->router_w), H, logits_rw};
     MOE_CK(launch_topk(logits, false, T, E, K, d->score, d->bias, d->renorm, tw, tid, nullptr, topk_w_out,

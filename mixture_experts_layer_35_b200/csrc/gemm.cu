@@ -298,16 +298,24 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
                 mt[ci] = 0;
                 mw[ci] = 0.0f;
                 const int colm = 32 * half + 32 * nhalf * ci + lane;
-                if (MODE == GM_FC2 && !ti.shared && colm < ti.n) {
+                if (MODE == GM_FC2 && !ti.shared && colm < ti.n && ti.row0 + ti.n <= a.T * a.K) {
                     const int src = a.perm[ti.row0 + colm];
-                    const int kk = src / a.T;
-                    mt[ci] = src - kk * a.T;
-                    mw[ci] = a.topk_w[(size_t)mt[ci] * a.K + kk];
+                    if ((unsigned)src < (unsigned)(a.T * a.K)) {
+                        const int kk = src / a.T;
+                        mt[ci] = src - kk * a.T;
+                        mw[ci] = a.topk_w[(size_t)mt[ci] * a.K + kk];
+                    } else {  // never from a valid permutation: flag it, contribute nothing
+                        set_dev_error(a.err, MOE_DEVERR_BAD_INDEX);
+                    }
                 }
             }
             const bool waited = mbar_wait(tfull_bar(buf), tph, abort_flag, a.err);
             if (!waited) break;
             tc_fence_after();
+            // The tile's rows must lie inside their buffer (they do for any permutation the
+            // permute kernel writes); otherwise flag it and store nothing for this tile.
+            const bool rows_ok = a.dense || ti.row0 + ti.n <= (ti.shared ? a.T : a.T * a.K);
+            if (!rows_ok && lane == 0) set_dev_error(a.err, MOE_DEVERR_BAD_INDEX);
             const int f = ti.ft * BM + q * 32 + lane;
             const int feat = ti.shared ? a.feat_s : a.feat_r;
             const bool fok = f < feat;
@@ -315,7 +323,7 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
 #pragma unroll
             for (int ci = 0; ci < kChunks; ++ci) {
                 const int c0 = 32 * half + 32 * nhalf * ci;
-                if (c0 >= ti.n) break;
+                if (c0 >= ti.n || !rows_ok) break;
                 uint32_t v[32];
                 tmem_ld32(tb + c0, v);
                 uint32_t u[32];
@@ -379,7 +387,7 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
                                 r[3] = u1;
                             }
                             const int tok = __shfl_sync(0xffffffffu, mt[ci], j0 + i4);
-                            if (c0 + j0 + i4 < ti.n && fok4)
+                            if (c0 + j0 + i4 < ti.n && fok4 && (unsigned)tok < (unsigned)a.T)
                                 red_add_v4_f32(a.acc + (size_t)tok * a.feat_r + (f - i4), r[0], r[1], r[2], r[3]);
                         }
                     }
@@ -414,7 +422,14 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
             for (int j = 0; j < C::kBN / 16; ++j) {
                 const int r = rsub + 16 * j;
                 tok[j] = -1;
-                if (r < ti.n) tok[j] = ti.shared ? ti.row0 + r : (a.perm[ti.row0 + r] % a.T);
+                if (r < ti.n && (ti.shared || ti.row0 + ti.n <= a.T * a.K)) {
+                    const int src = ti.shared ? ti.row0 + r : a.perm[ti.row0 + r];
+                    if ((unsigned)src < (unsigned)(ti.shared ? a.T : a.T * a.K)) {
+                        tok[j] = ti.shared ? src : src % a.T;
+                    } else {  // never from a valid permutation: flag it, gather zeros
+                        set_dev_error(a.err, MOE_DEVERR_BAD_INDEX);
+                    }
+                }
             }
             bool ok = true;
             for (int kb = 0; kb < nk; ++kb, ++it) {

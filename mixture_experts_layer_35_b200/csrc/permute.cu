@@ -151,8 +151,12 @@ __global__ void __launch_bounds__(kThreads) permute_fast_kernel(const PermuteArg
         if ((unsigned)e < (unsigned)E) {
             const int t = (int)(i / a.K), k = (int)(i - (long long)t * a.K);
             const int pos = s_off[e] + atomicAdd(cursor + e, 1);
-            a.perm[pos] = k * a.M + t;
-            if (a.inv) a.inv[k * a.M + t] = pos;
+            if ((unsigned)pos < (unsigned)(a.M * a.K)) {
+                a.perm[pos] = k * a.M + t;
+                if (a.inv) a.inv[k * a.M + t] = pos;
+            } else {  // the counts disagree with the ids: flag it, place nothing out of range
+                set_dev_error(a.err, MOE_DEVERR_BAD_INDEX);
+            }
         } else {
             set_dev_error(a.err, MOE_DEVERR_BAD_EXPERT_ID);
         }
