@@ -186,6 +186,9 @@ def accounting(shape, T: int, U: int, router: bool, Is: int):
     k["router"] = {"bytes": E * H * 2 + T * H * 2 + T * E * 4, "flops": 2 * T * E * H}
     k["topk"] = {"bytes": T * E * 4 + T * K * 8, "flops": 0}
     k["route"] = {"bytes": T * E * 4 + T * K * 8, "flops": 0}
+    # exact re-evaluation of ~K candidate logits per token: an x row and a router row each
+    k["refine"] = {"bytes": T * K * H * 2 * 2, "flops": 2 * T * K * H}
+    k["select"] = {"bytes": T * K * 12 + T * K * 8, "flops": 0}
     k["permute"] = {"bytes": T * K * 4 * 2, "flops": 0}
     k["fc1"] = {"bytes": U * rows1 * H * 2 + rows1s * H * 2 + T * H * 2 + h_bytes,
                 "flops": 2 * T * K * rows1 * H + 2 * T * rows1s * H}
@@ -204,8 +207,8 @@ def kernel_names(path: str, router: bool, launches: int = 0):
     names = ["router"] if router else []
     if path == "small":
         return names + ["route", "fc1", "fc2"]
-    if launches == len(names) + 4:
-        return names + ["route", "fc1", "fc2", "finalize"]
+    if launches == len(names) + 7:  # top-k after the tensor-core router: screen, refine, final
+        return names + ["topk", "refine", "select", "permute", "fc1", "fc2", "finalize"]
     return names + ["topk", "permute", "fc1", "fc2", "finalize"]
 
 

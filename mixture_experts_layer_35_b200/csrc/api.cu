@@ -14,8 +14,12 @@ bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) 
 
 // Workspace carve-up of moe_fused_forward, 256-byte aligned regions after the header.
 struct WsLayout {
-    size_t logits, route, topk_w, topk_ids, offsets, tiles1, tiles2, counts, perm, h, hs, acc, ys, total;
+    size_t logits, route, topk_w, topk_ids, offsets, tiles1, tiles2, counts, perm, cand, h, hs, acc, ys, total;
 };
+// Candidate-list capacity per token of the three-kernel top-k (rows with more fall back).
+constexpr size_t kCandPerRow = 32;
+// Slot counters: per-expert counts, per-expert cursors, then the candidate count.
+inline size_t counter_ints(size_t E) { return 2 * (E + 2) + 4; }
 WsLayout layout(const moe_layer_desc* d) {
     const size_t T = (size_t)d->T, E = (size_t)d->E, K = (size_t)d->top_k, H = (size_t)d->H, I = (size_t)d->I,
                  Is = (size_t)d->I_shared;
@@ -33,8 +37,9 @@ WsLayout layout(const moe_layer_desc* d) {
     L.offsets = take((E + 2) * 4);
     L.tiles1 = take((E + 2) * 4);
     L.tiles2 = take((E + 2) * 4);
-    L.counts = take(2 * (E + 2) * 4);  // per-expert counts, then per-expert cursors
+    L.counts = take(counter_ints(E) * 4);
     L.perm = take(T * K * 4);
+    L.cand = take(T * (2 + 3 * kCandPerRow) * 4);  // row_base, row_n, cand_row, cand_e, cand_val
     L.h = take(T * K * I * 2);
     L.hs = take(T * Is * 2);
     L.acc = take(T * H * 4);
@@ -237,10 +242,24 @@ int moe_select_path(const moe_layer_desc* d) {
     return resolve_path(d);
 }
 
+// The tensor-core router runs when the logits are not given and the few-token router does
+// not apply.  Its top-k is split in three kernels for more than 256 experts: there the
+// one-kernel top-k, whose warps hold 16+ logits each and refine their candidates one after
+// another, runs at low occupancy (measured at E = 512, T = 4096: 97 -> 83 us; at E <= 256 the
+// extra launches cost more than they save).  Softmax without renorm keeps the one-kernel
+// form, whose weights need every logit of the row.
+static bool dense_router_for(const moe_layer_desc* d) {
+    return !d->router_logits && !(d->T <= 64 && router_small_supported(d->H));
+}
+static bool split_topk_mode(const moe_layer_desc* d) {
+    return d->E > 256 && (d->score == MOE_SCORE_SIGMOID || d->renorm);
+}
+
 int moe_fused_forward_launches(const moe_layer_desc* d) {
     if (validate_desc(d) != MOE_OK || d->T == 0) return 0;
     const int router = d->router_logits ? 0 : 1;
     if (resolve_path(d) == MOE_PATH_SMALL) return router + 3;  // route table, fc1, fc2
+    if (dense_router_for(d) && split_topk_mode(d)) return router + 7;  // screen, refine, final, ...
     return router + 5;                                          // topk, permute, fc1, fc2, finalize
 }
 
@@ -278,8 +297,7 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
     // 0. the many-token path's slot counters start at zero.  Cleared before the first
     // kernel, so that every kernel launched with programmatic overlap follows a kernel
     // (a memset between two kernels would leave the second one's overlap undefined).
-    if (path == MOE_PATH_LARGE)
-        MOE_CK(cudaMemsetAsync(w8 + L.counts, 0, 2 * (size_t)(E + 2) * sizeof(int), s));
+    if (path == MOE_PATH_LARGE) MOE_CK(cudaMemsetAsync(w8 + L.counts, 0, counter_ints(E) * sizeof(int), s));
 
     // 1. router logits
     const float* logits = d->router_logits;
@@ -355,8 +373,23 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
     // 2. top-k (also counts the slots per expert; the counters were cleared in step 0)
     if (!mark()) return MOE_ERR_CUDA;
     RefineArgs ra = {x, static_cast<const bf16*>(d->router_w), H, logits_rw};
-    MOE_CK(launch_topk(logits, false, T, E, K, d->score, d->bias, d->renorm, tw, tid, nullptr, topk_w_out,
-                       topk_ids_out, s, pdl && chain, dense_router ? &ra : nullptr, counts));
+    if (dense_router && split_topk_mode(d)) {  // screen, refine, final
+        int* cbase = reinterpret_cast<int*>(w8 + L.cand);
+        CandList cl;
+        cl.count = counts + 2 * (E + 2);
+        cl.row_base = cbase;
+        cl.row_n = cbase + T;
+        cl.cand_row = cbase + 2 * (size_t)T;
+        cl.cand_e = cl.cand_row + kCandPerRow * (size_t)T;
+        cl.cand_val = reinterpret_cast<float*>(cl.cand_e + kCandPerRow * (size_t)T);
+        cl.cap = (int)(kCandPerRow * (size_t)T);
+        const std::function<bool()> mark_fn = mark;
+        MOE_CK(launch_topk_split(logits, T, E, K, d->score, d->bias, d->renorm, tw, tid, topk_w_out, topk_ids_out,
+                                 cl, ra, counts, err, sms, s, pdl && chain, timed ? &mark_fn : nullptr));
+    } else {
+        MOE_CK(launch_topk(logits, false, T, E, K, d->score, d->bias, d->renorm, tw, tid, nullptr, topk_w_out,
+                           topk_ids_out, s, pdl && chain, dense_router ? &ra : nullptr, counts));
+    }
     // 3. permutation + tile tables
     PermuteArgs pa;
     std::memset(&pa, 0, sizeof(pa));

@@ -38,6 +38,21 @@ cudaError_t launch_topk(const void* logits, bool bf16_in, int M, int E, int K, i
                         int renorm, float* topk_w, int32_t* topk_ids, int32_t* src_idx, float* w_copy,
                         int32_t* id_copy, cudaStream_t s, bool pdl, const RefineArgs* refine = nullptr,
                         int* counts = nullptr);
+// Candidate list of the three-kernel top-k after the tensor-core router.
+struct CandList {
+    int* count;       // [1] candidates appended so far (zero on entry)
+    int* row_base;    // [M] first list entry of each row
+    int* row_n;       // [M] candidates of each row
+    int* cand_row;    // [cap]
+    int* cand_e;      // [cap]
+    float* cand_val;  // [cap] exact logits
+    int cap;
+};
+// screen, refine and final kernels; `mark` (optional) records a timing event between them.
+cudaError_t launch_topk_split(const float* logits, int M, int E, int K, int score, const float* bias, int renorm,
+                              float* topk_w, int32_t* topk_ids, float* w_copy, int32_t* id_copy, const CandList& cl,
+                              const RefineArgs& ra, int* counts, int* err, int num_sms, cudaStream_t s, bool pdl,
+                              const std::function<bool()>* mark);
 bool router_small_supported(int H);
 cudaError_t launch_router_small(const bf16* x, const bf16* wr, int T, int H, int E, float* logits,
                                 float* logits_copy, int* err, cudaStream_t s, bool pdl);

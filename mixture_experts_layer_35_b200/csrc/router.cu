@@ -89,6 +89,190 @@ cudaError_t launch_topk(const void* logits, bool bf16_in, int M, int E, int K, i
     return cudaErrorInvalidValue;
 }
 
+// ---------------------------------------------------------------- top-k after the tensor-core router
+// In three kernels, so that the exact re-evaluation of the candidates runs with one warp
+// per candidate (thousands of independent dot products) instead of one warp walking its
+// row's candidates one after another:
+//   screen: warp per row; screening select on the tensor-core logits, and the row's
+//           candidates (keys within the window of the K-th) appended to a global list
+//           (one atomic per row reserves a contiguous range);
+//   refine: warp per candidate; exact logit (FP64 sum of the exact products), written to
+//           the list and back into the logits;
+//   final:  warp per row; the candidates, one per lane, keyed on exact values (correctly
+//           rounded sigmoid), top K by (key desc, id asc), weights, slot counts.
+// The K selected are always candidates (see route_refine_keys), so the final select over
+// the candidates alone is the select over exact keys.  A row with more than 32 candidates
+// (not seen on any workload) is routed by the one-kernel path with per-row refinement.
+template <int V>
+__global__ void __launch_bounds__(32 * kTopkRowsPerBlock) topk_screen_kernel(const float* __restrict__ logits, int M,
+                                                                              int E, int K, int score,
+                                                                              const float* __restrict__ bias,
+                                                                              const CandList cl) {
+    pdl_wait();
+    const int lane = threadIdx.x & 31;
+    const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (row < M) {
+        const bool sig = score == MOE_SCORE_SIGMOID;
+        float l[V], key[V];
+        load_row_f32<V>(logits + (size_t)row * E, E, lane, l);
+        screening_keys<V>(l, key, E, sig, bias, lane);
+        float kth, ua, ub;
+        warp_select<V, false>(key, key, key, E, K, lane, kth, ua, ub);
+        const float lo = kth - screen_window(kth, sig, kTcLogitErr);
+        unsigned mc[V];
+        int before[V], n = 0;
+#pragma unroll
+        for (int c = 0; c < V; ++c) {
+            mc[c] = __ballot_sync(0xffffffffu, lane + 32 * c < E && !(key[c] < lo));
+            before[c] = n;
+            n += __popc(mc[c]);
+        }
+        int base = 0;
+        if (lane == 0) {
+            base = atomicAdd(cl.count, n);
+            cl.row_base[row] = base;
+            cl.row_n[row] = n;
+        }
+        base = __shfl_sync(0xffffffffu, base, 0);
+        const unsigned lt = (1u << lane) - 1u;
+#pragma unroll
+        for (int c = 0; c < V; ++c) {
+            if ((mc[c] >> lane) & 1u) {
+                const int pos = base + before[c] + __popc(mc[c] & lt);
+                if (pos < cl.cap) {
+                    cl.cand_row[pos] = row;
+                    cl.cand_e[pos] = lane + 32 * c;
+                }
+            }
+        }
+    }
+    pdl_trigger();
+}
+
+__global__ void __launch_bounds__(256) refine_kernel(const bf16* __restrict__ x, const bf16* __restrict__ wr, int M,
+                                                    int H, int E, const CandList cl, float* __restrict__ logits_rw,
+                                                    int* err) {
+    pdl_wait();
+    const int lane = threadIdx.x & 31;
+    const int nw = (gridDim.x * blockDim.x) >> 5;
+    const int n = min(*cl.count, cl.cap);
+    for (int it = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; it < n; it += nw) {
+        const int row = cl.cand_row[it], e = cl.cand_e[it];
+        if ((unsigned)row >= (unsigned)M || (unsigned)e >= (unsigned)E) {
+            if (lane == 0) set_dev_error(err, MOE_DEVERR_BAD_INDEX);
+            continue;
+        }
+        const float v = warp_dot_exact(x + (size_t)row * H, wr + (size_t)e * H, H, lane);
+        if (lane == 0) {
+            cl.cand_val[it] = v;
+            if (logits_rw) logits_rw[(size_t)row * E + e] = v;
+        }
+    }
+    pdl_trigger();
+}
+
+template <int V>
+__global__ void __launch_bounds__(32 * kTopkRowsPerBlock) topk_final_kernel(
+    const float* __restrict__ logits, int M, int E, int K, int score, const float* __restrict__ bias, int renorm,
+    const CandList cl, float* __restrict__ topk_w, int32_t* __restrict__ topk_ids, float* __restrict__ w_copy,
+    int32_t* __restrict__ id_copy, int* __restrict__ counts, const bf16* __restrict__ x,
+    const bf16* __restrict__ wr, int H, float* logits_rw) {
+    __shared__ float s_wbuf[kTopkRowsPerBlock][32];
+    pdl_wait();
+    const int lane = threadIdx.x & 31;
+    const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (row >= M) {
+        pdl_trigger();
+        return;
+    }
+    const bool sig = score == MOE_SCORE_SIGMOID;
+    const int n = cl.row_n[row], base = cl.row_base[row];
+    int id = 0;
+    float w = 0.0f;
+    if (n <= 32 && base + n <= cl.cap) {
+        const float NEG_INF = __int_as_float(0xff800000);
+        const bool has = lane < n;
+        const int e = has ? cl.cand_e[base + lane] : 0x7fffffff;
+        const float lv = has ? cl.cand_val[base + lane] : 0.0f;
+        const float sv = (has && sig) ? sigmoid_f32_rn(lv) : 0.0f;
+        float k = sig ? sv : lv;
+        if (has && bias) k = __fadd_rn(k, bias[e]);
+        const uint32_t code0 = has ? key_code((k != k) ? NEG_INF : k) : 0u;
+        uint32_t code = code0;
+        float sel_l = 0.0f, sel_s = 0.0f;
+        for (int r = 0; r < K; ++r) {  // K rounds over one candidate per lane
+            const uint32_t best = __reduce_max_sync(0xffffffffu, code);
+            const uint32_t mine = (code != 0u && code == best) ? (uint32_t)e : 0x7fffffffu;
+            const int win = (int)__reduce_min_sync(0xffffffffu, mine);
+            const int src = __ffs(__ballot_sync(0xffffffffu, code != 0u && e == win)) - 1;
+            const float wl = __shfl_sync(0xffffffffu, lv, src & 31);
+            const float ws = __shfl_sync(0xffffffffu, sv, src & 31);
+            if (lane == r) {
+                id = win;
+                sel_l = wl;
+                sel_s = ws;
+            }
+            if (lane == src) code = 0u;
+        }
+        if (sig) {
+            const float sk = (lane < K) ? sel_s : 0.0f;
+            double sum = 0.0;
+            for (int r = 0; r < K; ++r) sum += (double)__shfl_sync(0xffffffffu, sk, r);
+            w = renorm ? __double2float_rn((double)sk / sum) : sk;
+        } else {  // softmax with renorm (the only softmax mode routed here)
+            float lmax = (lane < K) ? sel_l : NEG_INF;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) lmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
+            const double ex = (lane < K) ? exp_f64((double)sel_l - (double)lmax) : 0.0;
+            double sum = 0.0;
+            for (int r = 0; r < K; ++r) sum += __shfl_sync(0xffffffffu, ex, r);
+            w = __double2float_rn(ex / sum);
+        }
+    } else {  // many candidates: route the row in one warp with per-candidate refinement
+        float l[V];
+        load_row_f32<V>(logits + (size_t)row * E, E, lane, l);
+        const RowRefine rf{x + (size_t)row * H, wr, H, E, row, lane, logits_rw};
+        float lg;
+        warp_route_row<V>(l, E, K, score, bias, renorm, lane, kTcLogitErr, rf, s_wbuf[threadIdx.x >> 5], id, w, lg);
+    }
+    if (lane < K) {
+        const size_t o = (size_t)row * K + lane;
+        topk_w[o] = w;
+        topk_ids[o] = id;
+        if (w_copy) w_copy[o] = w;
+        if (id_copy) id_copy[o] = id;
+        if (counts) atomicAdd(counts + id, 1);
+    }
+    pdl_trigger();
+}
+
+cudaError_t launch_topk_split(const float* logits, int M, int E, int K, int score, const float* bias, int renorm,
+                              float* topk_w, int32_t* topk_ids, float* w_copy, int32_t* id_copy, const CandList& cl,
+                              const RefineArgs& ra, int* counts, int* err, int num_sms, cudaStream_t s, bool pdl,
+                              const std::function<bool()>* mark) {
+    dim3 grid(cdiv(M, kTopkRowsPerBlock)), block(32 * kTopkRowsPerBlock);
+    const int v = topk_v(E);
+    cudaError_t st = cudaErrorInvalidValue;
+#define MOE_S(VV) \
+    if (v == VV) st = launch_k(topk_screen_kernel<VV>, grid, block, 0, s, pdl, logits, M, E, K, score, bias, cl);
+    MOE_S(1) MOE_S(2) MOE_S(4) MOE_S(8) MOE_S(16) MOE_S(32)
+#undef MOE_S
+    if (st != cudaSuccess) return st;
+    if (mark && !(*mark)()) return cudaErrorUnknown;
+    st = launch_k(refine_kernel, dim3(num_sms * 8), dim3(256), 0, s, pdl, ra.x, ra.wr, M, ra.H, E, cl,
+                  ra.logits_rw, err);
+    if (st != cudaSuccess) return st;
+    if (mark && !(*mark)()) return cudaErrorUnknown;
+    st = cudaErrorInvalidValue;
+#define MOE_F(VV)                                                                                             \
+    if (v == VV)                                                                                              \
+        st = launch_k(topk_final_kernel<VV>, grid, block, 0, s, pdl, logits, M, E, K, score, bias, renorm, cl, \
+                      topk_w, topk_ids, w_copy, id_copy, counts, ra.x, ra.wr, ra.H, ra.logits_rw);
+    MOE_F(1) MOE_F(2) MOE_F(4) MOE_F(8) MOE_F(16) MOE_F(32)
+#undef MOE_F
+    return st;
+}
+
 // ---------------------------------------------------------------- router logits, few tokens
 // l[t, e] = x[t,:] . Wr[e,:]: each BF16 x BF16 product is exact in FP32 and is summed in
 // FP64, rounded once to FP32 (the oracle's definition; see warp_dot_exact).  CTA (i, g):

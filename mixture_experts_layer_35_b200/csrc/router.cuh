@@ -143,6 +143,31 @@ __device__ __forceinline__ int warp_select(const float (&key)[V], const float (&
     return my;
 }
 
+// Window around the K-th screening key: the screening error of a key (logit error eps_l,
+// sigmoid slope <= 1/4, fast-sigmoid error, key rounding), doubled because both sides of a
+// comparison carry it.
+__device__ __forceinline__ float screen_window(float kth, bool sig, float eps_l) {
+    const float mag = fmaxf(1.0f, fabsf(kth));
+    return 2.0f * (sig ? (0.25f * eps_l + 4e-6f * mag) : (eps_l + 4e-7f * mag));
+}
+
+// Screening keys of one row (fast sigmoid for sigmoid scores; -inf past E and for NaN).
+template <int V>
+__device__ __forceinline__ void screening_keys(const float (&l)[V], float (&key)[V], int E, bool sig,
+                                               const float* bias, int lane) {
+    const float NEG_INF = __int_as_float(0xff800000);
+#pragma unroll
+    for (int c = 0; c < V; ++c) {
+        const int e = lane + 32 * c;
+        key[c] = NEG_INF;
+        if (e < E) {
+            float k = sig ? sigmoid_fast(l[c]) : l[c];
+            if (bias) k = __fadd_rn(k, bias[e]);
+            key[c] = (k != k) ? NEG_INF : k;
+        }
+    }
+}
+
 struct NoRefine {
     __device__ float operator()(int) const { return 0.0f; }
 };
@@ -162,9 +187,7 @@ __device__ __forceinline__ void route_refine_keys(float (&l)[V], float (&key)[V]
     warp_select<V, false>(key, key, key, E, K, lane, kth, ua, ub);
     // Window: screening error of a key (logit error, sigmoid slope <= 1/4, fast-sigmoid
     // error, key rounding), doubled because both sides of a comparison carry it.
-    const float mag = fmaxf(1.0f, fabsf(kth));
-    const float win = 2.0f * (sig ? (0.25f * eps_l + 4e-6f * mag) : (eps_l + 4e-7f * mag));
-    const float lo = kth - win;
+    const float lo = kth - screen_window(kth, sig, eps_l);
     unsigned mc[V];  // candidate lanes of each chunk
     int base[V];     // candidates in the chunks before
     int ncand = 0;
@@ -269,18 +292,9 @@ __device__ __forceinline__ void warp_route_row(float (&l)[V], int E, int K, int 
     const bool sig = score == MOE_SCORE_SIGMOID;
     float key[V];
     float sx[V];  // exact sigmoid of the candidates (sigmoid scores only)
+    screening_keys<V>(l, key, E, sig, bias, lane);
 #pragma unroll
-    for (int c = 0; c < V; ++c) {
-        const int e = lane + 32 * c;
-        key[c] = NEG_INF;
-        sx[c] = 0.0f;
-        if (e < E) {
-            const float lv = l[c];
-            float k = sig ? sigmoid_fast(lv) : lv;
-            if (bias) k = __fadd_rn(k, bias[e]);
-            key[c] = (k != k) ? NEG_INF : k;
-        }
-    }
+    for (int c = 0; c < V; ++c) sx[c] = 0.0f;
     // exact logits keyed directly (softmax, eps 0): the screening keys are the keys
     if (sig || eps_l > 0.0f) route_refine_keys<V>(l, key, sx, E, K, sig, bias, lane, eps_l, refine, wbuf);
     float kth, sel_s;

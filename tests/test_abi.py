@@ -102,6 +102,10 @@ def test_path_selection_and_launch_counts():
     d = _desc(T=4096)
     assert moe.select_path(d) == "large"
     assert moe.launches(d) == 6
+    d = _desc(T=4096, E=512, top_k=10)
+    assert moe.launches(d) == 8  # router, top-k in three kernels, permute, fc1, fc2, finalize
+    d = _desc(T=4096, E=512, top_k=10, score="softmax", renorm=False)
+    assert moe.launches(d) == 6  # full softmax keeps the one-kernel top-k
     d = _desc(T=4, path="large")
     assert moe.select_path(d) == "large"
     assert moe.launches(d) == 6

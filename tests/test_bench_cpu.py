@@ -38,7 +38,8 @@ def test_roofline_bound_choice():
 
 def test_kernel_names_follow_launch_order():
     assert bench.kernel_names("small", True) == ["router", "route", "fc1", "fc2"]
-    assert bench.kernel_names("large", True, 5) == ["router", "route", "fc1", "fc2", "finalize"]
+    assert bench.kernel_names("large", True, 8) == ["router", "topk", "refine", "select", "permute", "fc1", "fc2",
+                                                    "finalize"]
     assert bench.kernel_names("large", False, 5) == ["topk", "permute", "fc1", "fc2", "finalize"]
     assert bench.kernel_names("large", False) == ["topk", "permute", "fc1", "fc2", "finalize"]
 

@@ -137,6 +137,19 @@ def test_fused_routing_every_row(shape, T):
                               h["bias"], False)
 
 
+TIED = LayerShape("tied-router", 256, 128, 320, 4, "swiglu", "softmax", True, None, 0)
+
+
+@pytest.mark.parametrize("T", [100, 300])
+def test_many_candidates_fall_back_to_per_row_refinement(T):
+    """Every expert has the same router row, so all 320 logits of a row tie and every expert
+    is a top-k candidate (more than the 32 the three-kernel top-k carries per row): those
+    rows take the per-row refinement path, and the lower-id tie break must hold exactly."""
+    d = _util.device_layer(TIED, T, seed=5)
+    d["router_w"] = d["router_w"][:1].expand_as(d["router_w"]).contiguous()
+    _check(TIED, d, "large")
+
+
 def test_small_path_deterministic_and_graph_replay():
     shape = gen.QWEN36
     d = _util.device_layer(shape, 4, seed=5)
