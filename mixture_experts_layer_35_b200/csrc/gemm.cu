@@ -64,8 +64,11 @@ struct Cfg {
     // Two accumulator buffers (the epilogue of one tile overlaps the next mainloop) when
     // they fit TMEM's 512 columns; a 256-token SwiGLU tile (gate + up = 512 columns) has one.
     static constexpr int kAccBufs = (2 * kAccCols) <= 512 ? 2 : 1;
+    // Buffer stride in TMEM columns, padded to a multiple of 64.
+    static constexpr int kAccStride = (kAccCols + 63) / 64 * 64;
     static constexpr int kTmemCols =
-        (kAccBufs * kAccCols) > 256 ? 512 : ((kAccBufs * kAccCols) > 128 ? 256 : 128);
+        (kAccBufs * kAccStride) > 256 ? 512 : ((kAccBufs * kAccStride) > 128 ? 256 : 128);
+    static_assert(kAccBufs * kAccStride <= 512 || kAccBufs == 1, "accumulator buffers exceed TMEM");
     static_assert(kAccCols <= 512, "accumulator exceeds TMEM");
     static constexpr int kThreads = 64 + 32 * kEpiWarps + (kGather ? 128 : 0);
     // FC1 gather: stages of token rows in flight before the gather warps signal the oldest
@@ -241,7 +244,7 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
                 const uint32_t tph = (uint32_t)(tcount / C::kAccBufs) & 1u;
                 if (!mbar_wait(tempty_bar(buf), tph ^ 1u, abort_flag, a.err)) break;
                 tc_fence_after();
-                const uint32_t d0 = tmem_base + (uint32_t)(buf * C::kAccCols);
+                const uint32_t d0 = tmem_base + (uint32_t)(buf * C::kAccStride);
                 const uint32_t d1 = d0 + C::kBN;
                 bool ok = true;
                 for (int kb = 0; kb < nk; ++kb, ++it) {
@@ -319,7 +322,7 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
             const int f = ti.ft * BM + q * 32 + lane;
             const int feat = ti.shared ? a.feat_s : a.feat_r;
             const bool fok = f < feat;
-            const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * C::kAccCols);
+            const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * C::kAccStride);
 #pragma unroll
             for (int ci = 0; ci < kChunks; ++ci) {
                 const int c0 = 32 * half + 32 * nhalf * ci;
@@ -521,9 +524,8 @@ int gemm_token_tile(int mode, int T, int K, int E) {
     if (mode == GM_DENSE) return default_bn<GM_DENSE>();
     if (T <= 32) return 32;  // no expert has more rows than a tile
     const double rows = (double)T * K / E;  // average rows per expert
-    // FC2: a tile that covers an expert's rows streams its W2 slice once, and FC2 is bound
-    // by the bytes its ring keeps in flight: 192 holds almost every expert of ~128 rows
-    // and leaves room for 4 stages.
+    // FC2: a tile that covers an expert's rows streams its W2 slice once; 192 holds almost
+    // every expert of ~128 rows with 5 stages (measured: 160 with 6 stages is no faster).
     if (mode == GM_FC2) return rows <= 64.0 ? 128 : (rows <= 150.0 ? 192 : 256);
     // FC1: a tile re-streams the expert's weight slice, so an expert just over a tile's
     // width costs a second, nearly empty tile; 256-token tiles keep most experts at one.
