@@ -217,8 +217,8 @@ def kernel_names(path: str, router: bool, launches: int = 0):
 # The capture and its command are summarised in profiles/; an entry is removed whenever
 # its kernel changes, so that a stale count is never reported.
 NCU_TRAFFIC = {
-    ("qwen36", 4096, "router", "fc1"): 1.259206e9 + 65.595392e6,
-    ("qwen36", 4096, "router", "fc2"): 0.634541e9 + 10.745600e6,
+    ("qwen36", 4096, "router", "fc1"): 1.273545e9 + 65.571072e6,
+    ("qwen36", 4096, "router", "fc2"): 0.632232e9 + 10.936576e6,
 }
 
 

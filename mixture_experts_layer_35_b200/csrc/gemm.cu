@@ -55,9 +55,9 @@ struct Cfg {
     static constexpr int kBN = BN;
     static constexpr int kBBytes = kBN * BK * 2;
     static constexpr int kStageBytes = kNA * A_BYTES + kBBytes;
-    // Epilogue warps: FC2's epilogue (staging + bulk reduce) is heavier than its short
-    // mainloop, so with wide tiles it gets two warps per TMEM lane quarter, splitting the
-    // token columns.
+    // Epilogue warps: FC2's epilogue (weighting, transposes, vector reductions) is heavy
+    // next to its short mainloop, so with wide tiles it gets two warps per TMEM lane
+    // quarter, splitting the token columns.
     static constexpr int kEpiWarps = (MODE == GM_FC2 && BN > 32) ? 8 : 4;
     static constexpr int kEpiBytes = 0;  // epilogues work from registers
     static constexpr int kAccCols = kSwiglu ? 2 * kBN : kBN;
@@ -284,8 +284,7 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
                 z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
         int tcount = 0;
-        // (the abort flag is checked through the per-tile wait and vote below, so that the
-        // epilogue warps always take the same number of tiles)
+        // (the abort flag is checked through the per-tile wait below)
         // 32-token chunks per half of the epilogue warps (the last may lie past the tile)
         constexpr int kChunks = (C::kBN + 32 * (C::kEpiWarps / 4) - 1) / (32 * (C::kEpiWarps / 4));
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++tcount) {
