@@ -217,7 +217,6 @@ def kernel_names(path: str, router: bool, launches: int = 0):
 # The capture and its command are summarised in profiles/; an entry is removed whenever
 # its kernel changes, so that a stale count is never reported.
 NCU_TRAFFIC = {
-    ("qwen36", 4096, "router", "fc1"): 1.273545e9 + 65.571072e6,
     ("qwen36", 4096, "router", "fc2"): 0.632232e9 + 10.936576e6,
 }
 

@@ -156,7 +156,7 @@ struct GemmMaps {
 // Token rows per tile of a grouped GEMM for a call over T tokens, top-k K and E experts:
 // 32 when T <= 32 (no expert can have more rows), else by the average rows per expert
 // (FC1: 64 up to 48 rows, else 128, and 256 above 96 for ReLU^2; FC2: 128 up to 64
-// rows, else 256).  Narrow tiles leave shared memory for a deeper
+// rows, 192 up to 150, else 256).  Narrow tiles leave shared memory for a deeper
 // weight ring.  The permute kernel's tile tables must use the same value as the launch.
 int gemm_token_tile(int mode, int T, int K, int E);
 cudaError_t launch_gemm(int mode, int bn, const GemmArgs& a, const GemmMaps& m, int grid, cudaStream_t s, bool pdl);
