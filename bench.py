@@ -217,7 +217,8 @@ def kernel_names(path: str, router: bool, launches: int = 0):
 # The capture and its command are summarised in profiles/; an entry is removed whenever
 # its kernel changes, so that a stale count is never reported.
 NCU_TRAFFIC = {
-    ("qwen36", 4096, "router", "fc2"): 0.632232e9 + 10.936576e6,
+    ("qwen36", 4096, "router", "fc1"): 1.185122e9 + 64.430848e6,
+    ("qwen36", 4096, "router", "fc2"): 0.631720e9 + 12.998400e6,
 }
 
 
@@ -252,6 +253,10 @@ class Bench:
         # One complete layer forward per CUDA-graph replay (the launch sequence is
         # captured once; replays carry no host launch overhead).
         self.stream = torch.cuda.Stream(device)
+        # The inputs were generated, and the workspace allocated, in the default stream's
+        # order: the side stream may only start once that work is done (the workspace can
+        # reuse a block that a pending generator kernel still writes).
+        torch.cuda.synchronize(device)
         self.step_eager(stream=self.stream)  # tensor-map and attribute set-up outside capture
         torch.cuda.synchronize(device)
         self.graph = torch.cuda.CUDAGraph()
@@ -470,6 +475,7 @@ def run_router_topk(args, rank, local, world):
     flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     stream = torch.cuda.Stream(device)
     call = lambda x=lg: moe.router_topk(x, K, "sigmoid", bias, True, stream=stream, out=outs)  # noqa: E731
+    torch.cuda.synchronize(device)  # inputs and outputs were made in the default stream's order
     call()
     torch.cuda.synchronize(device)
     graph = torch.cuda.CUDAGraph()

@@ -132,6 +132,11 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmArgs& a, const int* s_
     ti.shared = sh;
     ti.nk = cdiv(sh ? a.kdim_s : a.kdim, BK);
     ti.ntok = ntok;
+    if (ti.n <= 0 || ti.row0 < 0) {  // only from corrupted tables: every role skips the tile
+        set_dev_error(a.err, MOE_DEVERR_BAD_INDEX);
+        ti.n = 0;
+        ti.nk = 0;
+    }
     return ti;
 }
 
@@ -426,7 +431,7 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
         for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
             const TileInfo ti = decode_tile<C::kBN>(a, s_tiles, s_offs, G, tile);
             const int kd = ti.shared ? a.kdim_s : a.kdim;
-            const int nk = cdiv(kd, BK);
+            const int nk = ti.nk;
             const int npad = cdiv(ti.n, 16) * 16;
             int tok[C::kBN / 16];
 #pragma unroll
