@@ -218,7 +218,6 @@ def kernel_names(path: str, router: bool, launches: int = 0):
 # its kernel changes, so that a stale count is never reported.
 NCU_TRAFFIC = {
     ("qwen36", 4096, "router", "fc1"): 1.185122e9 + 64.430848e6,
-    ("qwen36", 4096, "router", "fc2"): 0.631720e9 + 12.998400e6,
 }
 
 

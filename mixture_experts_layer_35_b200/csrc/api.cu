@@ -455,9 +455,9 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
     // 5. FC2 + weighted scatter-add (shared expert -> ys)
     GemmMaps m2;
     std::memset(&m2, 0, sizeof(m2));
-    if (!map3d(&m2.a_r, d->w2, I, H, E, 128) || !map2d(&m2.b_r, h, I, (uint64_t)T * K, 16)) return MOE_ERR_CUDA;
+    if (!map3d(&m2.a_r, d->w2, I, H, E, 128) || !map2d(&m2.b_r, h, I, (uint64_t)T * K, kFc2BoxRows)) return MOE_ERR_CUDA;
     if (Is) {
-        if (!map2d(&m2.a_s, d->ws2, Is, H, 128) || !map2d(&m2.b_s, hs, Is, T, 16)) return MOE_ERR_CUDA;
+        if (!map2d(&m2.a_s, d->ws2, Is, H, 128) || !map2d(&m2.b_s, hs, Is, T, kFc2BoxRows)) return MOE_ERR_CUDA;
     } else {
         m2.a_s = m2.a_r;
         m2.b_s = m2.b_r;

@@ -12,7 +12,7 @@
 //       the expert's tokens gathered row by row from x with cp.async into the swizzled
 //       layout; epilogue applies SwiGLU / ReLU^2 and stores h (BF16) in permuted order.
 //   FC2: A = W2[e] rows of 128 output features, B = the expert's contiguous h rows
-//       (TMA, 16-row boxes); epilogue scales by the routing weight, transposes 4x4 blocks
+//       (TMA, 32-row boxes); epilogue scales by the routing weight, transposes 4x4 blocks
 //       within groups of 4 lanes and adds into the FP32 accumulator acc[t, :] with 16-byte
 //       vector reductions, 4 consecutive features of one token per lane ("weighted output
 //       combination").
@@ -23,8 +23,9 @@
 //   warp 0      TMA producer (weights; FC2/DENSE token rows)
 //   warp 1      TMEM allocator and single-thread MMA issuer
 //   warps 2-5   epilogue: tcgen05.ld of the accumulator (warp w reads TMEM lanes of
-//               quarter w % 4), activation / scaling, stores; FC2 has eight epilogue
-//               warps (2-9), the second four taking the odd 32-token column chunks
+//               quarter w % 4), activation / scaling, stores; FC2 with wide tiles has
+//               twelve epilogue warps (2-13), the three warps of a quarter taking every
+//               third 32-token column chunk
 //   warps 6-9   FC1 only: cp.async gather of token rows of x
 // Shared memory holds a ring of stages (full/empty mbarriers); TMEM holds two
 // accumulator buffers so the epilogue of one tile overlaps the mainloop of the next.
@@ -35,7 +36,14 @@ namespace {
 
 constexpr int BM = 128, BK = 64;
 constexpr int A_BYTES = BM * BK * 2;  // 16 KB
-constexpr int BBOX = 16;              // token rows per TMA box of the B operand
+// Token rows per TMA box of the B operand: FC2's h rows come in 32-row boxes (half the
+// copies per stage of 16-row boxes; measured -18 % on FC2 at 192 rows per expert), the
+// router's x rows in 16-row boxes.  A box may run past the tile's rows: the MMA reads
+// only the tile's rows rounded up to 16, so the extra rows are never used.
+template <int MODE>
+__host__ __device__ constexpr int b_box_rows() {
+    return MODE == GM_FC2 ? kFc2BoxRows : 16;
+}
 
 // Token rows per tile (MMA N) of each mode at prefill sizes: FC2 takes up to 256 so that
 // an expert's W2 tile is streamed once for all its tokens; FC1 keeps 128 so that its gate
@@ -56,9 +64,11 @@ struct Cfg {
     static constexpr int kBBytes = kBN * BK * 2;
     static constexpr int kStageBytes = kNA * A_BYTES + kBBytes;
     // Epilogue warps: FC2's epilogue (weighting, transposes, vector reductions) is heavy
-    // next to its short mainloop, so with wide tiles it gets two warps per TMEM lane
-    // quarter, splitting the token columns.
-    static constexpr int kEpiWarps = (MODE == GM_FC2 && BN > 32) ? 8 : 4;
+    // next to its short mainloop, so with wide tiles it gets three warps per TMEM lane
+    // quarter, splitting the token columns (measured at T = 4096 / 8192 of the
+    // Qwen3.6-shaped layer, FC2: 4 warps 240 / 582 us, 8 warps 144 / 322 us, 12 warps
+    // 137 / 276 us, 16 warps 140 / 304 us).
+    static constexpr int kEpiWarps = (MODE == GM_FC2 && BN > 32) ? 12 : 4;
     static constexpr int kEpiBytes = 0;  // epilogues work from registers
     static constexpr int kAccCols = kSwiglu ? 2 * kBN : kBN;
     // Two accumulator buffers (the epilogue of one tile overlaps the next mainloop) when
@@ -88,6 +98,7 @@ struct Cfg {
     static constexpr size_t kSmem = 1024 + (size_t)kStages * kStageBytes + kEpiBytes + kMeta;
     static constexpr int kLag = (kStages - 2) < kLagMax ? (kStages - 2) : kLagMax;
     static_assert(kStages >= 3, "ring too shallow");
+    static_assert(kGather || kBN % b_box_rows<MODE>() == 0, "a tile's boxes must fit its stage");
     static_assert(8 * (2 * kStages + 4) + 8 <= 256, "barrier block");
 };
 
@@ -213,6 +224,7 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
                 const CUtensorMap* ta = sh ? &tm_a_s : &tm_a_r;
                 const CUtensorMap* tb = sh ? &tm_b_s : &tm_b_r;
                 const int frow = ti.ft * BM;
+                constexpr int BBOX = b_box_rows<MODE>();
                 const int nbox = cdiv(ti.n, BBOX);
                 const uint32_t bytes = C::kNA * A_BYTES + (C::kGather ? 0u : (uint32_t)nbox * BBOX * BK * 2);
                 for (int kb = 0; kb < ti.nk; ++kb, ++it) {
@@ -370,18 +382,18 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
                         // Column j of this chunk is token t_j with routing weight w_j; lane l
                         // holds feature f0 + l.  Each block of 4 columns is transposed within
                         // groups of 4 lanes (two XOR-shuffle stages), after which lane 4g+i
-                        // holds features f0+4g .. f0+4g+3 of token t_{j0+i} and adds them into
-                        // acc with one 16-byte vector reduction (FP32 add in L2).  No shared
-                        // memory is staged, so the ring keeps it for weights.
+                        // holds features f0+4g .. f0+4g+3 of token t_{j0+i}, scales them by
+                        // w_{j0+i} (one shuffle brings the token, one the weight) and adds
+                        // them into acc with one 16-byte vector reduction (FP32 add in L2).
+                        // No shared memory is staged, so the ring keeps it for weights.
                         const int i4 = lane & 3;
                         const bool fok4 = f - i4 + 3 < a.feat_r;  // features of my group (feat_r % 8 == 0)
 #pragma unroll
                         for (int j0 = 0; j0 < 32; j0 += 4) {
                             float r[4];
 #pragma unroll
-                            for (int jj = 0; jj < 4; ++jj)
-                                r[jj] = __shfl_sync(0xffffffffu, mw[ci], j0 + jj) * __uint_as_float(v[j0 + jj]);
-                            // r[jj] = w_j * y[feature of this lane, token j0 + jj]; 4x4 transpose
+                            for (int jj = 0; jj < 4; ++jj) r[jj] = __uint_as_float(v[j0 + jj]);
+                            // r[jj] = y[feature of this lane, token j0 + jj]; 4x4 transpose
                             float t0 = (i4 & 1) ? r[0] : r[1], t1 = (i4 & 1) ? r[2] : r[3];
                             t0 = __shfl_xor_sync(0xffffffffu, t0, 1);
                             t1 = __shfl_xor_sync(0xffffffffu, t1, 1);
@@ -403,8 +415,10 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
                                 r[3] = u1;
                             }
                             const int tok = __shfl_sync(0xffffffffu, mt[ci], j0 + i4);
+                            const float wt = __shfl_sync(0xffffffffu, mw[ci], j0 + i4);
                             if (c0 + j0 + i4 < ti.n && fok4 && (unsigned)tok < (unsigned)a.T)
-                                red_add_v4_f32(a.acc + (size_t)tok * a.feat_r + (f - i4), r[0], r[1], r[2], r[3]);
+                                red_add_v4_f32(a.acc + (size_t)tok * a.feat_r + (f - i4), wt * r[0], wt * r[1],
+                                               wt * r[2], wt * r[3]);
                         }
                     }
                 } else {  // GM_DENSE

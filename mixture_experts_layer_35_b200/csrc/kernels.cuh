@@ -159,6 +159,8 @@ struct GemmMaps {
 // rows, 192 up to 150, else 256).  Narrow tiles leave shared memory for a deeper
 // weight ring.  The permute kernel's tile tables must use the same value as the launch.
 int gemm_token_tile(int mode, int T, int K, int E);
+// Rows per TMA box of FC2's h / hs tensor maps (the kernel's copies use the same box).
+constexpr int kFc2BoxRows = 32;
 cudaError_t launch_gemm(int mode, int bn, const GemmArgs& a, const GemmMaps& m, int grid, cudaStream_t s, bool pdl);
 
 // finalize: out = bf16(bf16(acc) + ys) or bf16(acc)
