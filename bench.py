@@ -217,7 +217,6 @@ def kernel_names(path: str, router: bool, launches: int = 0):
 # The capture and its command are summarised in profiles/; an entry is removed whenever
 # its kernel changes, so that a stale count is never reported.
 NCU_TRAFFIC = {
-    ("qwen36", 4096, "router", "fc1"): 1.185122e9 + 64.430848e6,
 }
 
 

@@ -22,11 +22,11 @@
 // Warp roles (one CTA per SM, persistent over a group-major tile list):
 //   warp 0      TMA producer (weights; FC2/DENSE token rows)
 //   warp 1      TMEM allocator and single-thread MMA issuer
-//   warps 2-5   epilogue: tcgen05.ld of the accumulator (warp w reads TMEM lanes of
-//               quarter w % 4), activation / scaling, stores; FC2 with wide tiles has
-//               twelve epilogue warps (2-13), the three warps of a quarter taking every
-//               third 32-token column chunk
-//   warps 6-9   FC1 only: cp.async gather of token rows of x
+//   warps 2-    epilogue: tcgen05.ld of the accumulator (warp w reads TMEM lanes of
+//               quarter w % 4), activation / scaling, stores.  Four warps, or with
+//               wide tiles eight (FC1) or twelve (FC2): the warps of a quarter take
+//               32-token column chunks in turn
+//   then        FC1 only: eight warps gathering token rows of x with cp.async
 // Shared memory holds a ring of stages (full/empty mbarriers); TMEM holds two
 // accumulator buffers so the epilogue of one tile overlaps the mainloop of the next.
 #include "kernels.cuh"
@@ -67,8 +67,10 @@ struct Cfg {
     // next to its short mainloop, so with wide tiles it gets three warps per TMEM lane
     // quarter, splitting the token columns (measured at T = 4096 / 8192 of the
     // Qwen3.6-shaped layer, FC2: 4 warps 240 / 582 us, 8 warps 144 / 322 us, 12 warps
-    // 137 / 276 us, 16 warps 140 / 304 us).
-    static constexpr int kEpiWarps = (MODE == GM_FC2 && BN > 32) ? 12 : 4;
+    // 137 / 276 us, 16 warps 140 / 304 us).  FC1 with tiles of 128+ tokens gets two
+    // per quarter (together with 8 gather warps: FC1 244 -> 227 us at T = 4096).
+    static constexpr int kEpiWarps =
+        (MODE == GM_FC2 && BN > 32) ? 12 : ((kGather && BN >= 128) ? 8 : 4);
     static constexpr int kEpiBytes = 0;  // epilogues work from registers
     static constexpr int kAccCols = kSwiglu ? 2 * kBN : kBN;
     // Two accumulator buffers (the epilogue of one tile overlaps the next mainloop) when
@@ -80,7 +82,14 @@ struct Cfg {
         (kAccBufs * kAccStride) > 256 ? 512 : ((kAccBufs * kAccStride) > 128 ? 256 : 128);
     static_assert(kAccBufs * kAccStride <= 512 || kAccBufs == 1, "accumulator buffers exceed TMEM");
     static_assert(kAccCols <= 512, "accumulator exceeds TMEM");
-    static constexpr int kThreads = 64 + 32 * kEpiWarps + (kGather ? 128 : 0);
+    // FC1 gather warps: each thread copies one 16-byte chunk (of 8 per 128-byte row) of
+    // every kGatherRowStep-th token row of a stage.  Eight warps keep more rows in flight
+    // than four (FC1 at T = 4096 of the Qwen3.6-shaped layer: 244 -> 235 us alone).
+    static constexpr int kGatherWarps = kGather ? 8 : 0;
+    static constexpr int kGatherThreads = 32 * kGatherWarps;
+    static constexpr int kGatherRowStep = kGather ? kGatherThreads / 8 : 16;  // (unused without a gather)
+    static_assert(!kGather || kBN % kGatherRowStep == 0, "gather rows must tile the token tile");
+    static constexpr int kThreads = 64 + 32 * kEpiWarps + kGatherThreads;
     // FC1 gather: stages of token rows in flight before the gather warps signal the oldest
     // one.  It must stay at most kStages - 2: the gather can only issue stage j + lag once
     // the MMA has freed that slot, so with lag = kStages - 1 the signal for stage j waits
@@ -177,7 +186,7 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kStages; ++s) {
-            mbar_init(full_bar(s), C::kGather ? 1 + 128 : 1);
+            mbar_init(full_bar(s), 1 + C::kGatherThreads);
             mbar_init(empty_bar(s), 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -439,7 +448,7 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
         }
     } else if (C::kGather) {
         // ------------------------------------------------------------ FC1 token gather
-        const int p = threadIdx.x - 192;  // 0..127
+        const int p = threadIdx.x - (64 + 32 * C::kEpiWarps);  // 0 .. kGatherThreads - 1
         const int chunk = p & 7, rsub = p >> 3;
         int it = 0;
         for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
@@ -447,10 +456,10 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
             const int kd = ti.shared ? a.kdim_s : a.kdim;
             const int nk = ti.nk;
             const int npad = cdiv(ti.n, 16) * 16;
-            int tok[C::kBN / 16];
+            int tok[C::kBN / C::kGatherRowStep];
 #pragma unroll
-            for (int j = 0; j < C::kBN / 16; ++j) {
-                const int r = rsub + 16 * j;
+            for (int j = 0; j < C::kBN / C::kGatherRowStep; ++j) {
+                const int r = rsub + C::kGatherRowStep * j;
                 tok[j] = -1;
                 if (r < ti.n && (ti.shared || ti.row0 + ti.n <= a.T * a.K)) {
                     const int src = ti.shared ? ti.row0 + r : a.perm[ti.row0 + r];
@@ -472,8 +481,8 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
                 const uint32_t bs = base_u32 + (uint32_t)s * C::kStageBytes + C::kNA * A_BYTES;
                 const int kcol = kb * BK + chunk * 8;
 #pragma unroll
-                for (int j = 0; j < C::kBN / 16; ++j) {
-                    const int r = rsub + 16 * j;
+                for (int j = 0; j < C::kBN / C::kGatherRowStep; ++j) {
+                    const int r = rsub + C::kGatherRowStep * j;
                     if (r < npad) {
                         const uint32_t dst = bs + (uint32_t)r * 128u + ((uint32_t)(chunk ^ (r & 7)) << 4);
                         const bool v = tok[j] >= 0 && kcol < kd;
