@@ -202,8 +202,9 @@ def accounting(shape, T: int, U: int, router: bool, Is: int):
 
 
 def kernel_names(path: str, router: bool, launches: int = 0):
-    """Names of a forward's kernels in launch order.  The tensor-core path routes few
-    tokens in one kernel (route + permutation), which shows as one launch fewer."""
+    """Names of a forward's kernels in launch order: the streaming path's route table,
+    the three-kernel top-k after the tensor-core router (more than 256 experts), or the
+    one-kernel top-k + permute of the other cases."""
     names = ["router"] if router else []
     if path == "small":
         return names + ["route", "fc1", "fc2"]
