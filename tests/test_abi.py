@@ -109,6 +109,8 @@ def test_path_selection_and_launch_counts():
     d = _desc(T=4, path="large")
     assert moe.select_path(d) == "large"
     assert moe.launches(d) == 6
+    d.router_logits = FAKE * 8
+    assert moe.launches(d) == 5  # logits given: no router launch
     d = _desc(T=64, path="small")
     assert moe.select_path(d) == "small"
     assert _fwd(d, ws=FAKE * 8, ws_bytes=moe.workspace_size(d)) == moe.MOE_ERR_UNSUPPORTED

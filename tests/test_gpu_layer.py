@@ -150,6 +150,24 @@ def test_many_candidates_fall_back_to_per_row_refinement(T):
     _check(TIED, d, "large")
 
 
+@pytest.mark.parametrize("T", [16, 64])
+def test_tied_router_few_tokens(T):
+    """Few tokens on the many-token path (exact few-token router, top-k, permute).  Every
+    expert has the same router row, so all logits of a row tie and the lower-id tie break
+    decides every slot."""
+    d = _util.device_layer(TIED, T, seed=6)
+    d["router_w"] = d["router_w"][:1].expand_as(d["router_w"]).contiguous()
+    _check(TIED, d, "large")
+
+
+@pytest.mark.parametrize("shape,T", [(MULTI_A, 37), (MULTI_C, 3), (gen.LARGE_E, 64)])
+def test_given_logits_few_tokens(shape, T):
+    """Caller-supplied logits at few tokens on the many-token path, skewed routing so that
+    some experts take many slots and most take none."""
+    d = _util.device_layer(shape, T, seed=8, routing="zipf")
+    _check(shape, d, "large", given_logits=True)
+
+
 def test_small_path_deterministic_and_graph_replay():
     shape = gen.QWEN36
     d = _util.device_layer(shape, 4, seed=5)
