@@ -111,8 +111,9 @@ struct PermuteArgs {
 };
 size_t permute_smem_bytes(int E);
 cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s, bool pdl);
-// Fused-path permutation: the per-expert counts were accumulated by the top-k kernel;
-// slots are placed with per-expert atomic cursors (order within an expert is not
+// Fused-path permutation: the per-expert counts were accumulated by the top-k kernel.
+// Each CTA ranks its slots per expert in shared memory and reserves one contiguous range
+// per expert with a single atomic on the expert's cursor (order within an expert is not
 // fixed).  `cursor` [E] must be zero on entry.
 cudaError_t launch_permute_fast(const PermuteArgs& a, const int* counts, int* cursor, cudaStream_t s, bool pdl);
 

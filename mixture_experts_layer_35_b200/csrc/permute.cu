@@ -132,10 +132,16 @@ __device__ void write_tile_tables(const PermuteArgs& a, int my_cnt, int* s_warp)
 __global__ void __launch_bounds__(kThreads) permute_fast_kernel(const PermuteArgs a, const int* __restrict__ counts,
                                                                int* __restrict__ cursor) {
     __shared__ int s_off[MOE_MAX_EXPERTS];
+    __shared__ int s_cnt[MOE_MAX_EXPERTS];   // this CTA's slots per expert
+    __shared__ int s_base[MOE_MAX_EXPERTS];  // this CTA's first position inside each expert
     __shared__ int s_warp[33];
     const int tid = threadIdx.x, E = a.E;
     pdl_wait();
+    const long long i = (long long)blockIdx.x * kThreads + tid;
+    const bool has = i < (long long)a.M * a.K;
+    const int e = has ? a.ids[i] : -1;  // issued before the scan, so its latency overlaps it
     const int my_cnt = (tid < E) ? counts[tid] : 0;
+    if (tid < E) s_cnt[tid] = 0;  // ordered before the counting below by the scan's barriers
     int total;
     const int off = block_exclusive_scan(my_cnt, s_warp, total);
     if (tid < E) s_off[tid] = off;
@@ -144,22 +150,24 @@ __global__ void __launch_bounds__(kThreads) permute_fast_kernel(const PermuteArg
         if (tid == 0) a.offsets[E] = total;
         if (a.tiles1) write_tile_tables(a, my_cnt, s_warp);
     }
+    // Rank of the slot among this CTA's slots of the same expert, then one global atomic
+    // per (CTA, expert) reserves the CTA's contiguous range inside the expert's segment.
+    const bool ok = has && (unsigned)e < (unsigned)E;
+    const int local = ok ? atomicAdd(&s_cnt[e], 1) : 0;
     __syncthreads();
-    const long long i = (long long)blockIdx.x * kThreads + tid;
-    if (i < (long long)a.M * a.K) {
-        const int e = a.ids[i];
-        if ((unsigned)e < (unsigned)E) {
-            const int t = (int)(i / a.K), k = (int)(i - (long long)t * a.K);
-            const int pos = s_off[e] + atomicAdd(cursor + e, 1);
-            if ((unsigned)pos < (unsigned)(a.M * a.K)) {
-                a.perm[pos] = k * a.M + t;
-                if (a.inv) a.inv[k * a.M + t] = pos;
-            } else {  // the counts disagree with the ids: flag it, place nothing out of range
-                set_dev_error(a.err, MOE_DEVERR_BAD_INDEX);
-            }
-        } else {
-            set_dev_error(a.err, MOE_DEVERR_BAD_EXPERT_ID);
+    if (tid < E) s_base[tid] = s_cnt[tid] > 0 ? atomicAdd(cursor + tid, s_cnt[tid]) : 0;
+    __syncthreads();
+    if (ok) {
+        const int t = (int)(i / a.K), k = (int)(i - (long long)t * a.K);
+        const int pos = s_off[e] + s_base[e] + local;
+        if ((unsigned)pos < (unsigned)(a.M * a.K)) {
+            a.perm[pos] = k * a.M + t;
+            if (a.inv) a.inv[k * a.M + t] = pos;
+        } else {  // the counts disagree with the ids: flag it, place nothing out of range
+            set_dev_error(a.err, MOE_DEVERR_BAD_INDEX);
         }
+    } else if (has) {
+        set_dev_error(a.err, MOE_DEVERR_BAD_EXPERT_ID);
     }
     pdl_trigger();
 }
