@@ -45,16 +45,6 @@ __host__ __device__ constexpr int b_box_rows() {
     return MODE == GM_FC2 ? kFc2BoxRows : 16;
 }
 
-// Token rows per tile (MMA N) of each mode at prefill sizes: FC2 takes up to 256 so that
-// an expert's W2 tile is streamed once for all its tokens; FC1 keeps 128 so that its gate
-// and up accumulators stay double-buffered in TMEM.  When every expert has at most 32
-// rows (T <= 32) both use 32-row tiles, whose smaller token stages leave room for a
-// deeper weight ring.
-template <int MODE>
-constexpr int default_bn() {
-    return MODE == GM_FC2 ? 256 : (MODE == GM_DENSE ? kDenseTokenTile : 128);
-}
-
 template <int MODE, int BN>
 struct Cfg {
     static constexpr bool kGather = (MODE == GM_FC1_SWIGLU || MODE == GM_FC1_RELU2);
@@ -557,7 +547,7 @@ static cudaError_t launch_mode(const GemmArgs& a, const GemmMaps& m, int grid, c
 }
 
 int gemm_token_tile(int mode, int T, int K, int E) {
-    if (mode == GM_DENSE) return default_bn<GM_DENSE>();
+    if (mode == GM_DENSE) return kDenseTokenTile;
     if (T <= 32) return 32;  // no expert has more rows than a tile
     const double rows = (double)T * K / E;  // average rows per expert
     // FC2: a tile that covers an expert's rows streams its W2 slice once; 192 holds almost
@@ -593,7 +583,7 @@ cudaError_t launch_gemm(int mode, int bn, const GemmArgs& a, const GemmMaps& m, 
             if (bn == 192) return launch_mode<GM_FC2, 192>(a, m, grid, s, pdl);
             if (bn == 256) return launch_mode<GM_FC2, 256>(a, m, grid, s, pdl);
             break;
-        case GM_DENSE: return launch_mode<GM_DENSE, default_bn<GM_DENSE>()>(a, m, grid, s, pdl);
+        case GM_DENSE: return launch_mode<GM_DENSE, kDenseTokenTile>(a, m, grid, s, pdl);
     }
     return cudaErrorInvalidValue;
 }

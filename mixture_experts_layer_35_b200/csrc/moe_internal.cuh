@@ -46,19 +46,6 @@ __device__ __forceinline__ float dot8(const uint4& a, const uint4& b, float acc)
     return acc;
 }
 
-// Same in FP64: BF16 x BF16 products are exact in double, so only the additions round.
-__device__ __forceinline__ double dot8_f64(const uint4& a, const uint4& b, double acc) {
-    acc = fma((double)bf16lo(a.x), (double)bf16lo(b.x), acc);
-    acc = fma((double)bf16hi(a.x), (double)bf16hi(b.x), acc);
-    acc = fma((double)bf16lo(a.y), (double)bf16lo(b.y), acc);
-    acc = fma((double)bf16hi(a.y), (double)bf16hi(b.y), acc);
-    acc = fma((double)bf16lo(a.z), (double)bf16lo(b.z), acc);
-    acc = fma((double)bf16hi(a.z), (double)bf16hi(b.z), acc);
-    acc = fma((double)bf16lo(a.w), (double)bf16lo(b.w), acc);
-    acc = fma((double)bf16hi(a.w), (double)bf16hi(b.w), acc);
-    return acc;
-}
-
 // Eight exact BF16 products formed in FP32, accumulated in FP64.
 __device__ __forceinline__ double dot8_f64p(const uint4& a, const uint4& b, double acc) {
     acc += (double)__fmul_rn(bf16lo(a.x), bf16lo(b.x));
@@ -208,14 +195,6 @@ __device__ __forceinline__ uint64_t l2_policy_evict_first() {
     uint64_t p;
     asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
     return p;
-}
-__device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const CUtensorMap* tm, uint32_t bar, int c0, int c1,
-                                                 uint64_t pol) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
-        " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(tm)), "r"(bar), "r"(c0), "r"(c1), "l"(pol)
-        : "memory");
 }
 __device__ __forceinline__ void tma_load_3d_hint(uint32_t dst, const CUtensorMap* tm, uint32_t bar, int c0, int c1,
                                                  int c2, uint64_t pol) {
