@@ -299,7 +299,21 @@ class Bench:
         clk = sampler.stop() if sampler else None
         barrier(world, self.device)
         per = [a.elapsed_time(b) for a, b in evs]
+        self.last_step_s = statistics.median(per) / 1e3 + 2e-5
         return per, clk
+
+    def clock_soak(self, seconds: float):
+        """Clocks while the same step (L2 flush + graph replay) repeats back to back for
+        about ``seconds``: a longer window than a short timed region gives the sampler."""
+        n = max(1, int(seconds / max(self.last_step_s, 1e-5)))
+        sampler = ClockSampler(self.device.index)
+        for _ in range(n):
+            self.flush()
+            self.step()
+        torch.cuda.synchronize(self.device)
+        out = sampler.stop()
+        out["steps"] = n
+        return out
 
     def per_kernel(self, steps: int):
         """Average duration of each kernel of the step, from events recorded between the
@@ -399,6 +413,39 @@ def cpu_oracle_rate(shape, d, budget_s: float, max_tokens: int):
     return done / dt, done, dt
 
 
+def cpu_oracle_rate_all_cores(shape, d, tokens_per_core: int):
+    """Tokens/s of the same single-threaded oracle sharded by token ranges over every host
+    core as separate processes (oracle.parallel).  The workers are started, and have
+    mapped the inputs, before the timed span."""
+    from oracle import parallel as opar
+    h = gen.to_numpy_inputs(d)
+    T = h["x"].shape[0]
+    cores = opar.host_cores()
+    n = min(T, cores * tokens_per_core)
+    rows = np.random.default_rng(1).permutation(T)[:n].astype(np.int32)
+    with opar.ShardedOracle(shape, h, cores) as pool:
+        pool.forward(rows[:cores])  # workers started and inputs mapped before the timed span
+        t0 = time.perf_counter()
+        pool.forward(rows)
+        dt = time.perf_counter() - t0
+    return n / dt, n, dt, cores
+
+
+def host_cpu_info():
+    """Core count and CPU model of the host (lscpu), for the CPU-baseline lines."""
+    from oracle import parallel as opar
+    model = None
+    try:
+        r = subprocess.run(["lscpu"], capture_output=True, text=True, timeout=10)
+        for line in r.stdout.splitlines():
+            if line.startswith("Model name:"):
+                model = line.split(":", 1)[1].strip()
+                break
+    except (OSError, subprocess.SubprocessError):
+        pass
+    return {"nproc": opar.host_cores(), "cpu_count": os.cpu_count(), "model": model}
+
+
 def run_ours(args, rank, local, world):
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
@@ -431,6 +478,7 @@ def run_ours(args, rank, local, world):
     e2e_serial = max_over_ranks(e2e_serial, world, device)
     e2e_value = world * args.T / (e2e_pipe / 1e3)
 
+    clk_soak = b.clock_soak(args.soak_s) if args.soak_s > 0 else None
     dev_err = b.moe.get_error(b.ws)
     line = {
         "metric": METRIC,
@@ -454,6 +502,7 @@ def run_ours(args, rank, local, world):
         "gpu_launches": b.launches * args.steps,
         "device_error": dev_err,
         "clocks": clk,
+        "clocks_soak": clk_soak,
         "us_per_step_p10_p50_p90": [float(np.percentile(per, q)) * 1e3 for q in (10, 50, 90)],
     }
     del b
@@ -462,9 +511,17 @@ def run_ours(args, rank, local, world):
         line["sweep"] = sweep(args, device, peaks)
     if rank == 0 and world == 1 and not args.no_cpu:
         dcpu = gen.make_layer(shape, args.T, seed=args.seed, device=str(device), routing=args.routing)
-        rate, n, dt = cpu_oracle_rate(shape, dcpu, args.cpu_budget, 400)
-        line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                                "sample": f"{n} tokens of the same workload in {dt:.1f} s (single-threaded FP64 C)"}
+        rate1, n1, dt1 = cpu_oracle_rate(shape, dcpu, args.cpu_budget / 3, 400)
+        per_core = max(1, int(rate1 * args.cpu_budget * 2 / 3))
+        rate, n, dt, cores = cpu_oracle_rate_all_cores(shape, dcpu, per_core)
+        info = host_cpu_info()
+        line["cpu_baseline"] = {
+            "value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n} random tokens of the same workload in {dt:.1f} s: the single-threaded FP64 C oracle "
+                      f"sharded by token ranges over {cores} processes",
+            "host": info,
+            "single_core": {"value": rate1, "unit": "tokens/s", "cores": 1,
+                            "sample": f"{n1} tokens in {dt1:.1f} s on one core"}}
         del dcpu
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -485,12 +542,14 @@ def sweep(args, device, peaks):
         print(f"sweep: {cfg} T={T}", file=sys.stderr, flush=True)
         try:
             b = Bench(shape, T, device, seed=1, routing="router", path=args.path)
-            per, _ = b.timed(8, 2)
+            per, _ = b.timed(args.sweep_steps, 5)
             med = statistics.median(per)
             U = b.distinct_experts()
             acc = accounting(shape, T, U, True, b.Is)["layer"]
             rf = roofline_of(acc, med / 1e3, peaks)
-            rows.append({"config": cfg, "T": T, "path": b.path, "us": med * 1e3, "tokens_per_s": T / (med / 1e3),
+            rows.append({"config": cfg, "T": T, "path": b.path, "us": med * 1e3,
+                         "us_p10_p90": [float(np.percentile(per, 10)) * 1e3, float(np.percentile(per, 90)) * 1e3],
+                         "steps": len(per), "tokens_per_s": T / (med / 1e3),
                          "distinct_experts": U, "bound": rf["bound"], "frac_of_roofline": rf["frac"],
                          "achieved": rf["achieved"], "unit": rf["unit"],
                          "device_error": b.moe.get_error(b.ws)})
@@ -614,17 +673,30 @@ def run_reference(args, rank, local, world):
     import oracle
     h = gen.to_numpy_inputs(d)
     del d
-    sample = max(1, args.ref_tokens)
+    from oracle import parallel as opar
+    cores = opar.host_cores() if args.ref_cores == 0 else args.ref_cores
+    sample = max(1, args.ref_tokens) * cores
     rng = np.random.default_rng(0)
     times = []
-    for i in range(args.warmup + args.steps):
-        rows = rng.choice(args.T, sample, replace=False).astype(np.int32)
-        t0 = time.perf_counter()
-        oracle.forward(shape, h, rows)
-        dt = time.perf_counter() - t0
-        if i >= args.warmup:
-            times.append(dt)
+    # The worker processes and their memory-mapped copy of the inputs are set up once,
+    # outside the timed steps (as loading the weights is for the GPU arm).
+    pool = opar.ShardedOracle(shape, h, cores) if cores > 1 else None
+    try:
+        for i in range(args.warmup + args.steps):
+            rows = rng.choice(args.T, min(sample, args.T), replace=False).astype(np.int32)
+            t0 = time.perf_counter()
+            if pool is None:
+                oracle.forward(shape, h, rows)
+            else:
+                pool.forward(rows)
+            dt = time.perf_counter() - t0
+            if i >= args.warmup:
+                times.append(dt)
+    finally:
+        if pool is not None:
+            pool.close()
     tot = sum(times)
+    sample = min(sample, args.T)
     value = sample * args.steps / tot
     line = {"impl": "reference", "metric": METRIC,
             "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -632,8 +704,10 @@ def run_reference(args, rank, local, world):
             "dtype": "f64", "data": "synthetic (seeded generator)",
             "config": {"workload": f"{shape.name} T={args.T} routing={args.routing}",
                        "sample": f"{sample} tokens per step"},
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                             "sample": f"{sample} random tokens of the workload per step, single-threaded FP64 C"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{sample} random tokens of the workload per step, the single-threaded "
+                                       f"FP64 C oracle sharded by token ranges over {cores} processes",
+                             "host": host_cpu_info()},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -656,7 +730,11 @@ def main(argv=None):
     p.add_argument("--sweep-all", action="store_true")
     p.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline (profiling runs)")
     p.add_argument("--cpu-budget", type=float, default=15.0)
-    p.add_argument("--ref-tokens", type=int, default=4)
+    p.add_argument("--ref-tokens", type=int, default=4, help="reference arm: tokens per core per step")
+    p.add_argument("--ref-cores", type=int, default=0, help="reference arm: processes (0 = every host core)")
+    p.add_argument("--sweep-steps", type=int, default=30)
+    p.add_argument("--soak-s", type=float, default=1.0,
+                   help="seconds of repeated steps after the timed region, for a longer clock record")
     args = p.parse_args(argv)
     args.warmup = max(args.warmup, 3)
     rank, local, world = dist_env()

@@ -59,6 +59,9 @@ typedef enum { MOE_PATH_AUTO = 0, MOE_PATH_SMALL = 1, MOE_PATH_LARGE = 2 } moe_p
 #define MOE_DEVERR_BAD_EXPERT_ID 0x1   /* an expert id outside [0, E) reached the permute */
 #define MOE_DEVERR_WAIT_TIMEOUT 0x2    /* a bounded device-side wait gave up */
 #define MOE_DEVERR_BAD_INDEX 0x4       /* a computed row/slot index fell outside its buffer; the access was skipped */
+#define MOE_DEVERR_ROUTER_BOUND 0x8    /* a tensor-core router logit lay outside its proven error bound: the
+                                          hardware accumulation model behind exact routing did not hold, so
+                                          this call's expert ids are not guaranteed to be the exact ones */
 
 /* Limits of this build. */
 #define MOE_MAX_EXPERTS 1024
@@ -149,15 +152,37 @@ int moe_select_path(const moe_layer_desc* d);
  *                router_logits when those are given).
  *   ws, ws_bytes workspace of at least moe_workspace_size(d) bytes, 256-byte aligned;
  *                its first 256 bytes hold the device error word.
- * The shared expert uses the routed activation and no gate.  Routing is computed with
- * an FP32 logit accumulation whose order differs from a reference FP64 sum; experts
- * whose keys differ by less than that rounding may be chosen either way. */
+ * The shared expert uses the routed activation and no gate.
+ * Routing is exact: expert ids and weights are those of the exact logits (the FP32
+ * rounding of the exact sum of the BF16 products, up to an FP64 summation error far
+ * below an FP32 unit).  Up to 64 tokens the logits are computed that way directly.  With
+ * more tokens a tensor-core GEMM screens them; every expert whose key lies within twice
+ * a proven per-token error bound of the K-th key is re-evaluated exactly, so no expert
+ * outside that window can belong to the top K.  The bound assumes the tensor core's FP32
+ * accumulation is faithful to within 2 units in the last place per addition; a logit
+ * found outside it sets MOE_DEVERR_ROUTER_BOUND (read it with moe_get_error). */
 moe_status_t moe_fused_forward(const moe_layer_desc* d, const void* x, void* out,
                                float* topk_w_out, int32_t* topk_ids_out, float* logits_out,
                                void* ws, size_t ws_bytes, void* stream);
 
 /* Number of kernels moe_fused_forward enqueues for this description (for accounting). */
 int moe_fused_forward_launches(const moe_layer_desc* d);
+
+/* Token rows per tile of the many-token path's grouped GEMMs for this description (the
+ * MMA N of one tile: FC1 and FC2 each pick one width per call from T * top_k / E).
+ * Returns MOE_OK, or the description's validation error. */
+moe_status_t moe_token_tiles(const moe_layer_desc* d, int* fc1_rows, int* fc2_rows);
+
+/* Where moe_fused_forward keeps an intermediate in the workspace, for inspection after a
+ * call (tests, debugging).  Valid after a many-token-path (MOE_PATH_LARGE) call with this
+ * description, until the workspace is reused:
+ *   MOE_WS_TOPK_IDS  [T, K] int32 expert ids      MOE_WS_TOPK_W  [T, K] FP32 weights
+ *   MOE_WS_OFFSETS   [E + 1] int32 expert offsets of the internal permutation
+ *   MOE_WS_PERM      [T * K] int32 source slots k * T + t grouped by expert (the order
+ *                    within an expert is unspecified; the set of each expert is exact)
+ * Writes the region's byte offset from the workspace start and its size. */
+enum { MOE_WS_TOPK_IDS = 0, MOE_WS_TOPK_W = 1, MOE_WS_OFFSETS = 2, MOE_WS_PERM = 3 };
+moe_status_t moe_workspace_region(const moe_layer_desc* d, int region, size_t* offset, size_t* bytes);
 
 /* moe_fused_forward with per-kernel timing: `events` holds n_events >= launches + 1
  * cudaEvent_t handles created by the caller; event i is recorded on `stream` before the
@@ -184,15 +209,27 @@ moe_status_t moe_fused_forward_timed(const moe_layer_desc* d, const void* x, voi
  *     more scratch than that (moe_workspace_size(d) > MOE_NOALLOC_SCRATCH_BYTES); the
  *     other errors are those of moe_fused_forward.
  *   - The first call on each device (with that device current) looks up the array's
- *     device address; make that first call before any stream capture begins.
+ *     device address and clears its error word; make that first call before any
+ *     stream capture begins.  The lookup is repeated when the device's CUDA context
+ *     changes (after cudaDeviceReset).
  *   - All calls on a device share the array: calls whose GPU work overlaps (different
  *     streams, concurrent graph launches) race and give wrong results.
- *   - Device error flags are cleared at the start of each call and are not reported.
+ *   - Device error flags (MOE_DEVERR_*) accumulate in the array's error word over calls
+ *     until moe_noalloc_get_error reads and clears them.
  * ---------------------------------------------------------------------------------- */
 #define MOE_NOALLOC_SCRATCH_BYTES (4u << 20)
 moe_status_t moe_fused_forward_noalloc(const moe_layer_desc* d, const void* x, void* out,
                                        float* topk_w_out, int32_t* topk_ids_out, float* logits_out,
                                        void* stream);
+
+/* moe_noalloc_get_error -- moe_get_error for the static scratch of the current device:
+ * reads and clears the error word that moe_fused_forward_noalloc calls on this device
+ * write.  Synchronises `stream`; allocates nothing (on a device with no call yet, it sets
+ * the array up as the first call would).
+ *   code  out: OR of MOE_DEVERR_* flags set since the last read (0 = none).
+ * Returns MOE_ERR_DEVICE when code != 0, MOE_OK otherwise, MOE_ERR_CUDA if a CUDA call
+ * fails, MOE_ERR_INVALID_ARG when code is NULL. */
+moe_status_t moe_noalloc_get_error(int* code, void* stream);
 
 /* ------------------------------------------------------------------------------------
  * moe_get_error -- read and clear the device error word at the start of `ws`

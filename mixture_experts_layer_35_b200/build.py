@@ -1,6 +1,10 @@
 """Build libmoe.so in-tree: every kernel is compiled for sm_100a only.
 
     python -m mixture_experts_layer_35_b200.build [--force] [--ptxas-v]
+
+Each CUDA source compiles to its own object in parallel (no cross-file device code:
+every translation unit is a separate device module), then one link step makes the
+shared library.
 """
 from __future__ import annotations
 
@@ -8,6 +12,7 @@ import glob
 import os
 import subprocess
 import sys
+from concurrent.futures import ThreadPoolExecutor
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
@@ -15,8 +20,10 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmoe.so")
 
-NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
-              "-Xcompiler", "-fPIC", "-shared", "-cudart", "static"]
+OBJ_DIR = os.path.join(PKG, "_build")
+COMPILE_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
+                 "-Xcompiler", "-fPIC"]
+LINK_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-cudart", "static"]
 
 
 def _nvcc() -> str:
@@ -41,11 +48,27 @@ def _stale() -> bool:
 def build(force: bool = False, ptxas_verbose: bool = False) -> str:
     if not force and not _stale():
         return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [_nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-o", tmp, *sources()]
-    if ptxas_verbose:
-        cmd[1:1] = ["-Xptxas", "-v"]
-    subprocess.check_call(cmd)
+    os.makedirs(OBJ_DIR, exist_ok=True)
+    tag = os.getpid()
+
+    def compile_one(src):
+        obj = os.path.join(OBJ_DIR, os.path.basename(src)[:-3] + f".{tag}.o")
+        cmd = [_nvcc(), *COMPILE_FLAGS, "-I", INCLUDE, "-I", CSRC, "-c", "-o", obj, src]
+        if ptxas_verbose:
+            cmd[1:1] = ["-Xptxas", "-v"]
+        subprocess.check_call(cmd)
+        return obj
+
+    srcs = sources()
+    with ThreadPoolExecutor(max_workers=max(1, min(len(srcs), os.cpu_count() or 1))) as ex:
+        objs = list(ex.map(compile_one, srcs))
+    tmp = LIB + f".tmp{tag}"
+    try:
+        subprocess.check_call([_nvcc(), *LINK_FLAGS, "-o", tmp, *objs])
+    finally:
+        for o in objs:
+            if os.path.exists(o):
+                os.remove(o)
     os.replace(tmp, LIB)
     return LIB
 

@@ -18,8 +18,11 @@ struct WsLayout {
 };
 // Candidate-list capacity per token of the three-kernel top-k (rows with more fall back).
 constexpr size_t kCandPerRow = 32;
-// Slot counters: per-expert counts, per-expert cursors, then the candidate count.
+// Counters zeroed before each many-token call: per-expert counts, per-expert cursors,
+// then the candidate count and the router weight-row norm bound (a float, atomicMax).
 inline size_t counter_ints(size_t E) { return 2 * (E + 2) + 4; }
+inline size_t cand_count_int(size_t E) { return 2 * (E + 2); }
+inline size_t wnorm2_int(size_t E) { return 2 * (E + 2) + 1; }
 WsLayout layout(const moe_layer_desc* d) {
     const size_t T = (size_t)d->T, E = (size_t)d->E, K = (size_t)d->top_k, H = (size_t)d->H, I = (size_t)d->I,
                  Is = (size_t)d->I_shared;
@@ -39,7 +42,7 @@ WsLayout layout(const moe_layer_desc* d) {
     L.tiles2 = take((E + 2) * 4);
     L.counts = take(counter_ints(E) * 4);
     L.perm = take(T * K * 4);
-    L.cand = take(T * (2 + 3 * kCandPerRow) * 4);  // row_base, row_n, cand_row, cand_e, cand_val
+    L.cand = take(T * (3 + 3 * kCandPerRow) * 4);  // row_base, row_n, row_eps, cand_row, cand_e, cand_val
     L.h = take(T * K * I * 2);
     L.hs = take(T * Is * 2);
     L.acc = take(T * H * 4);
@@ -127,8 +130,8 @@ bool map3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint
     } while (0)
 
 // Router logits x . Wr^T on the tensor cores for many tokens (A = Wr, B = x rows).
-moe_status_t run_router_dense(const moe_layer_desc* d, const bf16* x, float* logits, float* copy, int sms,
-                              cudaStream_t s, int* err, bool pdl) {
+moe_status_t run_router_dense(const moe_layer_desc* d, const bf16* x, float* logits, float* copy, float* wnorm2,
+                              int sms, cudaStream_t s, int* err, bool pdl) {
     GemmArgs g;
     std::memset(&g, 0, sizeof(g));
     g.T = d->T;
@@ -139,6 +142,7 @@ moe_status_t run_router_dense(const moe_layer_desc* d, const bf16* x, float* log
     g.dense = 1;
     g.logits = logits;
     g.logits_copy = copy;
+    g.wnorm2 = wnorm2;
     g.err = err;
     GemmMaps m;
     std::memset(&m, 0, sizeof(m));
@@ -242,6 +246,31 @@ int moe_select_path(const moe_layer_desc* d) {
     return resolve_path(d);
 }
 
+moe_status_t moe_token_tiles(const moe_layer_desc* d, int* fc1_rows, int* fc2_rows) {
+    const moe_status_t st = validate_desc(d);
+    if (st != MOE_OK) return st;
+    if (!fc1_rows || !fc2_rows) return MOE_ERR_INVALID_ARG;
+    const int fc1_mode = d->act == MOE_ACT_SWIGLU ? GM_FC1_SWIGLU : GM_FC1_RELU2;
+    *fc1_rows = gemm_token_tile(fc1_mode, d->T, d->top_k, d->E);
+    *fc2_rows = gemm_token_tile(GM_FC2, d->T, d->top_k, d->E);
+    return MOE_OK;
+}
+
+moe_status_t moe_workspace_region(const moe_layer_desc* d, int region, size_t* offset, size_t* bytes) {
+    const moe_status_t st = validate_desc(d);
+    if (st != MOE_OK) return st;
+    if (!offset || !bytes) return MOE_ERR_INVALID_ARG;
+    const WsLayout L = layout(d);
+    const size_t TK = (size_t)d->T * d->top_k;
+    switch (region) {
+        case MOE_WS_TOPK_IDS: *offset = L.topk_ids; *bytes = TK * 4; return MOE_OK;
+        case MOE_WS_TOPK_W: *offset = L.topk_w; *bytes = TK * 4; return MOE_OK;
+        case MOE_WS_OFFSETS: *offset = L.offsets; *bytes = ((size_t)d->E + 1) * 4; return MOE_OK;
+        case MOE_WS_PERM: *offset = L.perm; *bytes = TK * 4; return MOE_OK;
+    }
+    return MOE_ERR_INVALID_ARG;
+}
+
 // The tensor-core router runs when the logits are not given and the few-token router does
 // not apply.  Its top-k is split in three kernels for more than 256 experts: there the
 // one-kernel top-k, whose warps hold 16+ logits each and refine their candidates one after
@@ -310,7 +339,8 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
         if (T <= 64 && router_small_supported(H)) {
             MOE_CK(launch_router_small(x, static_cast<const bf16*>(d->router_w), T, H, E, lg, nullptr, err, s, false));
         } else {
-            st = run_router_dense(d, x, lg, nullptr, sms, s, err, false);
+            float* wn2 = reinterpret_cast<float*>(w8 + L.counts) + wnorm2_int(E);
+            st = run_router_dense(d, x, lg, nullptr, wn2, sms, s, err, false);
             if (st != MOE_OK) return st;
             dense_router = true;
         }
@@ -372,14 +402,16 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
     const int bn1 = gemm_token_tile(fc1_mode, T, K, E), bn2 = gemm_token_tile(GM_FC2, T, K, E);
     // 2. top-k (also counts the slots per expert; the counters were cleared in step 0)
     if (!mark()) return MOE_ERR_CUDA;
-    RefineArgs ra = {x, static_cast<const bf16*>(d->router_w), H, logits_rw};
+    RefineArgs ra = {x, static_cast<const bf16*>(d->router_w), H, logits_rw,
+                     reinterpret_cast<const float*>(counts + wnorm2_int(E)), err};
     if (dense_router && split_topk_mode(d)) {  // screen, refine, final
         int* cbase = reinterpret_cast<int*>(w8 + L.cand);
         CandList cl;
-        cl.count = counts + 2 * (E + 2);
+        cl.count = counts + cand_count_int(E);
         cl.row_base = cbase;
         cl.row_n = cbase + T;
-        cl.cand_row = cbase + 2 * (size_t)T;
+        cl.row_eps = reinterpret_cast<float*>(cbase + 2 * (size_t)T);
+        cl.cand_row = cbase + 3 * (size_t)T;
         cl.cand_e = cl.cand_row + kCandPerRow * (size_t)T;
         cl.cand_val = reinterpret_cast<float*>(cl.cand_e + kCandPerRow * (size_t)T);
         cl.cap = (int)(kCandPerRow * (size_t)T);

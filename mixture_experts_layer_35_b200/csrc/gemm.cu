@@ -17,7 +17,10 @@
 //       vector reductions, 4 consecutive features of one token per lane ("weighted output
 //       combination").
 //       The shared expert is one more group whose FC2 output is rounded to BF16 into ys.
-//   DENSE: router logits, A = Wr (128 experts per tile), B = x rows (TMA).
+//   DENSE: router logits, A = Wr (128 experts per tile), B = x rows (TMA).  Four more
+//       warps read each A tile out of the ring as it arrives and sum the squares of its
+//       rows: the squared L2 norm of every router weight row, whose maximum bounds the
+//       tensor-core logits' accumulation error (used by the top-k kernels).
 //
 // Warp roles (one CTA per SM, persistent over a group-major tile list):
 //   warp 0      TMA producer (weights; FC2/DENSE token rows)
@@ -27,6 +30,7 @@
 //               wide tiles eight (FC1) or twelve (FC2): the warps of a quarter take
 //               32-token column chunks in turn
 //   then        FC1 only: eight warps gathering token rows of x with cp.async
+//               DENSE only: four warps summing squares of the weight rows in the ring
 // Shared memory holds a ring of stages (full/empty mbarriers); TMEM holds two
 // accumulator buffers so the epilogue of one tile overlaps the mainloop of the next.
 #include "kernels.cuh"
@@ -79,7 +83,9 @@ struct Cfg {
     static constexpr int kGatherThreads = 32 * kGatherWarps;
     static constexpr int kGatherRowStep = kGather ? kGatherThreads / 8 : 16;  // (unused without a gather)
     static_assert(!kGather || kBN % kGatherRowStep == 0, "gather rows must tile the token tile");
-    static constexpr int kThreads = 64 + 32 * kEpiWarps + kGatherThreads;
+    // DENSE: one thread per A row (128) sums the squares of that weight row.
+    static constexpr int kNormWarps = (MODE == GM_DENSE) ? BM / 32 : 0;
+    static constexpr int kThreads = 64 + 32 * kEpiWarps + kGatherThreads + 32 * kNormWarps;
     // FC1 gather: stages of token rows in flight before the gather warps signal the oldest
     // one.  It must stay at most kStages - 2: the gather can only issue stage j + lag once
     // the MMA has freed that slot, so with lag = kStages - 1 the signal for stage j waits
@@ -177,7 +183,7 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kStages; ++s) {
             mbar_init(full_bar(s), 1 + C::kGatherThreads);
-            mbar_init(empty_bar(s), 1);
+            mbar_init(empty_bar(s), 1 + C::kNormWarps);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(tfull_bar(b), 1);
@@ -492,6 +498,40 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
         cp_async_wait<0>();
         fence_proxy_async_smem();
         for (int j = max(0, it - C::kLag); j < it; ++j) mbar_arrive(full_bar(j % C::kStages));
+    } else if (C::kNormWarps) {
+        // ------------------------------------------------------------ DENSE: weight-row norms
+        // Thread r owns A row r of every stage: its 64 BF16 values occupy bytes
+        // [128 r, 128 r + 128) of the tile (the 128-byte swizzle only permutes the 16-byte
+        // chunks inside a row), so the sum of their squares needs no unswizzling.  Rows
+        // past E are zero-filled by TMA.  The FP32 sum of H squares is within a relative
+        // H * 2^-24 of the exact value; it is scaled up by (1 + 2^-8) (H <= 2^16), so the
+        // result is an upper bound.  The maximum over rows goes to a.wnorm2 (atomicMax on
+        // the bits of a non-negative float orders like the float).
+        const int r = threadIdx.x - (64 + 32 * C::kEpiWarps + C::kGatherThreads);
+        int it = 0;
+        for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
+            const TileInfo ti = decode_tile<C::kBN>(a, s_tiles, s_offs, G, tile);
+            float ss = 0.0f;
+            bool ok = true;
+            for (int kb = 0; kb < ti.nk; ++kb, ++it) {
+                const int s = it % C::kStages;
+                const uint32_t ph = (uint32_t)(it / C::kStages) & 1u;
+                if (!mbar_wait(full_bar(s), ph, abort_flag, a.err)) {
+                    ok = false;
+                    break;
+                }
+                const uint4* row = reinterpret_cast<const uint4*>(base + (size_t)s * C::kStageBytes + (size_t)r * 128);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) ss = dot8(row[c], row[c], ss);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(empty_bar(s));
+            }
+            if (!ok) break;
+            float m = ss * (1.0f + 0x1p-8f);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            if (lane == 0 && a.wnorm2) atomicMax(reinterpret_cast<int*>(a.wnorm2), __float_as_int(m));
+        }
     }
 
     tc_fence_before();

@@ -33,6 +33,8 @@ struct RefineArgs {
     const bf16* wr;      // [E, H]
     int H;
     float* logits_rw;    // refined logits are written back here (the logits buffer)
+    const float* wnorm2; // max over experts of |Wr[e]|_2^2 (upper bound), from the router GEMM
+    int* err;            // device error word (MOE_DEVERR_ROUTER_BOUND)
 };
 cudaError_t launch_topk(const void* logits, bool bf16_in, int M, int E, int K, int score, const float* bias,
                         int renorm, float* topk_w, int32_t* topk_ids, int32_t* src_idx, float* w_copy,
@@ -46,6 +48,7 @@ struct CandList {
     int* cand_row;    // [cap]
     int* cand_e;      // [cap]
     float* cand_val;  // [cap] exact logits
+    float* row_eps;   // [M] error bound of each row's tensor-core logits
     int cap;
 };
 // screen, refine and final kernels; `mark` (optional) records a timing event between them.
@@ -146,6 +149,8 @@ struct GemmArgs {
     float* logits_copy;      // GM_DENSE optional second output
     float* zero_ptr;         // FC1: buffer zeroed by the epilogue warps before their tiles
     size_t zero_n;           //      (floats, multiple of 4)
+    float* wnorm2;           // GM_DENSE: max over experts of |Wr[e]|_2^2 (upper bound), atomicMax;
+                             //           zero on entry, or null
     int* err;
 };
 struct GemmMaps {

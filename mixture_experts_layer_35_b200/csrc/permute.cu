@@ -1,9 +1,14 @@
 // permute.cu -- group the M*K token slots by expert (FlashInfer PR #4646, walkthrough:
 // routing permutation; review notes: count reduction, exclusive scan, per-expert
-// offsets).  Unpadded and deterministic: within an expert, slots are in ascending token
-// order.
+// offsets).  Unpadded.
 //
-// One CTA of 32 warps.  The tokens are split into 32 contiguous ranges, one per warp.
+// permute_kernel (the moe_permute entry point) is deterministic: within an expert, slots
+// are in ascending token order.  permute_fast_kernel (inside moe_fused_forward) places
+// slots with per-expert atomic cursors, so its order within an expert changes from run to
+// run; its offsets and the set of slots of each expert do not.  Only the order of the FP32
+// additions into the routed accumulator depends on it.
+//
+// permute_kernel: one CTA of 32 warps.  The tokens are split into 32 contiguous ranges, one per warp.
 //   1. each warp histograms its range into its own row hist[w][e] (shared memory);
 //   2. per expert, an exclusive scan down the 32 warp rows gives each warp's start
 //      inside the expert; a block scan over experts gives the expert offsets;
@@ -128,7 +133,8 @@ __device__ void write_tile_tables(const PermuteArgs& a, int my_cnt, int* s_warp)
 }
 
 // Every CTA scans the counts into offsets (E <= 1024 values); CTA 0 also publishes the
-// offsets and the tile tables; each thread then places one slot.
+// offsets and the tile tables; each thread then places one slot.  The order of the slots
+// within an expert's segment is unspecified (CTA and atomic arrival order).
 __global__ void __launch_bounds__(kThreads) permute_fast_kernel(const PermuteArgs a, const int* __restrict__ counts,
                                                                int* __restrict__ cursor) {
     __shared__ int s_off[MOE_MAX_EXPERTS];

@@ -5,19 +5,47 @@
 
 namespace moe {
 
-// Tensor-core router logits carry the MMA's FP32 accumulation error: at most 1.4e-5 on
-// the T = 4096 workloads (|l| < 5, measured against the exact logits); the routing window
-// assumes at most 2e-4.
-static constexpr float kTcLogitErr = 2e-4f;
+// Error bound of the tensor-core router logits of one token row (warp-collective).
+// The MMA forms every BF16 x BF16 product exactly in FP32 and sums the H products of a
+// logit (zero padding included) in FP32.  Whatever the association order and whether
+// each addition rounds or truncates, as long as every addition step is within 2 units
+// in the last place of an FP32 result -- or, for a multi-operand adder that aligns up to
+// 17 addends to the largest one and truncates them, within one such unit per addend --
+// the computed logit lies within H * 2^-22 * sum_h |x_h w_h| of the exact sum.  Cauchy-
+// Schwarz bounds the sum by |x_t|_2 * max_e |Wr[e]|_2; the router GEMM supplies an upper
+// bound of max_e |Wr[e]|_2^2, and |x_t|_2^2 is summed here in FP32 and scaled up by
+// (1 + 2^-8) to cover its own rounding (H <= 2^16).  A final factor (1 + 2^-8) covers the
+// roundings of this product.  Hmax = the padded reduction length, a multiple of 64.
+__device__ __forceinline__ float tc_logit_bound(const bf16* __restrict__ xr, int H, float wnorm2, int lane) {
+    float ss = 0.0f;
+    for (int c = lane; c < (H >> 3); c += 32) {
+        const uint4 v = ld_nc16(xr + (size_t)c * 8);
+        ss = dot8(v, v, ss);
+    }
+    ss = warp_sum(ss);
+    const float hpad = (float)(((H + 63) / 64) * 64);
+    const float xn = sqrtf(ss * (1.0f + 0x1p-8f));
+    const float wn = sqrtf(wnorm2);
+    return hpad * 0x1p-22f * xn * wn * (1.0f + 0x1p-8f);
+}
 
+// Exact re-evaluation of one candidate's logit (warp-collective), written back into the
+// logits buffer.  A re-evaluated logit that lies farther than the row's bound `eps` from
+// its tensor-core value (`screen`) means the bound's hardware model does not hold; that
+// sets MOE_DEVERR_ROUTER_BOUND (the routing of the call is then not guaranteed exact).
 struct RowRefine {
     const bf16* xr;
     const bf16* wr;
     int H, E, row, lane;
     float* logits_rw;
-    __device__ float operator()(int e) const {
+    float eps;
+    int* err;
+    __device__ float operator()(int e, float screen) const {
         const float v = warp_dot_exact(xr, wr + (size_t)e * H, H, lane);
-        if (logits_rw && lane == 0) logits_rw[(size_t)row * E + e] = v;
+        if (lane == 0) {
+            if (logits_rw) logits_rw[(size_t)row * E + e] = v;
+            if (!(fabsf(v - screen) <= eps)) set_dev_error(err, MOE_DEVERR_ROUTER_BOUND);
+        }
         return v;
     }
 };
@@ -32,6 +60,7 @@ __global__ void __launch_bounds__(32 * kTopkRowsPerBlock) topk_kernel(const void
                                                    int32_t* __restrict__ src_idx, float* __restrict__ w_copy,
                                                    int32_t* __restrict__ id_copy, const bf16* __restrict__ x,
                                                    const bf16* __restrict__ wr, int H, float* logits_rw,
+                                                   const float* __restrict__ wnorm2, int* err,
                                                    int* __restrict__ counts) {
     __shared__ float s_wbuf[kTopkRowsPerBlock][32];
     pdl_wait();
@@ -47,8 +76,10 @@ __global__ void __launch_bounds__(32 * kTopkRowsPerBlock) topk_kernel(const void
         int id;
         float w, lg;
         if (REFINE) {
-            const RowRefine rf{x + (size_t)row * H, wr, H, E, row, lane, logits_rw};
-            warp_route_row<V>(l, E, K, score, bias, renorm, lane, kTcLogitErr, rf, wbuf, id, w, lg);
+            const bf16* xr = x + (size_t)row * H;
+            const float eps = tc_logit_bound(xr, H, *wnorm2, lane);
+            const RowRefine rf{xr, wr, H, E, row, lane, logits_rw, eps, err};
+            warp_route_row<V>(l, E, K, score, bias, renorm, lane, eps, rf, wbuf, id, w, lg);
         } else {
             warp_route_row<V>(l, E, K, score, bias, renorm, lane, 0.0f, NoRefine{}, wbuf, id, w, lg);
         }
@@ -74,15 +105,20 @@ cudaError_t launch_topk(const void* logits, bool bf16_in, int M, int E, int K, i
     const bf16* wr = refine ? refine->wr : nullptr;
     const int H = refine ? refine->H : 0;
     float* lrw = refine ? refine->logits_rw : nullptr;
+    const float* wn2 = refine ? refine->wnorm2 : nullptr;
+    int* err = refine ? refine->err : nullptr;
 #define MOE_L(VV)                                                                                              \
     if (v == VV) {                                                                                             \
         if (refine)                                                                                            \
             return launch_k(topk_kernel<VV, false, true>, grid, block, 0, s, pdl, logits, M, E, K, score, bias, \
-                            renorm, topk_w, topk_ids, src_idx, w_copy, id_copy, x, wr, H, lrw, counts);        \
+                            renorm, topk_w, topk_ids, src_idx, w_copy, id_copy, x, wr, H, lrw, wn2, err,       \
+                            counts);                                                                           \
         return bf16_in ? launch_k(topk_kernel<VV, true, false>, grid, block, 0, s, pdl, logits, M, E, K, score, \
-                                  bias, renorm, topk_w, topk_ids, src_idx, w_copy, id_copy, x, wr, H, lrw, counts) \
+                                  bias, renorm, topk_w, topk_ids, src_idx, w_copy, id_copy, x, wr, H, lrw, wn2, \
+                                  err, counts)                                                                 \
                        : launch_k(topk_kernel<VV, false, false>, grid, block, 0, s, pdl, logits, M, E, K, score, \
-                                  bias, renorm, topk_w, topk_ids, src_idx, w_copy, id_copy, x, wr, H, lrw, counts); \
+                                  bias, renorm, topk_w, topk_ids, src_idx, w_copy, id_copy, x, wr, H, lrw, wn2, \
+                                  err, counts);                                                                \
     }
     MOE_L(1) MOE_L(2) MOE_L(4) MOE_L(8) MOE_L(16) MOE_L(32)
 #undef MOE_L
@@ -107,7 +143,9 @@ template <int V>
 __global__ void __launch_bounds__(32 * kTopkRowsPerBlock) topk_screen_kernel(const float* __restrict__ logits, int M,
                                                                               int E, int K, int score,
                                                                               const float* __restrict__ bias,
-                                                                              const CandList cl) {
+                                                                              const CandList cl,
+                                                                              const bf16* __restrict__ x, int H,
+                                                                              const float* __restrict__ wnorm2) {
     pdl_wait();
     const int lane = threadIdx.x & 31;
     const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -115,10 +153,12 @@ __global__ void __launch_bounds__(32 * kTopkRowsPerBlock) topk_screen_kernel(con
         const bool sig = score == MOE_SCORE_SIGMOID;
         float l[V], key[V];
         load_row_f32<V>(logits + (size_t)row * E, E, lane, l);
+        const float eps = tc_logit_bound(x + (size_t)row * H, H, *wnorm2, lane);
+        if (lane == 0) cl.row_eps[row] = eps;
         screening_keys<V>(l, key, E, sig, bias, lane);
         float kth, ua, ub;
         warp_select<V, false>(key, key, key, E, K, lane, kth, ua, ub);
-        const float lo = kth - screen_window(kth, sig, kTcLogitErr);
+        const float lo = kth - screen_window(kth, sig, eps);
         unsigned mc[V];
         int before[V], n = 0;
 #pragma unroll
@@ -165,7 +205,11 @@ __global__ void __launch_bounds__(256) refine_kernel(const bf16* __restrict__ x,
         const float v = warp_dot_exact(x + (size_t)row * H, wr + (size_t)e * H, H, lane);
         if (lane == 0) {
             cl.cand_val[it] = v;
-            if (logits_rw) logits_rw[(size_t)row * E + e] = v;
+            if (logits_rw) {  // the tensor-core value must lie within the row's bound
+                const float screen = logits_rw[(size_t)row * E + e];
+                if (!(fabsf(v - screen) <= cl.row_eps[row])) set_dev_error(err, MOE_DEVERR_ROUTER_BOUND);
+                logits_rw[(size_t)row * E + e] = v;
+            }
         }
     }
     pdl_trigger();
@@ -176,7 +220,7 @@ __global__ void __launch_bounds__(32 * kTopkRowsPerBlock) topk_final_kernel(
     const float* __restrict__ logits, int M, int E, int K, int score, const float* __restrict__ bias, int renorm,
     const CandList cl, float* __restrict__ topk_w, int32_t* __restrict__ topk_ids, float* __restrict__ w_copy,
     int32_t* __restrict__ id_copy, int* __restrict__ counts, const bf16* __restrict__ x,
-    const bf16* __restrict__ wr, int H, float* logits_rw) {
+    const bf16* __restrict__ wr, int H, float* logits_rw, int* err) {
     __shared__ float s_wbuf[kTopkRowsPerBlock][32];
     pdl_wait();
     const int lane = threadIdx.x & 31;
@@ -231,9 +275,10 @@ __global__ void __launch_bounds__(32 * kTopkRowsPerBlock) topk_final_kernel(
     } else {  // many candidates: route the row in one warp with per-candidate refinement
         float l[V];
         load_row_f32<V>(logits + (size_t)row * E, E, lane, l);
-        const RowRefine rf{x + (size_t)row * H, wr, H, E, row, lane, logits_rw};
+        const float eps = cl.row_eps[row];
+        const RowRefine rf{x + (size_t)row * H, wr, H, E, row, lane, logits_rw, eps, err};
         float lg;
-        warp_route_row<V>(l, E, K, score, bias, renorm, lane, kTcLogitErr, rf, s_wbuf[threadIdx.x >> 5], id, w, lg);
+        warp_route_row<V>(l, E, K, score, bias, renorm, lane, eps, rf, s_wbuf[threadIdx.x >> 5], id, w, lg);
     }
     if (lane < K) {
         const size_t o = (size_t)row * K + lane;
@@ -253,8 +298,10 @@ cudaError_t launch_topk_split(const float* logits, int M, int E, int K, int scor
     dim3 grid(cdiv(M, kTopkRowsPerBlock)), block(32 * kTopkRowsPerBlock);
     const int v = topk_v(E);
     cudaError_t st = cudaErrorInvalidValue;
-#define MOE_S(VV) \
-    if (v == VV) st = launch_k(topk_screen_kernel<VV>, grid, block, 0, s, pdl, logits, M, E, K, score, bias, cl);
+#define MOE_S(VV)                                                                                           \
+    if (v == VV)                                                                                            \
+        st = launch_k(topk_screen_kernel<VV>, grid, block, 0, s, pdl, logits, M, E, K, score, bias, cl, ra.x, \
+                      ra.H, ra.wnorm2);
     MOE_S(1) MOE_S(2) MOE_S(4) MOE_S(8) MOE_S(16) MOE_S(32)
 #undef MOE_S
     if (st != cudaSuccess) return st;
@@ -267,7 +314,7 @@ cudaError_t launch_topk_split(const float* logits, int M, int E, int K, int scor
 #define MOE_F(VV)                                                                                             \
     if (v == VV)                                                                                              \
         st = launch_k(topk_final_kernel<VV>, grid, block, 0, s, pdl, logits, M, E, K, score, bias, renorm, cl, \
-                      topk_w, topk_ids, w_copy, id_copy, counts, ra.x, ra.wr, ra.H, ra.logits_rw);
+                      topk_w, topk_ids, w_copy, id_copy, counts, ra.x, ra.wr, ra.H, ra.logits_rw, err);
     MOE_F(1) MOE_F(2) MOE_F(4) MOE_F(8) MOE_F(16) MOE_F(32)
 #undef MOE_F
     return st;

@@ -169,7 +169,7 @@ __device__ __forceinline__ void screening_keys(const float (&l)[V], float (&key)
 }
 
 struct NoRefine {
-    __device__ float operator()(int) const { return 0.0f; }
+    __device__ float operator()(int, float) const { return 0.0f; }
 };
 
 // Screening + exact values for the candidates.  On entry key[] holds the screening keys;
@@ -203,7 +203,8 @@ __device__ __forceinline__ void route_refine_keys(float (&l)[V], float (&key)[V]
             while (m) {
                 const int src = __ffs(m) - 1;
                 m &= m - 1;
-                const float ex = refine(src + 32 * c);
+                const float screen = __shfl_sync(0xffffffffu, l[c], src);
+                const float ex = refine(src + 32 * c, screen);
                 if (lane == src) l[c] = ex;
             }
         }
@@ -281,8 +282,8 @@ __device__ __forceinline__ void finish_route_row(const float (&l)[V], int E, int
 
 // One routing row.  l[c]: logit of expert lane + 32c (any value for e >= E), exact when
 // eps_l == 0, otherwise within eps_l (absolute) of the exact FP32 value and re-evaluated
-// with refine(e) (warp-collective) where it matters; refined logits are written back
-// into l.  wbuf: 32 floats of shared memory owned by this warp.  Outputs on lanes k < K:
+// with refine(e, screening value) (warp-collective) where it matters; refined logits are
+// written back into l.  wbuf: 32 floats of shared memory owned by this warp.  Outputs on lanes k < K:
 // slot k's expert id, weight and exact logit.
 template <int V, class Refine>
 __device__ __forceinline__ void warp_route_row(float (&l)[V], int E, int K, int score, const float* bias, int renorm,

@@ -90,20 +90,45 @@ def bits_to_bf16(a: np.ndarray) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
 
 
+X_MODES = ("normal", "scale32", "scale256", "outliers")
+
+
+def _shape_x(x: torch.Tensor, mode: str, seed: int) -> torch.Tensor:
+    """Activation scale of the router stress cases.  ``scale32`` / ``scale256``
+    multiply x by a power of two (exact in BF16).  ``outliers`` mimics hidden states with
+    outlier channels: 16 seeded columns are multiplied by 64 and 1 % of the tokens
+    (at least one) by 16, all powers of two."""
+    if mode == "normal":
+        return x
+    if mode in ("scale32", "scale256"):
+        return (x.float() * float(mode[5:])).to(torch.bfloat16)
+    if mode == "outliers":
+        T, H = x.shape
+        g = _gen(seed + 104729, "cpu")
+        cols = torch.randperm(H, generator=g)[:16].to(x.device)
+        rows = torch.randperm(T, generator=g)[:max(1, T // 100)].to(x.device)
+        y = x.float()
+        y[:, cols] *= 64.0
+        y[rows] *= 16.0
+        return y.to(torch.bfloat16)
+    raise ValueError(mode)
+
+
 def make_layer(shape: LayerShape, T: int, seed: int = 0, device: str = "cpu",
-               routing: str = "router", zipf_s: float = 1.2) -> dict:
+               routing: str = "router", zipf_s: float = 1.2, x_mode: str = "normal") -> dict:
     """Draw one layer's inputs.
 
     ``routing="router"``: logits come from the router weight (x . Wr^T on the path).
     ``routing="zipf"``: FP32 router logits are drawn directly as
     ``log p_e + Gumbel(0,1)`` with ``p_e ~ rank_e^-s`` over a seeded random ranking of
     the experts, so that per-token expert choice is Zipf-skewed (load imbalance).
+    ``x_mode``: activation scale (see ``_shape_x``); the other draws do not change.
     Returns torch tensors on ``device`` (bf16 / fp32).
     """
     H, I, E = shape.H, shape.I, shape.E
     g = _gen(seed, device)
     d = {}
-    d["x"] = _normal_bf16((T, H), 1.0, g, device)
+    d["x"] = _shape_x(_normal_bf16((T, H), 1.0, g, device), x_mode, seed)
     d["router_w"] = _normal_bf16((E, H), 1.0 / H, g, device)
     if shape.bias_var is not None:
         d["bias"] = torch.randn((E,), generator=g, device=device) * math.sqrt(shape.bias_var)

@@ -20,12 +20,14 @@ SCORE = {"softmax": 0, "sigmoid": 1}
 ACT = {"swiglu": 0, "relu2": 1}
 PATH = {"auto": 0, "small": 1, "large": 2}
 DT_BF16, DT_FP32 = 0, 1
-DEVERR_BAD_EXPERT_ID, DEVERR_WAIT_TIMEOUT = 0x1, 0x2
+DEVERR_BAD_EXPERT_ID, DEVERR_WAIT_TIMEOUT, DEVERR_BAD_INDEX, DEVERR_ROUTER_BOUND = 0x1, 0x2, 0x4, 0x8
+WS_TOPK_IDS, WS_TOPK_W, WS_OFFSETS, WS_PERM = range(4)
 
 # Every symbol include/moe.h declares.
 EXPORTS = ("moe_router_topk", "moe_permute_workspace_size", "moe_permute", "moe_workspace_size",
-           "moe_select_path", "moe_fused_forward", "moe_fused_forward_launches", "moe_fused_forward_timed",
-           "moe_fused_forward_noalloc", "moe_get_error", "moe_status_string")
+           "moe_select_path", "moe_fused_forward", "moe_fused_forward_launches", "moe_token_tiles",
+           "moe_workspace_region", "moe_fused_forward_timed", "moe_fused_forward_noalloc",
+           "moe_noalloc_get_error", "moe_get_error", "moe_status_string")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with `python -m mixture_experts_layer_35_b200.build`")
@@ -53,6 +55,10 @@ _lib.moe_select_path.argtypes = [ctypes.POINTER(LayerDesc)]
 _lib.moe_select_path.restype = _ci
 _lib.moe_fused_forward_launches.argtypes = [ctypes.POINTER(LayerDesc)]
 _lib.moe_fused_forward_launches.restype = _ci
+_lib.moe_token_tiles.argtypes = [ctypes.POINTER(LayerDesc), ctypes.POINTER(_ci), ctypes.POINTER(_ci)]
+_lib.moe_token_tiles.restype = _ci
+_lib.moe_workspace_region.argtypes = [ctypes.POINTER(LayerDesc), _ci, ctypes.POINTER(_sz), ctypes.POINTER(_sz)]
+_lib.moe_workspace_region.restype = _ci
 _lib.moe_fused_forward.argtypes = [ctypes.POINTER(LayerDesc), _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
 _lib.moe_fused_forward.restype = _ci
 _lib.moe_fused_forward_timed.argtypes = [ctypes.POINTER(LayerDesc), _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp,
@@ -61,6 +67,8 @@ _lib.moe_fused_forward_timed.restype = _ci
 _lib.moe_fused_forward_noalloc.argtypes = [ctypes.POINTER(LayerDesc), _vp, _vp, _vp, _vp, _vp, _vp]
 _lib.moe_fused_forward_noalloc.restype = _ci
 NOALLOC_SCRATCH_BYTES = 4 << 20  # MOE_NOALLOC_SCRATCH_BYTES
+_lib.moe_noalloc_get_error.argtypes = [ctypes.POINTER(_ci), _vp]
+_lib.moe_noalloc_get_error.restype = _ci
 _lib.moe_get_error.argtypes = [_vp, ctypes.POINTER(_ci), _vp]
 _lib.moe_get_error.restype = _ci
 _lib.moe_status_string.argtypes = [_ci]
@@ -142,6 +150,15 @@ def get_error(ws: torch.Tensor, stream=None) -> int:
     return code.value
 
 
+def noalloc_get_error(stream=None) -> int:
+    """Read and clear the error word of the static scratch (moe_noalloc_get_error)."""
+    code = _ci(0)
+    st = _lib.moe_noalloc_get_error(ctypes.byref(code), _stream(stream))
+    if st not in (MOE_OK, MOE_ERR_DEVICE):
+        raise MoEError(st, "moe_noalloc_get_error")
+    return code.value
+
+
 def make_desc(T: int, H: int, I: int, E: int, top_k: int, act: str, score: str, renorm: bool, I_shared: int,
               path: str = "auto", router_w=None, router_logits=None, bias=None, w13=None, w2=None, ws13=None,
               ws2=None) -> LayerDesc:
@@ -164,6 +181,21 @@ def select_path(desc: LayerDesc) -> str:
 
 def launches(desc: LayerDesc) -> int:
     return _lib.moe_fused_forward_launches(ctypes.byref(desc))
+
+
+def token_tiles(desc: LayerDesc):
+    """(FC1, FC2) token rows per grouped-GEMM tile for this description."""
+    a, b = _ci(0), _ci(0)
+    _check(_lib.moe_token_tiles(ctypes.byref(desc), ctypes.byref(a), ctypes.byref(b)), "moe_token_tiles")
+    return a.value, b.value
+
+
+def workspace_view(desc: LayerDesc, ws: torch.Tensor, region: int, dtype=torch.int32) -> torch.Tensor:
+    """A view of one intermediate kept in the workspace (moe_workspace_region)."""
+    off, nb = _sz(0), _sz(0)
+    _check(_lib.moe_workspace_region(ctypes.byref(desc), region, ctypes.byref(off), ctypes.byref(nb)),
+           "moe_workspace_region")
+    return ws[off.value:off.value + nb.value].view(dtype)
 
 
 def fused_forward_raw(desc: LayerDesc, x: torch.Tensor, out: torch.Tensor, ws: torch.Tensor,

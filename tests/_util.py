@@ -13,9 +13,9 @@ OUT_MEAN_REL = 1e-3
 W_REL = 1e-6
 
 
-def device_layer(shape, T, seed=0, routing="router", device="cuda"):
+def device_layer(shape, T, seed=0, routing="router", device="cuda", x_mode="normal"):
     """Inputs drawn on the device (fast for full-size weights)."""
-    return inp_mod.make_layer(shape, T, seed=seed, device=device, routing=routing)
+    return inp_mod.make_layer(shape, T, seed=seed, device=device, routing=routing, x_mode=x_mode)
 
 
 def host_copy(d):

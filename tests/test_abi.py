@@ -138,3 +138,35 @@ def test_router_topk_and_permute_validation():
     assert L.moe_permute(FAKE, 8, 4, 16, FAKE, FAKE, None, FAKE * 8, need - 1, None) == moe.MOE_ERR_WORKSPACE
     assert L.moe_permute(FAKE, 8, 40, 16, FAKE, FAKE, None, FAKE * 8, need, None) == moe.MOE_ERR_UNSUPPORTED
     assert L.moe_permute(FAKE, -1, 4, 16, FAKE, FAKE, None, FAKE * 8, need, None) == moe.MOE_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("act,T,K,E,tiles", [
+    ("swiglu", 20, 2, 8, (32, 32)), ("swiglu", 150, 2, 8, (64, 128)), ("swiglu", 300, 2, 8, (128, 192)),
+    ("swiglu", 800, 2, 8, (128, 256)), ("relu2", 150, 2, 8, (64, 128)), ("relu2", 300, 2, 8, (128, 192)),
+    ("relu2", 800, 2, 8, (256, 256)), ("swiglu", 4096, 8, 256, (128, 192)), ("swiglu", 8192, 8, 256, (128, 256)),
+    ("relu2", 4096, 6, 128, (256, 256))])
+def test_token_tile_widths(act, T, K, E, tiles):
+    """Token rows per grouped-GEMM tile follow the average rows per expert T*K/E."""
+    d = _desc(T=T, top_k=K, E=E, act=act, I_shared=0)
+    assert moe.token_tiles(d) == tiles
+
+
+def test_workspace_regions_lie_inside_the_workspace():
+    d = _desc(T=300, top_k=4, E=16)
+    need = moe.workspace_size(d)
+    seen = []
+    for region, nbytes in ((moe.WS_TOPK_IDS, 300 * 4 * 4), (moe.WS_TOPK_W, 300 * 4 * 4), (moe.WS_OFFSETS, 17 * 4),
+                           (moe.WS_PERM, 300 * 4 * 4)):
+        off, nb = ctypes.c_size_t(0), ctypes.c_size_t(0)
+        assert moe.lib().moe_workspace_region(ctypes.byref(d), region, ctypes.byref(off), ctypes.byref(nb)) == 0
+        assert nb.value == nbytes and off.value % 256 == 0 and off.value + nb.value <= need
+        seen.append((off.value, off.value + nb.value))
+    seen.sort()
+    assert all(a[1] <= b[0] for a, b in zip(seen, seen[1:])), "regions overlap"
+    off, nb = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    assert moe.lib().moe_workspace_region(ctypes.byref(d), 9, ctypes.byref(off), ctypes.byref(nb)) == \
+        moe.MOE_ERR_INVALID_ARG
+
+
+def test_noalloc_get_error_validates_before_any_cuda_call():
+    assert moe.lib().moe_noalloc_get_error(None, None) == moe.MOE_ERR_INVALID_ARG

@@ -298,3 +298,19 @@ def test_forward_rows_subset_and_given_logits():
     w4, i4, _ = oracle.topk(lg, K, "sigmoid", inp["bias"])
     np.testing.assert_array_equal(i4, ids)
     np.testing.assert_array_equal(w4, w)
+
+
+def test_sharded_oracle_equals_one_process():
+    from mixture_experts_layer_35_b200 import inputs as gen
+    """oracle.parallel runs the same C oracle on token ranges in spawned processes; the
+    concatenation must equal the single-process result bit for bit."""
+    from oracle import parallel as opar
+    shape = gen.TINY
+    h = gen.to_numpy_inputs(gen.make_layer(shape, 37, seed=4))
+    one = oracle.forward(shape, h)
+    rows = np.arange(37, dtype=np.int32)[::-1].copy()
+    many = opar.forward_parallel(shape, h, rows, procs=3)
+    ref = oracle.forward(shape, h, rows)
+    for a, b in zip(many, ref):
+        np.testing.assert_array_equal(a, b)
+    np.testing.assert_array_equal(many[0][::-1], one[0])
