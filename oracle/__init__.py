@@ -37,7 +37,8 @@ def build(force: bool = False) -> str:
 class _Layer(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in ("T", "H", "I", "E", "K", "act", "score", "renorm", "I_shared")] + [
         ("router_w", ctypes.c_void_p), ("router_logits", ctypes.c_void_p), ("bias", ctypes.c_void_p),
-        ("w13", ctypes.c_void_p), ("w2", ctypes.c_void_p), ("ws13", ctypes.c_void_p), ("ws2", ctypes.c_void_p)]
+        ("w13", ctypes.c_void_p), ("w2", ctypes.c_void_p), ("ws13", ctypes.c_void_p), ("ws2", ctypes.c_void_p),
+        ("routed_scale", ctypes.c_double), ("shared_gate", ctypes.c_void_p), ("shared_out", ctypes.c_void_p)]
 
 
 _lib = None
@@ -122,10 +123,13 @@ def permute(ids: np.ndarray, E: int):
     return offsets, perm, inv
 
 
-def forward(shape, inp: dict, rows=None):
+def forward(shape, inp: dict, rows=None, routed_scale: float = 1.0):
     """Layer forward for token ``rows`` (default: all).  ``inp`` is a numpy input dict
-    (see ``mixture_experts_layer_35_b200.inputs.to_numpy_inputs``).  Returns
-    ``(out_bits[r,H], logits[r,E], w[r,K], ids[r,K])``."""
+    (see ``mixture_experts_layer_35_b200.inputs.to_numpy_inputs``); optional entries
+    ``shared_gate`` ([H] BF16 bits: the shared expert's sigmoid gate row) and
+    ``shared_out`` ([T,H] BF16 bits: a caller-computed shared output, used when there is
+    no internal shared expert).  ``routed_scale`` multiplies the routed sum before its
+    BF16 rounding.  Returns ``(out_bits[r,H], logits[r,E], w[r,K], ids[r,K])``."""
     x = _c(inp["x"], np.uint16)
     T, H = x.shape
     if rows is None:
@@ -137,10 +141,12 @@ def forward(shape, inp: dict, rows=None):
     L.act, L.score, L.renorm = ACT[shape.act], SCORE[shape.score], int(shape.renorm)
     L.I_shared = shape.I_shared if inp.get("ws13") is not None else 0
     for name, dt in (("router_w", np.uint16), ("router_logits", np.float32), ("bias", np.float32),
-                     ("w13", np.uint16), ("w2", np.uint16), ("ws13", np.uint16), ("ws2", np.uint16)):
+                     ("w13", np.uint16), ("w2", np.uint16), ("ws13", np.uint16), ("ws2", np.uint16),
+                     ("shared_gate", np.uint16), ("shared_out", np.uint16)):
         a = _c(inp.get(name), dt)
         keep[name] = a
         setattr(L, name, _p(a))
+    L.routed_scale = float(routed_scale)
     n = len(rows)
     out = np.empty((n, H), np.uint16)
     lg = np.empty((n, shape.E), np.float32)

@@ -13,6 +13,13 @@
  *   - the expert activation h is rounded to BF16 (it feeds a BF16 GEMM).
  *   - the routed sum is rounded to BF16, the shared-expert output is rounded to
  *     BF16, and their sum is rounded to BF16.
+ *   - optional routed scale: the routed sum is multiplied by it before its BF16
+ *     rounding.
+ *   - optional shared-expert gate: an FP32 logit (one rounding of the FP64 dot product
+ *     of x with the gate row) through the same FP32 sigmoid as the router; the shared
+ *     expert's FP64 output is multiplied by it before its BF16 rounding.
+ *   - optional caller-computed shared output (BF16): added in place of the shared
+ *     expert's own output, in the same order.
  *
  * Sources (page title, section):
  *   [P4] "Laguna exact M=8 BF16-input router top-k preregistration",
@@ -22,6 +29,13 @@
  *   [P5] FlashInfer PR #4646 "add cuTile fused MoE backend for BF16 and NVFP4 Unified
  *        MoE", description (SwiGLU gated / ReLU2 ungated) and walkthrough (routing
  *        permutation, grouped BF16 GEMM, weighted output combination).
+ *   [P3] vLLM PR #64636 "SM80 skinny GEMM plans", cold-L2 table: the shared-expert gate,
+ *        a (1, H) linear of the decode step.
+ * The routed scale follows [P4] "Question and arithmetic contract" (the router's own
+ * scale is 1.0; the configured routed scale is applied later to the routed output).  The
+ * caller-computed shared output, optionally aliased by the layer output, follows [P2]
+ * (the fused gather takes the completed shared-expert output; separate-output and
+ * shared-output-alias forms).
  */
 #include <math.h>
 #include <stdint.h>
@@ -224,13 +238,17 @@ typedef struct {
     const uint16_t* w2;          /* [E, H, I] */
     const uint16_t* ws13;        /* [2I_s or I_s, H] or NULL */
     const uint16_t* ws2;         /* [H, I_s] or NULL */
+    double routed_scale;         /* multiplies the routed sum before its BF16 rounding */
+    const uint16_t* shared_gate; /* [H] gate row of the shared expert, or NULL */
+    const uint16_t* shared_out;  /* [T,H] caller-computed shared output (BF16), or NULL */
 } oracle_layer;
 
 /* Forward for a subset of tokens rows[0..nrows) of a T-token batch (tokens are
  * independent, so a subset is exact).  x is the full [T,H] input.  Outputs, per listed
  * row r: out[r,H] BF16 bits; optional logits[r,E], w[r,K], ids[r,K].
  * Combine order [P2]: routed FP32 (here FP64) accumulation over the slots in slot
- * order -> BF16 -> add the BF16 shared-expert output -> BF16. */
+ * order -> (times the routed scale) -> BF16 -> add the BF16 shared-expert output (gated,
+ * or the caller's) -> BF16. */
 int oracle_forward_rows(const oracle_layer* L, const uint16_t* x, const int32_t* rows, int nrows,
                         uint16_t* out, float* logits_out, float* w_out, int32_t* ids_out) {
     const int H = L->H, I = L->I, E = L->E, K = L->K, T = L->T;
@@ -265,12 +283,20 @@ int oracle_forward_rows(const oracle_layer* L, const uint16_t* x, const int32_t*
             for (int c = 0; c < H; ++c) acc[c] += (double)w[k] * y[c];
         }
         for (int c = 0; c < H; ++c) {
-            double routed = bf16_round(acc[c]);
+            double routed = bf16_round(L->routed_scale * acc[c]);
             acc[c] = routed;
         }
         if (Is > 0) {
             expert_ffn(L->ws13, L->ws2, L->act, H, Is, xd, h, y);
-            for (int c = 0; c < H; ++c) acc[c] = acc[c] + bf16_round(y[c]);
+            double gate = 1.0;
+            if (L->shared_gate) {
+                float lg;
+                oracle_router_logits(x + (size_t)t * H, L->shared_gate, 1, H, 1, &lg);
+                gate = (double)oracle_sigmoid_f32(lg);
+            }
+            for (int c = 0; c < H; ++c) acc[c] = acc[c] + bf16_round(gate * y[c]);
+        } else if (L->shared_out) {
+            for (int c = 0; c < H; ++c) acc[c] = acc[c] + oracle_bf16_to_double(L->shared_out[(size_t)t * H + c]);
         }
         for (int c = 0; c < H; ++c) out[(size_t)r * H + c] = oracle_double_to_bf16(acc[c]);
         if (logits_out) memcpy(logits_out + (size_t)r * E, l, sizeof(float) * (size_t)E);

@@ -314,3 +314,107 @@ def test_sharded_oracle_equals_one_process():
     for a, b in zip(many, ref):
         np.testing.assert_array_equal(a, b)
     np.testing.assert_array_equal(many[0][::-1], one[0])
+
+
+# ---------------------------------------------------------------- routed scale, shared gate, shared output
+
+def _small_layer_inputs(seed, H=32, I=16, E=6, K=2, shared=True):
+    g = torch.Generator().manual_seed(seed)
+    inp = {"x": _rand_bits((5, H), 1.0, g), "router_w": _rand_bits((E, H), 0.3, g),
+           "bias": (torch.randn(E, generator=g) * 0.3).numpy(), "router_logits": None,
+           "w13": _rand_bits((E, 2 * I, H), H ** -0.5, g), "w2": _rand_bits((E, H, I), I ** -0.5, g),
+           "ws13": _rand_bits((2 * I, H), H ** -0.5, g) if shared else None,
+           "ws2": _rand_bits((H, I), I ** -0.5, g) if shared else None}
+    return LayerShape("extras", H, I, E, K, "swiglu", "sigmoid", True, 0.09, I if shared else 0), inp
+
+
+@pytest.mark.parametrize("act", ["swiglu", "relu2"])
+def test_routed_scale_on_a_dense_mlp(act):
+    """One expert, K = 1: the routed output is bf16(scale * dense MLP(x)), the dense MLP
+    taken from a torch float64 composition ("Laguna ...", "Question and arithmetic
+    contract": the configured routed scale multiplies the routed output)."""
+    H, I, T, scale = 40, 24, 6, 2.5
+    shape = LayerShape("dense", H, I, 1, 1, act, "softmax", True, None, 0)
+    g = torch.Generator().manual_seed(12)
+    rows1 = 2 * I if act == "swiglu" else I
+    inp = {"x": _rand_bits((T, H), 1.0, g), "router_w": _rand_bits((1, H), 0.2, g), "bias": None,
+           "router_logits": None, "w13": _rand_bits((1, rows1, H), H ** -0.5, g),
+           "w2": _rand_bits((1, H, I), I ** -0.5, g), "ws13": None, "ws2": None}
+    out, *_ = oracle.forward(shape, inp, routed_scale=scale)
+    ref = scale * _dense_mlp_ref(torch.from_numpy(oracle.bits_to_f64(inp["x"])),
+                                 torch.from_numpy(oracle.bits_to_f64(inp["w13"][0])),
+                                 torch.from_numpy(oracle.bits_to_f64(inp["w2"][0])), act, I).numpy()
+    got = oracle.bits_to_f64(out)
+    assert np.abs(got - ref).max() <= 4e-3 * np.abs(ref).max()
+    assert not np.array_equal(out, oracle.forward(shape, inp)[0])
+
+
+def test_routed_scale_two_is_w2_doubled():
+    """A routed scale of 2 equals doubling every routed W2 (exact in BF16), bit for bit,
+    with the shared expert unchanged."""
+    shape, inp = _small_layer_inputs(13)
+    w2x2 = bf16_bits(torch.from_numpy(oracle.bits_to_f64(inp["w2"]) * 2).to(torch.bfloat16))
+    a, *_ = oracle.forward(shape, inp, routed_scale=2.0)
+    b, *_ = oracle.forward(shape, dict(inp, w2=w2x2))
+    np.testing.assert_array_equal(a, b)
+
+
+def test_shared_gate_special_values():
+    """A zero gate row gives sigmoid(0) = 1/2, the same bits as halving the shared W2
+    (exact); a gate logit far above 0 gives sigmoid = 1.0 in FP32, the ungated bits."""
+    shape, inp = _small_layer_inputs(14)
+    H = shape.H
+    zero = np.zeros(H, np.uint16)
+    half = bf16_bits(torch.from_numpy(oracle.bits_to_f64(inp["ws2"]) / 2).to(torch.bfloat16))
+    a, *_ = oracle.forward(shape, dict(inp, shared_gate=zero))
+    b, *_ = oracle.forward(shape, dict(inp, ws2=half))
+    np.testing.assert_array_equal(a, b)
+    # gate row = 2^7 * sign(x) on every column of every token: logit >= 128 * min |x| sum
+    x = oracle.bits_to_f64(inp["x"])
+    assert (np.abs(x).sum(1) * 128 > 120).all()
+    big = np.full(H, 0x4300, np.uint16)  # 128.0
+    xs = np.abs(x)
+    sign_x = bf16_bits(torch.from_numpy(np.abs(x) / np.where(xs > 0, xs, 1.0)).to(torch.bfloat16))
+    inp_pos = dict(inp, x=sign_x)  # every x entry +1 or 0: gate logit = 128 * (count of nonzero) >= 128
+    c, *_ = oracle.forward(shape, dict(inp_pos, shared_gate=big))
+    d, *_ = oracle.forward(shape, inp_pos)
+    np.testing.assert_array_equal(c, d)
+
+
+def test_shared_gate_against_torch_composition():
+    """The gated shared output is bf16(sigmoid(fp32(x . w_g)) * shared FFN(x)) added after
+    the routed rounding (torch float64 composition, the same tolerance as the layer)."""
+    shape, inp = _small_layer_inputs(15, E=4, K=4)
+    g = torch.Generator().manual_seed(16)
+    gate = _rand_bits((shape.H,), 0.4, g)
+    with_gate, *_ = oracle.forward(shape, dict(inp, shared_gate=gate))
+    no_shared = dict(inp, ws13=None, ws2=None)
+    routed, *_ = oracle.forward(LayerShape("r", shape.H, shape.I, shape.E, shape.K, "swiglu", "sigmoid", True, 0.09, 0),
+                                no_shared)
+    x = torch.from_numpy(oracle.bits_to_f64(inp["x"]))
+    lg = (x @ torch.from_numpy(oracle.bits_to_f64(gate))).float().double()
+    s = torch.sigmoid(lg).float().double()
+    y = _dense_mlp_ref(x, torch.from_numpy(oracle.bits_to_f64(inp["ws13"])),
+                       torch.from_numpy(oracle.bits_to_f64(inp["ws2"])), "swiglu", shape.I)
+    ys = (s[:, None] * y).float().to(torch.bfloat16).double()
+    ref = (torch.from_numpy(oracle.bits_to_f64(routed)) + ys).numpy()
+    got = oracle.bits_to_f64(with_gate)
+    assert np.abs(got - ref).max() <= 1e-2 * np.abs(ref).max()
+    assert np.abs(got - ref).mean() <= 1e-3 * np.abs(ref).max()
+
+
+@pytest.mark.parametrize("gated", [False, True])
+def test_caller_shared_output_equals_internal_shared_expert(gated):
+    """The shared output the layer would compute, handed in by the caller instead (the
+    "MTP1 isolated gather/shared-add closure" form), gives the same bits: the internal
+    shared output is read off a run whose routed W2 is zero (routed sum 0)."""
+    shape, inp = _small_layer_inputs(17)
+    if gated:
+        inp["shared_gate"] = _rand_bits((shape.H,), 0.4, torch.Generator().manual_seed(18))
+    zero_w2 = np.zeros_like(inp["w2"])
+    ys, *_ = oracle.forward(shape, dict(inp, w2=zero_w2))
+    full, *_ = oracle.forward(shape, inp, routed_scale=1.5)
+    ext_shape = LayerShape("ext", shape.H, shape.I, shape.E, shape.K, "swiglu", "sigmoid", True, 0.09, 0)
+    ext, *_ = oracle.forward(ext_shape, dict(inp, ws13=None, ws2=None, shared_gate=None, shared_out=ys),
+                             routed_scale=1.5)
+    np.testing.assert_array_equal(ext, full)
