@@ -136,6 +136,26 @@ typedef struct {
     const void* w2;              /* [E, H, I] BF16 */
     const void* ws13;            /* shared expert, [2I_s, H] or [I_s, H] BF16, or NULL */
     const void* ws2;             /* shared expert, [H, I_s] BF16, or NULL */
+    /* Optional parts of the layer; a zero-initialised field leaves the plain layer.
+     *  routed_scale   the routed FP32 sum is multiplied by it before its BF16 rounding
+     *                 (a routed scaling factor applied to the routed output after the
+     *                 router, as "Laguna exact M=8 BF16-input router top-k
+     *                 preregistration", "Question and arithmetic contract", describes);
+     *                 0 means 1.  Must be finite.
+     *  shared_gate_w  [H] BF16 gate row of the internal shared expert (needs I_shared > 0)
+     *                 or NULL: the shared output of token t is multiplied by
+     *                 g_t = sigmoid(x[t] . w) (an FP32 logit of the exact products, the
+     *                 router's correctly rounded FP32 sigmoid) before its BF16 rounding --
+     *                 the (1, H) shared-expert gate of vLLM PR #64636's decode table.
+     *  shared_out     [T, H] BF16 shared-expert output computed by the caller, or NULL;
+     *                 only with I_shared == 0.  It is added in place of an internal shared
+     *                 expert, in the same order (routed BF16, then the BF16 add).  `out`
+     *                 may be this very buffer (the in-place, shared-output-alias form of
+     *                 "MTP1 isolated gather/shared-add closure"); it must not overlap it
+     *                 otherwise. */
+    float routed_scale;
+    const void* shared_gate_w;
+    const void* shared_out;
 } moe_layer_desc;
 
 /* Bytes of workspace moe_fused_forward needs for this description (either path). */
@@ -145,7 +165,8 @@ size_t moe_workspace_size(const moe_layer_desc* d);
 int moe_select_path(const moe_layer_desc* d);
 
 /*   x            [T, H] BF16 in.
- *   out          [T, H] BF16 out; must not alias any input.
+ *   out          [T, H] BF16 out; must not overlap x or any weight, and may overlap
+ *                d->shared_out only by being exactly that buffer.
  *   topk_w_out   [T, K] FP32 out or NULL (routing weights, as moe_router_topk).
  *   topk_ids_out [T, K] int32 out or NULL.
  *   logits_out   [T, E] FP32 out or NULL (the router logits used; a copy of

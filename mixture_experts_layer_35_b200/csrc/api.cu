@@ -14,7 +14,7 @@ bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) 
 
 // Workspace carve-up of moe_fused_forward, 256-byte aligned regions after the header.
 struct WsLayout {
-    size_t logits, route, topk_w, topk_ids, offsets, tiles1, tiles2, counts, perm, cand, h, hs, acc, ys, total;
+    size_t logits, route, topk_w, topk_ids, offsets, tiles1, tiles2, counts, perm, cand, h, hs, acc, ys, gate, total;
 };
 // Candidate-list capacity per token of the three-kernel top-k (rows with more fall back).
 constexpr size_t kCandPerRow = 32;
@@ -47,6 +47,7 @@ WsLayout layout(const moe_layer_desc* d) {
     L.hs = take(T * Is * 2);
     L.acc = take(T * H * 4);
     L.ys = take(Is ? T * H * 2 : 0);
+    L.gate = take(d->shared_gate_w ? T * 4 : 0);
     L.total = o;
     return L;
 }
@@ -65,10 +66,21 @@ moe_status_t validate_desc(const moe_layer_desc* d) {
     if (!d->router_w && !d->router_logits) return MOE_ERR_INVALID_ARG;
     if (!d->w13 || !d->w2) return MOE_ERR_INVALID_ARG;
     if (d->I_shared > 0 && (!d->ws13 || !d->ws2)) return MOE_ERR_INVALID_ARG;
-    const void* ptrs[] = {d->router_w, d->router_logits, d->bias, d->w13, d->w2, d->ws13, d->ws2};
+    if (!(d->routed_scale == d->routed_scale) || d->routed_scale > 3.4e38f || d->routed_scale < -3.4e38f)
+        return MOE_ERR_INVALID_ARG;  // NaN or infinite
+    if (d->shared_gate_w && d->I_shared == 0) return MOE_ERR_INVALID_ARG;
+    if (d->shared_out && d->I_shared > 0) return MOE_ERR_INVALID_ARG;
+    const void* ptrs[] = {d->router_w, d->router_logits, d->bias, d->w13, d->w2, d->ws13, d->ws2,
+                          d->shared_gate_w, d->shared_out};
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return MOE_ERR_INVALID_ARG;
     return MOE_OK;
+}
+
+// Byte ranges [a, a + na) and [b, b + nb) overlap.
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + nb && y < x + na;
 }
 
 // Token-count rule of MOE_PATH_AUTO.  The streaming path reads each routed expert once
@@ -302,6 +314,10 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
     if ((topk_w_out && !aligned16(topk_w_out)) || (topk_ids_out && !aligned16(topk_ids_out)) ||
         (logits_out && !aligned16(logits_out)))
         return MOE_ERR_INVALID_ARG;
+    const size_t act_bytes = (size_t)d->T * d->H * 2;
+    if (overlaps(out_, act_bytes, x_, act_bytes)) return MOE_ERR_INVALID_ARG;
+    if (d->shared_out && out_ != d->shared_out && overlaps(out_, act_bytes, d->shared_out, act_bytes))
+        return MOE_ERR_INVALID_ARG;  // in place only as the very same buffer
     const WsLayout L = layout(d);
     if (!ws || !aligned256(ws) || ws_bytes < L.total) return MOE_ERR_WORKSPACE;
     const int path = resolve_path(d);
@@ -322,6 +338,8 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
     bf16* out = static_cast<bf16*>(out_);
     const int T = d->T, H = d->H, I = d->I, E = d->E, K = d->top_k, Is = d->I_shared;
     const int sms = num_sms();
+    const float rscale = d->routed_scale == 0.0f ? 1.0f : d->routed_scale;
+    const bf16* sh_out = static_cast<const bf16*>(d->shared_out);
 
     // 0. the many-token path's slot counters start at zero.  Cleared before the first
     // kernel, so that every kernel launched with programmatic overlap follows a kernel
@@ -354,8 +372,9 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
     if (path == MOE_PATH_SMALL) {
         RouteTable* rt = reinterpret_cast<RouteTable*>(w8 + L.route);
         if (!mark()) return MOE_ERR_CUDA;
+        const GateArgs ga = {x, static_cast<const bf16*>(d->shared_gate_w), H, rt->gate};
         MOE_CK(launch_route_small(logits, T, E, K, d->score, d->bias, d->renorm, rt, topk_w_out, topk_ids_out, s,
-                                  pdl && !timed));
+                                  pdl && !timed, ga));
         SmallArgs a;
         std::memset(&a, 0, sizeof(a));
         a.T = T;
@@ -376,6 +395,9 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
         a.h = reinterpret_cast<bf16*>(w8 + L.h);
         a.hs = reinterpret_cast<bf16*>(w8 + L.hs);
         a.out = out;
+        a.routed_scale = rscale;
+        a.has_gate = d->shared_gate_w != nullptr;
+        a.sh_out = sh_out;
         const std::function<bool()> mark_fn = mark;
         MOE_CK(launch_small(a, sms, s, true, timed ? &mark_fn : nullptr));
         if (!mark()) return MOE_ERR_CUDA;
@@ -395,6 +417,8 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
     bf16* hs = reinterpret_cast<bf16*>(w8 + L.hs);
     float* acc = reinterpret_cast<float*>(w8 + L.acc);
     bf16* ys = Is ? reinterpret_cast<bf16*>(w8 + L.ys) : nullptr;
+    float* gate = d->shared_gate_w ? reinterpret_cast<float*>(w8 + L.gate) : nullptr;
+    const GateArgs ga = {x, static_cast<const bf16*>(d->shared_gate_w), H, gate};
 
     const bool chain = !timed;  // programmatic overlap between consecutive kernels
     const bool swiglu = d->act == MOE_ACT_SWIGLU;
@@ -417,10 +441,10 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
         cl.cap = (int)(kCandPerRow * (size_t)T);
         const std::function<bool()> mark_fn = mark;
         MOE_CK(launch_topk_split(logits, T, E, K, d->score, d->bias, d->renorm, tw, tid, topk_w_out, topk_ids_out,
-                                 cl, ra, counts, err, sms, s, pdl && chain, timed ? &mark_fn : nullptr));
+                                 cl, ra, counts, err, sms, s, pdl && chain, timed ? &mark_fn : nullptr, ga));
     } else {
         MOE_CK(launch_topk(logits, false, T, E, K, d->score, d->bias, d->renorm, tw, tid, nullptr, topk_w_out,
-                           topk_ids_out, s, pdl && chain, dense_router ? &ra : nullptr, counts));
+                           topk_ids_out, s, pdl && chain, dense_router ? &ra : nullptr, counts, &ga));
     }
     // 3. permutation + tile tables
     PermuteArgs pa;
@@ -504,6 +528,7 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
     g2.tiles = tiles2;
     g2.acc = acc;
     g2.ys = ys;
+    g2.sgate = gate;
     g2.zero_ptr = nullptr;
     g2.zero_n = 0;
     if (!mark()) return MOE_ERR_CUDA;
@@ -511,7 +536,7 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
 
     // 6. finalize
     if (!mark()) return MOE_ERR_CUDA;
-    MOE_CK(launch_finalize(acc, ys, out, (size_t)T * H, sms, s, chain));
+    MOE_CK(launch_finalize(acc, Is ? ys : sh_out, out, (size_t)T * H, rscale, sms, s, chain));
     if (!mark()) return MOE_ERR_CUDA;
     return MOE_OK;
 }

@@ -376,12 +376,15 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
                         }
                     }
                 } else if (MODE == GM_FC2) {
-                    if (ti.shared) {
+                    if (ti.shared) {  // shared rows are the tokens in order; optional sigmoid gate
 #pragma unroll
                         for (int j = 0; j < 32; ++j) {
                             const int col = c0 + j;
-                            if (col < ti.n && fok)
-                                a.ys[(size_t)(ti.row0 + col) * a.feat_s + f] = __float2bfloat16_rn(__uint_as_float(v[j]));
+                            if (col < ti.n && fok) {
+                                float y = __uint_as_float(v[j]);
+                                if (a.sgate) y = __fmul_rn(a.sgate[ti.row0 + col], y);
+                                a.ys[(size_t)(ti.row0 + col) * a.feat_s + f] = __float2bfloat16_rn(y);
+                            }
                         }
                     } else {
                         // Column j of this chunk is token t_j with routing weight w_j; lane l
@@ -547,14 +550,20 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
 }
 
 // ---------------------------------------------------------------- finalize
-__global__ void __launch_bounds__(256) finalize_kernel(const float* __restrict__ acc, const bf16* __restrict__ ys,
-                                                       bf16* __restrict__ out, size_t n) {
+// `ys` may be the caller's shared output and `out` that same buffer: each thread reads
+// its 8 elements before writing them, so the in-place form is safe (no __restrict__).
+__global__ void __launch_bounds__(256) finalize_kernel(const float* __restrict__ acc, const bf16* ys, bf16* out,
+                                                       size_t n, float scale) {
     pdl_wait();
     const size_t stride = (size_t)gridDim.x * blockDim.x * 8;
     for (size_t i = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) * 8; i < n; i += stride) {
         const float4 a0 = *reinterpret_cast<const float4*>(acc + i);
         const float4 a1 = *reinterpret_cast<const float4*>(acc + i + 4);
         float r[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+        if (scale != 1.0f) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) r[j] = __fmul_rn(scale, r[j]);
+        }
         if (ys) {
             const uint4 y = *reinterpret_cast<const uint4*>(ys + i);
             const uint32_t yw[4] = {y.x, y.y, y.z, y.w};
@@ -628,12 +637,12 @@ cudaError_t launch_gemm(int mode, int bn, const GemmArgs& a, const GemmMaps& m, 
     return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_finalize(const float* acc, const bf16* ys, bf16* out, size_t n, int num_sms, cudaStream_t s,
-                            bool pdl) {
+cudaError_t launch_finalize(const float* acc, const bf16* ys, bf16* out, size_t n, float scale, int num_sms,
+                            cudaStream_t s, bool pdl) {
     const size_t groups = n / 8;
     int grid = (int)std::min<size_t>((groups + 255) / 256, (size_t)num_sms * 4);
     if (grid < 1) grid = 1;
-    return launch_k(finalize_kernel, dim3(grid), dim3(256), 0, s, pdl, acc, ys, out, n);
+    return launch_k(finalize_kernel, dim3(grid), dim3(256), 0, s, pdl, acc, ys, out, n, scale);
 }
 
 }  // namespace moe

@@ -36,10 +36,18 @@ struct RefineArgs {
     const float* wnorm2; // max over experts of |Wr[e]|_2^2 (upper bound), from the router GEMM
     int* err;            // device error word (MOE_DEVERR_ROUTER_BOUND)
 };
+// Shared-expert gate of each token, computed by the routing kernels (one exact dot
+// product per row): out[t] = sigmoid_f32(x[t] . w), w == null = no gate.
+struct GateArgs {
+    const bf16* x;  // [M, H]
+    const bf16* w;  // [H] or null
+    int H;
+    float* out;     // [M]
+};
 cudaError_t launch_topk(const void* logits, bool bf16_in, int M, int E, int K, int score, const float* bias,
                         int renorm, float* topk_w, int32_t* topk_ids, int32_t* src_idx, float* w_copy,
                         int32_t* id_copy, cudaStream_t s, bool pdl, const RefineArgs* refine = nullptr,
-                        int* counts = nullptr);
+                        int* counts = nullptr, const GateArgs* gate = nullptr);
 // Candidate list of the three-kernel top-k after the tensor-core router.
 struct CandList {
     int* count;       // [1] candidates appended so far (zero on entry)
@@ -55,7 +63,7 @@ struct CandList {
 cudaError_t launch_topk_split(const float* logits, int M, int E, int K, int score, const float* bias, int renorm,
                               float* topk_w, int32_t* topk_ids, float* w_copy, int32_t* id_copy, const CandList& cl,
                               const RefineArgs& ra, int* counts, int* err, int num_sms, cudaStream_t s, bool pdl,
-                              const std::function<bool()>* mark);
+                              const std::function<bool()>* mark, const GateArgs& gate);
 bool router_small_supported(int H);
 cudaError_t launch_router_small(const bf16* x, const bf16* wr, int T, int H, int E, float* logits,
                                 float* logits_copy, int* err, cudaStream_t s, bool pdl);
@@ -74,9 +82,11 @@ struct RouteTable {
     int utok[kSmallMaxSlots];
     int ids[kSmallMaxSlots];
     float w[kSmallMaxSlots];
+    float gate[kSmallMaxT];  // shared-expert gate of each token (when the layer has one)
 };
 cudaError_t launch_route_small(const float* logits, int T, int E, int K, int score, const float* bias, int renorm,
-                               RouteTable* rt, float* w_out, int32_t* id_out, cudaStream_t s, bool pdl);
+                               RouteTable* rt, float* w_out, int32_t* id_out, cudaStream_t s, bool pdl,
+                               const GateArgs& gate);
 struct SmallArgs {
     int T, H, I, E, K, act, score, renorm, Is;
     const RouteTable* rt;
@@ -87,7 +97,10 @@ struct SmallArgs {
     const bf16* ws2;
     bf16* h;           // [T*K, I], row = slot k*T + t
     bf16* hs;          // [T, Is]
-    bf16* out;         // [T, H]
+    bf16* out;         // [T, H] (may equal sh_out)
+    float routed_scale;  // multiplies the routed sum before its BF16 rounding
+    int has_gate;        // the shared output is multiplied by rt->gate[t]
+    const bf16* sh_out;  // [T, H] caller-computed shared output (Is == 0), or null
 };
 bool small_path_supported(int T, int H, int I, int Is);
 // `mark` (optional) records a timing event before each of the two streaming kernels;
@@ -151,6 +164,7 @@ struct GemmArgs {
     size_t zero_n;           //      (floats, multiple of 4)
     float* wnorm2;           // GM_DENSE: max over experts of |Wr[e]|_2^2 (upper bound), atomicMax;
                              //           zero on entry, or null
+    const float* sgate;      // FC2: shared-expert gate per token (ys = bf16(gate[t] * y)), or null
     int* err;
 };
 struct GemmMaps {
@@ -169,9 +183,10 @@ int gemm_token_tile(int mode, int T, int K, int E);
 constexpr int kFc2BoxRows = 32;
 cudaError_t launch_gemm(int mode, int bn, const GemmArgs& a, const GemmMaps& m, int grid, cudaStream_t s, bool pdl);
 
-// finalize: out = bf16(bf16(acc) + ys) or bf16(acc)
-cudaError_t launch_finalize(const float* acc, const bf16* ys, bf16* out, size_t n, int num_sms, cudaStream_t s,
-                            bool pdl);
+// finalize: out = bf16(bf16(scale * acc) + ys) or bf16(scale * acc); out may equal ys
+// (each element is read before it is written, by the same thread).
+cudaError_t launch_finalize(const float* acc, const bf16* ys, bf16* out, size_t n, float scale, int num_sms,
+                            cudaStream_t s, bool pdl);
 
 // Driver entry point for tensor-map encoding (resolved once through the runtime).
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,

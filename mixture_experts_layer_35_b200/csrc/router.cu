@@ -50,6 +50,13 @@ struct RowRefine {
     }
 };
 
+// Shared-expert gate of one token row (warp-collective): the exact logit x[row] . w
+// (FP64 sum of the exact products, rounded once) through the correctly rounded sigmoid.
+__device__ __forceinline__ void shared_gate_row(const GateArgs& g, int row, int lane) {
+    const float l = warp_dot_exact(g.x + (size_t)row * g.H, g.w, g.H, lane);
+    if (lane == 0) g.out[row] = sigmoid_f32_rn(l);
+}
+
 // ---------------------------------------------------------------- top-k, one warp per row
 static constexpr int kTopkRowsPerBlock = 4;  // small blocks: the SM fills up to its register limit
 
@@ -61,7 +68,7 @@ __global__ void __launch_bounds__(32 * kTopkRowsPerBlock) topk_kernel(const void
                                                    int32_t* __restrict__ id_copy, const bf16* __restrict__ x,
                                                    const bf16* __restrict__ wr, int H, float* logits_rw,
                                                    const float* __restrict__ wnorm2, int* err,
-                                                   int* __restrict__ counts) {
+                                                   int* __restrict__ counts, const GateArgs gate) {
     __shared__ float s_wbuf[kTopkRowsPerBlock][32];
     pdl_wait();
     const int lane = threadIdx.x & 31;
@@ -92,14 +99,17 @@ __global__ void __launch_bounds__(32 * kTopkRowsPerBlock) topk_kernel(const void
             if (id_copy) id_copy[o] = id;
             if (counts) atomicAdd(counts + id, 1);
         }
+        if (gate.w) shared_gate_row(gate, row, lane);
     }
     pdl_trigger();
 }
 
 cudaError_t launch_topk(const void* logits, bool bf16_in, int M, int E, int K, int score, const float* bias,
                         int renorm, float* topk_w, int32_t* topk_ids, int32_t* src_idx, float* w_copy,
-                        int32_t* id_copy, cudaStream_t s, bool pdl, const RefineArgs* refine, int* counts) {
+                        int32_t* id_copy, cudaStream_t s, bool pdl, const RefineArgs* refine, int* counts,
+                        const GateArgs* gate_in) {
     dim3 grid(cdiv(M, kTopkRowsPerBlock)), block(32 * kTopkRowsPerBlock);
+    const GateArgs gate = gate_in ? *gate_in : GateArgs{nullptr, nullptr, 0, nullptr};
     const int v = topk_v(E);
     const bf16* x = refine ? refine->x : nullptr;
     const bf16* wr = refine ? refine->wr : nullptr;
@@ -112,13 +122,13 @@ cudaError_t launch_topk(const void* logits, bool bf16_in, int M, int E, int K, i
         if (refine)                                                                                            \
             return launch_k(topk_kernel<VV, false, true>, grid, block, 0, s, pdl, logits, M, E, K, score, bias, \
                             renorm, topk_w, topk_ids, src_idx, w_copy, id_copy, x, wr, H, lrw, wn2, err,       \
-                            counts);                                                                           \
+                            counts, gate);                                                                     \
         return bf16_in ? launch_k(topk_kernel<VV, true, false>, grid, block, 0, s, pdl, logits, M, E, K, score, \
                                   bias, renorm, topk_w, topk_ids, src_idx, w_copy, id_copy, x, wr, H, lrw, wn2, \
-                                  err, counts)                                                                 \
+                                  err, counts, gate)                                                           \
                        : launch_k(topk_kernel<VV, false, false>, grid, block, 0, s, pdl, logits, M, E, K, score, \
                                   bias, renorm, topk_w, topk_ids, src_idx, w_copy, id_copy, x, wr, H, lrw, wn2, \
-                                  err, counts);                                                                \
+                                  err, counts, gate);                                                          \
     }
     MOE_L(1) MOE_L(2) MOE_L(4) MOE_L(8) MOE_L(16) MOE_L(32)
 #undef MOE_L
@@ -220,7 +230,7 @@ __global__ void __launch_bounds__(32 * kTopkRowsPerBlock) topk_final_kernel(
     const float* __restrict__ logits, int M, int E, int K, int score, const float* __restrict__ bias, int renorm,
     const CandList cl, float* __restrict__ topk_w, int32_t* __restrict__ topk_ids, float* __restrict__ w_copy,
     int32_t* __restrict__ id_copy, int* __restrict__ counts, const bf16* __restrict__ x,
-    const bf16* __restrict__ wr, int H, float* logits_rw, int* err) {
+    const bf16* __restrict__ wr, int H, float* logits_rw, int* err, const GateArgs gate) {
     __shared__ float s_wbuf[kTopkRowsPerBlock][32];
     pdl_wait();
     const int lane = threadIdx.x & 31;
@@ -288,13 +298,14 @@ __global__ void __launch_bounds__(32 * kTopkRowsPerBlock) topk_final_kernel(
         if (id_copy) id_copy[o] = id;
         if (counts) atomicAdd(counts + id, 1);
     }
+    if (gate.w) shared_gate_row(gate, row, lane);
     pdl_trigger();
 }
 
 cudaError_t launch_topk_split(const float* logits, int M, int E, int K, int score, const float* bias, int renorm,
                               float* topk_w, int32_t* topk_ids, float* w_copy, int32_t* id_copy, const CandList& cl,
                               const RefineArgs& ra, int* counts, int* err, int num_sms, cudaStream_t s, bool pdl,
-                              const std::function<bool()>* mark) {
+                              const std::function<bool()>* mark, const GateArgs& gate) {
     dim3 grid(cdiv(M, kTopkRowsPerBlock)), block(32 * kTopkRowsPerBlock);
     const int v = topk_v(E);
     cudaError_t st = cudaErrorInvalidValue;
@@ -314,7 +325,7 @@ cudaError_t launch_topk_split(const float* logits, int M, int E, int K, int scor
 #define MOE_F(VV)                                                                                             \
     if (v == VV)                                                                                              \
         st = launch_k(topk_final_kernel<VV>, grid, block, 0, s, pdl, logits, M, E, K, score, bias, renorm, cl, \
-                      topk_w, topk_ids, w_copy, id_copy, counts, ra.x, ra.wr, ra.H, ra.logits_rw, err);
+                      topk_w, topk_ids, w_copy, id_copy, counts, ra.x, ra.wr, ra.H, ra.logits_rw, err, gate);
     MOE_F(1) MOE_F(2) MOE_F(4) MOE_F(8) MOE_F(16) MOE_F(32)
 #undef MOE_F
     return st;
@@ -429,7 +440,8 @@ __global__ void __launch_bounds__(32 * kSmallMaxT) route_small_kernel(const floa
                                                                       int K, int score, const float* __restrict__ bias,
                                                                       int renorm, RouteTable* __restrict__ rt,
                                                                       float* __restrict__ w_out,
-                                                                      int32_t* __restrict__ id_out) {
+                                                                      int32_t* __restrict__ id_out,
+                                                                      const GateArgs gate) {
     __shared__ int s_ids[kSmallMaxSlots];
     __shared__ int s_uidx[MOE_MAX_EXPERTS];
     __shared__ int s_ulist[kSmallMaxSlots];
@@ -453,6 +465,7 @@ __global__ void __launch_bounds__(32 * kSmallMaxT) route_small_kernel(const floa
             if (w_out) w_out[(size_t)t * K + lane] = w;
             if (id_out) id_out[(size_t)t * K + lane] = id;
         }
+        if (gate.w) shared_gate_row(gate, t, lane);  // gate.out = rt->gate
     }
     __syncthreads();
     for (int i = tid; i < TK; i += blockDim.x) atomicAdd(&s_uidx[s_ids[i]], 1);  // slots per expert
@@ -517,12 +530,14 @@ __global__ void __launch_bounds__(32 * kSmallMaxT) route_small_kernel(const floa
 }
 
 cudaError_t launch_route_small(const float* logits, int T, int E, int K, int score, const float* bias, int renorm,
-                               RouteTable* rt, float* w_out, int32_t* id_out, cudaStream_t s, bool pdl) {
+                               RouteTable* rt, float* w_out, int32_t* id_out, cudaStream_t s, bool pdl,
+                               const GateArgs& gate) {
     const int v = topk_v(E);
     dim3 grid(1), block(32 * std::max(1, std::min(T, kSmallMaxT)));
-#define MOE_RT(VV) \
-    if (v == VV)   \
-        return launch_k(route_small_kernel<VV>, grid, block, 0, s, pdl, logits, T, E, K, score, bias, renorm, rt, w_out, id_out);
+#define MOE_RT(VV)                                                                                              \
+    if (v == VV)                                                                                                \
+        return launch_k(route_small_kernel<VV>, grid, block, 0, s, pdl, logits, T, E, K, score, bias, renorm, rt, \
+                        w_out, id_out, gate);
     MOE_RT(1) MOE_RT(2) MOE_RT(4) MOE_RT(8) MOE_RT(16) MOE_RT(32)
 #undef MOE_RT
     return cudaErrorInvalidValue;

@@ -13,8 +13,9 @@
 //              h[slot, i] = act(.) in BF16.  Before that, the consumers L2-prefetch the
 //              CTA's share of the routed W2 for the next kernel.
 //   fc2_small: each CTA owns a slice of output features f.  For every token it sums
-//              w[t,k] * (W2[e_k, f, :] . h[slot]) in FP32 over the slots, rounds to BF16,
-//              adds the BF16 shared-expert output and rounds again ("MTP1 isolated
+//              w[t,k] * (W2[e_k, f, :] . h[slot]) in FP32 over the slots, scales the sum by
+//              the routed scale, rounds to BF16, adds the BF16 shared-expert output (its
+//              own, optionally gated, or the caller's) and rounds again ("MTP1 isolated
 //              gather/shared-add closure": routed FP32 accumulation -> BF16 -> shared BF16
 //              add -> BF16), writing the layer output directly.
 #include <cstring>
@@ -216,6 +217,7 @@ template <int VI>
 __global__ void __launch_bounds__(kSmallThreads, 1) fc2_small(const SmallArgs a) {
     __shared__ int s_ids[kSmallMaxSlots];
     __shared__ float s_w[kSmallMaxSlots];
+    __shared__ float s_gate[kSmallMaxT];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
     const int T = a.T, K = a.K, H = a.H, I = a.I, Is = a.Is;
     const int f0 = (int)((long long)blockIdx.x * H / gridDim.x);
@@ -226,6 +228,8 @@ __global__ void __launch_bounds__(kSmallThreads, 1) fc2_small(const SmallArgs a)
         s_ids[i] = a.rt->ids[i];
         s_w[i] = a.rt->w[i];
     }
+    if (a.has_gate)
+        for (int i = tid; i < T; i += blockDim.x) s_gate[i] = a.rt->gate[i];
     __syncthreads();
     const int nchI = I >> 3, nchS = Is >> 3;
     constexpr int KB = VI <= 2 ? 4 : (VI <= 4 ? 2 : 1);  // slots whose rows are in flight together
@@ -268,11 +272,14 @@ __global__ void __launch_bounds__(kSmallThreads, 1) fc2_small(const SmallArgs a)
             for (int c = lane; c < nchS; c += 32)
                 part = dot8(ld_nc16(row + (size_t)c * 8), ld_nc16(hr + (size_t)c * 8), part);
             ys = warp_sum(part);
+            if (a.has_gate) ys = __fmul_rn(s_gate[t], ys);
         }
         if (lane == 0) {
-            const float r = bf_round(routed);
-            const float o = Is ? __fadd_rn(r, bf_round(ys)) : r;
-            a.out[(size_t)t * H + f] = __float2bfloat16_rn(o);
+            const float r = bf_round(__fmul_rn(a.routed_scale, routed));
+            float o = r;
+            if (Is) o = __fadd_rn(r, bf_round(ys));
+            else if (a.sh_out) o = __fadd_rn(r, __bfloat162float(a.sh_out[(size_t)t * H + f]));  // read, then
+            a.out[(size_t)t * H + f] = __float2bfloat16_rn(o);                                     // written in place
         }
     }
     pdl_trigger();

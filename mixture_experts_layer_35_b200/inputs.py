@@ -115,7 +115,8 @@ def _shape_x(x: torch.Tensor, mode: str, seed: int) -> torch.Tensor:
 
 
 def make_layer(shape: LayerShape, T: int, seed: int = 0, device: str = "cpu",
-               routing: str = "router", zipf_s: float = 1.2, x_mode: str = "normal") -> dict:
+               routing: str = "router", zipf_s: float = 1.2, x_mode: str = "normal",
+               shared_gate: bool = False, shared_out: bool = False) -> dict:
     """Draw one layer's inputs.
 
     ``routing="router"``: logits come from the router weight (x . Wr^T on the path).
@@ -123,6 +124,9 @@ def make_layer(shape: LayerShape, T: int, seed: int = 0, device: str = "cpu",
     ``log p_e + Gumbel(0,1)`` with ``p_e ~ rank_e^-s`` over a seeded random ranking of
     the experts, so that per-token expert choice is Zipf-skewed (load imbalance).
     ``x_mode``: activation scale (see ``_shape_x``); the other draws do not change.
+    ``shared_gate``: also a gate row [H] ~ N(0, 1/H) for the shared expert (``shared_gate``);
+    ``shared_out``: also a caller-side shared output [T, H] ~ N(0, 1/4) (``shared_out``).
+    Both come from their own generators, so the other draws do not change.
     Returns torch tensors on ``device`` (bf16 / fp32).
     """
     H, I, E = shape.H, shape.I, shape.E
@@ -157,6 +161,8 @@ def make_layer(shape: LayerShape, T: int, seed: int = 0, device: str = "cpu",
         d["router_logits"] = (logp[None, :] + gumbel).to(torch.float32)
     elif routing != "router":
         raise ValueError(routing)
+    d["shared_gate"] = _normal_bf16((H,), 1.0 / H, _gen(seed + 7717, device), device) if shared_gate else None
+    d["shared_out"] = _normal_bf16((T, H), 0.25, _gen(seed + 6007, device), device) if shared_out else None
     return d
 
 

@@ -40,7 +40,8 @@ class LayerDesc(ctypes.Structure):
     """Mirror of moe_layer_desc."""
     _fields_ = [(n, _ci) for n in ("T", "H", "I", "E", "top_k", "act", "score", "renorm", "I_shared", "path")] + [
         ("router_w", _vp), ("router_logits", _vp), ("bias", _vp), ("w13", _vp), ("w2", _vp),
-        ("ws13", _vp), ("ws2", _vp)]
+        ("ws13", _vp), ("ws2", _vp), ("routed_scale", ctypes.c_float), ("shared_gate_w", _vp),
+        ("shared_out", _vp)]
 
 
 _lib.moe_router_topk.argtypes = [_vp, _ci, _ci, _ci, _ci, _ci, _vp, _ci, _vp, _vp, _vp, _vp]
@@ -161,12 +162,13 @@ def noalloc_get_error(stream=None) -> int:
 
 def make_desc(T: int, H: int, I: int, E: int, top_k: int, act: str, score: str, renorm: bool, I_shared: int,
               path: str = "auto", router_w=None, router_logits=None, bias=None, w13=None, w2=None, ws13=None,
-              ws2=None) -> LayerDesc:
+              ws2=None, routed_scale: float = 0.0, shared_gate_w=None, shared_out=None) -> LayerDesc:
     d = LayerDesc()
     d.T, d.H, d.I, d.E, d.top_k = T, H, I, E, top_k
     d.act, d.score, d.renorm, d.I_shared, d.path = ACT[act], SCORE[score], int(renorm), I_shared, PATH[path]
     d.router_w, d.router_logits, d.bias = _ptr(router_w), _ptr(router_logits), _ptr(bias)
     d.w13, d.w2, d.ws13, d.ws2 = _ptr(w13), _ptr(w2), _ptr(ws13), _ptr(ws2)
+    d.routed_scale, d.shared_gate_w, d.shared_out = routed_scale, _ptr(shared_gate_w), _ptr(shared_out)
     return d
 
 
@@ -227,18 +229,23 @@ def fused_forward_noalloc(desc: LayerDesc, x: torch.Tensor, out: torch.Tensor,
 class MoELayer:
     """A layer whose weights live on the device; ``forward`` enqueues moe_fused_forward."""
 
-    def __init__(self, shape, weights: dict, path: str = "auto"):
+    def __init__(self, shape, weights: dict, path: str = "auto", routed_scale: float = 0.0):
+        """``weights``: router_w, bias, w13, w2, and optionally ws13 / ws2 (internal shared
+        expert) and shared_gate (its [H] gate row).  ``routed_scale``: 0 = none."""
         self.shape = shape
         self.w = weights
         self.path = path
+        self.routed_scale = routed_scale
         self._ws = None
 
-    def desc(self, T: int, router_logits: Optional[torch.Tensor] = None) -> LayerDesc:
+    def desc(self, T: int, router_logits: Optional[torch.Tensor] = None,
+             shared_out: Optional[torch.Tensor] = None) -> LayerDesc:
         s, w = self.shape, self.w
         Is = s.I_shared if w.get("ws13") is not None else 0
         return make_desc(T, s.H, s.I, s.E, s.K, s.act, s.score, s.renorm, Is, self.path,
                          router_w=w.get("router_w"), router_logits=router_logits, bias=w.get("bias"),
-                         w13=w["w13"], w2=w["w2"], ws13=w.get("ws13"), ws2=w.get("ws2"))
+                         w13=w["w13"], w2=w["w2"], ws13=w.get("ws13"), ws2=w.get("ws2"),
+                         routed_scale=self.routed_scale, shared_gate_w=w.get("shared_gate"), shared_out=shared_out)
 
     def workspace(self, desc: LayerDesc, device) -> torch.Tensor:
         need = workspace_size(desc)
@@ -249,9 +256,11 @@ class MoELayer:
         return self._ws
 
     def forward(self, x: torch.Tensor, router_logits: Optional[torch.Tensor] = None, out=None,
-                return_routing: bool = False, stream=None):
+                return_routing: bool = False, stream=None, shared_out: Optional[torch.Tensor] = None):
+        """``shared_out``: a [T, H] BF16 shared-expert output to add (no internal shared
+        expert); ``out`` may be that same tensor (in-place form)."""
         T = x.shape[0]
-        d = self.desc(T, router_logits)
+        d = self.desc(T, router_logits, shared_out)
         ws = self.workspace(d, x.device)
         if out is None:
             out = torch.empty((T, self.shape.H), dtype=torch.bfloat16, device=x.device)

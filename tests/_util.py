@@ -23,7 +23,7 @@ def host_copy(d):
 
 
 def weights_of(d):
-    return {k: d[k] for k in ("router_w", "bias", "w13", "w2", "ws13", "ws2") if d.get(k) is not None}
+    return {k: d[k] for k in ("router_w", "bias", "w13", "w2", "ws13", "ws2", "shared_gate") if d.get(k) is not None}
 
 
 def bits_f64(t):

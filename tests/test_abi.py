@@ -170,3 +170,33 @@ def test_workspace_regions_lie_inside_the_workspace():
 
 def test_noalloc_get_error_validates_before_any_cuda_call():
     assert moe.lib().moe_noalloc_get_error(None, None) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_optional_parts_are_validated_on_the_host():
+    ws = FAKE * 16
+    d = _desc(T=4)
+    d.routed_scale = float("nan")
+    assert _fwd(d) == moe.MOE_ERR_INVALID_ARG
+    d = _desc(T=4)
+    d.routed_scale = float("inf")
+    assert _fwd(d) == moe.MOE_ERR_INVALID_ARG
+    d = _desc(T=4, I_shared=0)
+    d.ws13 = d.ws2 = None
+    d.shared_gate_w = FAKE * 9
+    assert _fwd(d) == moe.MOE_ERR_INVALID_ARG  # a gate needs an internal shared expert
+    d = _desc(T=4)
+    d.shared_out = FAKE * 9
+    assert _fwd(d) == moe.MOE_ERR_INVALID_ARG  # caller shared output and internal shared expert
+    d = _desc(T=4)
+    d.shared_gate_w = FAKE * 9 + 8
+    assert _fwd(d) == moe.MOE_ERR_INVALID_ARG  # misaligned
+    # output overlapping the input, or partly overlapping the caller's shared output
+    d = _desc(T=4, I_shared=0)
+    d.ws13 = d.ws2 = None
+    assert _fwd(d, x=FAKE * 6, out=FAKE * 6 + 256) == moe.MOE_ERR_INVALID_ARG
+    d.shared_out = FAKE * 9
+    assert _fwd(d, x=FAKE * 6, out=FAKE * 9 + 512) == moe.MOE_ERR_INVALID_ARG
+    # the in-place form (out is the shared output) passes validation and reaches the workspace check
+    assert _fwd(d, x=FAKE * 6, out=FAKE * 9) == moe.MOE_ERR_WORKSPACE
+    d.routed_scale = 2.5
+    assert _fwd(d, x=FAKE * 6, out=FAKE * 9) == moe.MOE_ERR_WORKSPACE
