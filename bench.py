@@ -183,6 +183,7 @@ def accounting(shape, T: int, U: int, router: bool, Is: int):
     rows1s = 2 * Is if shape.act == "swiglu" else Is
     h_bytes = (T * K * I + T * Is) * 2
     k = {}
+    k["prep"] = {"bytes": E * H * 2 if router and T > 64 else 0, "flops": 0}
     k["router"] = {"bytes": E * H * 2 + T * H * 2 + T * E * 4, "flops": 2 * T * E * H}
     k["topk"] = {"bytes": T * E * 4 + T * K * 8, "flops": 0}
     k["route"] = {"bytes": T * E * 4 + T * K * 8, "flops": 0}
@@ -208,6 +209,7 @@ def kernel_names(path: str, router: bool, launches: int = 0):
     names = ["router"] if router else []
     if path == "small":
         return names + ["route", "fc1", "fc2"]
+    names = ["prep"] + names
     if launches == len(names) + 7:  # top-k after the tensor-core router: screen, refine, final
         return names + ["topk", "refine", "select", "permute", "fc1", "fc2", "finalize"]
     return names + ["topk", "permute", "fc1", "fc2", "finalize"]

@@ -238,7 +238,7 @@ moe_status_t moe_fused_forward_timed(const moe_layer_desc* d, const void* x, voi
  *   - Device error flags (MOE_DEVERR_*) accumulate in the array's error word over calls
  *     until moe_noalloc_get_error reads and clears them.
  * ---------------------------------------------------------------------------------- */
-#define MOE_NOALLOC_SCRATCH_BYTES (4u << 20)
+#define MOE_NOALLOC_SCRATCH_BYTES (16u << 20)
 moe_status_t moe_fused_forward_noalloc(const moe_layer_desc* d, const void* x, void* out,
                                        float* topk_w_out, int32_t* topk_ids_out, float* logits_out,
                                        void* stream);

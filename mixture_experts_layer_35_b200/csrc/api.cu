@@ -12,17 +12,28 @@ namespace {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
 
+// SMs of the current device (148 on B200; also the value used without a device).
+int num_sms() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+    return n;
+}
+
 // Workspace carve-up of moe_fused_forward, 256-byte aligned regions after the header.
 struct WsLayout {
-    size_t logits, route, topk_w, topk_ids, offsets, tiles1, tiles2, counts, perm, cand, h, hs, acc, ys, gate, total;
+    size_t logits, route, topk_w, topk_ids, offsets, tiles1, tiles2, counts, wpart, perm, cand, h, hs, acc, skp, gate,
+        total;
 };
 // Candidate-list capacity per token of the three-kernel top-k (rows with more fall back).
 constexpr size_t kCandPerRow = 32;
-// Counters zeroed before each many-token call: per-expert counts, per-expert cursors,
-// then the candidate count and the router weight-row norm bound (a float, atomicMax).
-inline size_t counter_ints(size_t E) { return 2 * (E + 2) + 4; }
+// Counters zeroed at the start of each many-token call (prep kernel): per-expert counts,
+// per-expert cursors, the candidate count, then FC1's stream-K per-tile counters.
+inline size_t counter_ints(size_t E) { return 2 * (E + 2) + 4 + kStreamKMaxTiles; }
+inline size_t done_int(size_t E) { return 2 * (E + 2) + 4; }
 inline size_t cand_count_int(size_t E) { return 2 * (E + 2); }
-inline size_t wnorm2_int(size_t E) { return 2 * (E + 2) + 1; }
+// Per-CTA router weight-norm bounds of the prep kernel (its grid is at most E / 8 <= 128).
+constexpr size_t kMaxPrepGrid = (MOE_MAX_EXPERTS + 7) / 8;
 WsLayout layout(const moe_layer_desc* d) {
     const size_t T = (size_t)d->T, E = (size_t)d->E, K = (size_t)d->top_k, H = (size_t)d->H, I = (size_t)d->I,
                  Is = (size_t)d->I_shared;
@@ -41,12 +52,15 @@ WsLayout layout(const moe_layer_desc* d) {
     L.tiles1 = take((E + 2) * 4);
     L.tiles2 = take((E + 2) * 4);
     L.counts = take(counter_ints(E) * 4);
+    L.wpart = take(kMaxPrepGrid * 4);
     L.perm = take(T * K * 4);
     L.cand = take(T * (3 + 3 * kCandPerRow) * 4);  // row_base, row_n, row_eps, cand_row, cand_e, cand_val
     L.h = take(T * K * I * 2);
     L.hs = take(T * Is * 2);
-    L.acc = take(T * H * 4);
-    L.ys = take(Is ? T * H * 2 : 0);
+    L.acc = take(T * H * 4 * (Is ? 2 : 1));  // routed sum, then the shared expert's (FP32)
+    const int fc1_mode = d->act == MOE_ACT_SWIGLU ? GM_FC1_SWIGLU : GM_FC1_RELU2;
+    L.skp = take(fc1_streamk_bytes(gemm_token_tile(fc1_mode, d->T, d->top_k, d->E), d->act == MOE_ACT_SWIGLU,
+                                   num_sms()));
     L.gate = take(d->shared_gate_w ? T * 4 : 0);
     L.total = o;
     return L;
@@ -93,8 +107,12 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
 // streaming path was ahead at 100.7 MB of touched expert weights (Qwen3.6-shaped T = 2)
 // and behind at 108 MB (large-E-shaped T = 1, with its shared expert) and above.
 static constexpr double kSmallPathMaxBytes = 104e6;
+// The streaming path routes on exact logits: given ones, or the few-token router's.
+bool small_path_ok(const moe_layer_desc* d) {
+    return small_path_supported(d->T, d->H, d->I, d->I_shared) && (d->router_logits || router_small_supported(d->H));
+}
 int auto_path(const moe_layer_desc* d) {
-    if (!small_path_supported(d->T, d->H, d->I, d->I_shared)) return MOE_PATH_LARGE;
+    if (!small_path_ok(d)) return MOE_PATH_LARGE;
     const double m = d->act == MOE_ACT_SWIGLU ? 3.0 : 2.0;
     const double experts = (double)std::min(d->T * d->top_k, d->E);
     const double bytes = experts * m * d->H * d->I * 2.0 + m * d->H * (double)d->I_shared * 2.0;
@@ -105,12 +123,6 @@ int resolve_path(const moe_layer_desc* d) {
     return d->path;
 }
 
-int num_sms() {
-    int dev = 0, n = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
-    return n;
-}
 
 // ---------------------------------------------------------------- tensor maps
 bool map2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows) {
@@ -142,8 +154,8 @@ bool map3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint
     } while (0)
 
 // Router logits x . Wr^T on the tensor cores for many tokens (A = Wr, B = x rows).
-moe_status_t run_router_dense(const moe_layer_desc* d, const bf16* x, float* logits, float* copy, float* wnorm2,
-                              int sms, cudaStream_t s, int* err, bool pdl) {
+moe_status_t run_router_dense(const moe_layer_desc* d, const bf16* x, float* logits, float* copy, int sms,
+                              cudaStream_t s, int* err, bool pdl) {
     GemmArgs g;
     std::memset(&g, 0, sizeof(g));
     g.T = d->T;
@@ -154,7 +166,6 @@ moe_status_t run_router_dense(const moe_layer_desc* d, const bf16* x, float* log
     g.dense = 1;
     g.logits = logits;
     g.logits_copy = copy;
-    g.wnorm2 = wnorm2;
     g.err = err;
     GemmMaps m;
     std::memset(&m, 0, sizeof(m));
@@ -300,8 +311,8 @@ int moe_fused_forward_launches(const moe_layer_desc* d) {
     if (validate_desc(d) != MOE_OK || d->T == 0) return 0;
     const int router = d->router_logits ? 0 : 1;
     if (resolve_path(d) == MOE_PATH_SMALL) return router + 3;  // route table, fc1, fc2
-    if (dense_router_for(d) && split_topk_mode(d)) return router + 7;  // screen, refine, final, ...
-    return router + 5;                                          // topk, permute, fc1, fc2, finalize
+    if (dense_router_for(d) && split_topk_mode(d)) return router + 8;  // prep, screen, refine, final, ...
+    return router + 6;                                          // prep, topk, permute, fc1, fc2, finalize
 }
 
 static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, void* out_, float* topk_w_out,
@@ -321,7 +332,7 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
     const WsLayout L = layout(d);
     if (!ws || !aligned256(ws) || ws_bytes < L.total) return MOE_ERR_WORKSPACE;
     const int path = resolve_path(d);
-    if (path == MOE_PATH_SMALL && !small_path_supported(d->T, d->H, d->I, d->I_shared)) return MOE_ERR_UNSUPPORTED;
+    if (path == MOE_PATH_SMALL && !small_path_ok(d)) return MOE_ERR_UNSUPPORTED;
 
     cudaStream_t s = (cudaStream_t)stream;
     if (events && n_events < moe_fused_forward_launches(d) + 1) return MOE_ERR_INVALID_ARG;
@@ -341,32 +352,37 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
     const float rscale = d->routed_scale == 0.0f ? 1.0f : d->routed_scale;
     const bf16* sh_out = static_cast<const bf16*>(d->shared_out);
 
-    // 0. the many-token path's slot counters start at zero.  Cleared before the first
-    // kernel, so that every kernel launched with programmatic overlap follows a kernel
-    // (a memset between two kernels would leave the second one's overlap undefined).
-    if (path == MOE_PATH_LARGE) MOE_CK(cudaMemsetAsync(w8 + L.counts, 0, counter_ints(E) * sizeof(int), s));
+    // 0. many-token path: the prep kernel zeroes the slot counters and, before the
+    // tensor-core router, bounds the router rows' norms.  It is the call's first kernel
+    // (no programmatic overlap with the work before the call).
+    const bool dense_router = path == MOE_PATH_LARGE && dense_router_for(d);
+    float* wpart = reinterpret_cast<float*>(w8 + L.wpart);
+    bool pdl = false;
+    if (path == MOE_PATH_LARGE) {
+        if (!mark()) return MOE_ERR_CUDA;
+        MOE_CK(launch_prep(reinterpret_cast<int*>(w8 + L.counts), (int)counter_ints(E),
+                           dense_router ? static_cast<const bf16*>(d->router_w) : nullptr, E, H, wpart, sms, s));
+        pdl = !timed;
+    }
 
     // 1. router logits
     const float* logits = d->router_logits;
-    bool pdl = false;
-    bool dense_router = false;
     float* logits_rw = nullptr;
     if (!logits) {
         float* lg = logits_out ? logits_out : reinterpret_cast<float*>(w8 + L.logits);
         if (!mark()) return MOE_ERR_CUDA;
-        if (T <= 64 && router_small_supported(H)) {
-            MOE_CK(launch_router_small(x, static_cast<const bf16*>(d->router_w), T, H, E, lg, nullptr, err, s, false));
+        if (!dense_router && T <= 64 && router_small_supported(H)) {
+            MOE_CK(launch_router_small(x, static_cast<const bf16*>(d->router_w), T, H, E, lg, nullptr, err, s, pdl));
         } else {
-            float* wn2 = reinterpret_cast<float*>(w8 + L.counts) + wnorm2_int(E);
-            st = run_router_dense(d, x, lg, nullptr, wn2, sms, s, err, false);
+            st = run_router_dense(d, x, lg, nullptr, sms, s, err, pdl);
             if (st != MOE_OK) return st;
-            dense_router = true;
         }
         logits = lg;
         logits_rw = lg;
         pdl = !timed;
     } else if (logits_out) {
         MOE_CK(cudaMemcpyAsync(logits_out, logits, (size_t)T * E * 4, cudaMemcpyDeviceToDevice, s));
+        pdl = false;  // the next kernel follows a copy, not a kernel: no programmatic overlap
     }
 
     if (path == MOE_PATH_SMALL) {
@@ -416,7 +432,7 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
     bf16* h = reinterpret_cast<bf16*>(w8 + L.h);
     bf16* hs = reinterpret_cast<bf16*>(w8 + L.hs);
     float* acc = reinterpret_cast<float*>(w8 + L.acc);
-    bf16* ys = Is ? reinterpret_cast<bf16*>(w8 + L.ys) : nullptr;
+    float* acc_s = Is ? acc + (size_t)T * H : nullptr;
     float* gate = d->shared_gate_w ? reinterpret_cast<float*>(w8 + L.gate) : nullptr;
     const GateArgs ga = {x, static_cast<const bf16*>(d->shared_gate_w), H, gate};
 
@@ -426,8 +442,7 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
     const int bn1 = gemm_token_tile(fc1_mode, T, K, E), bn2 = gemm_token_tile(GM_FC2, T, K, E);
     // 2. top-k (also counts the slots per expert; the counters were cleared in step 0)
     if (!mark()) return MOE_ERR_CUDA;
-    RefineArgs ra = {x, static_cast<const bf16*>(d->router_w), H, logits_rw,
-                     reinterpret_cast<const float*>(counts + wnorm2_int(E)), err};
+    RefineArgs ra = {x, static_cast<const bf16*>(d->router_w), H, logits_rw, wpart, prep_grid(E, sms), err};
     if (dense_router && split_topk_mode(d)) {  // screen, refine, final
         int* cbase = reinterpret_cast<int*>(w8 + L.cand);
         CandList cl;
@@ -503,7 +518,10 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
     g1.h = h;
     g1.hs = hs;
     g1.zero_ptr = acc;
-    g1.zero_n = (size_t)T * H;
+    g1.zero_n = (size_t)T * H * (Is ? 2 : 1);
+    g1.streamk_max = gemm_streamk_max(fc1_mode, bn1, sms);
+    g1.skp = reinterpret_cast<float*>(w8 + L.skp);
+    g1.done = counts + done_int(E);
     g1.err = err;
     if (!mark()) return MOE_ERR_CUDA;
     MOE_CK(launch_gemm(fc1_mode, bn1, g1, m1, sms, s, chain));
@@ -527,16 +545,19 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
     g2.feat_s = H;
     g2.tiles = tiles2;
     g2.acc = acc;
-    g2.ys = ys;
+    g2.acc_s = acc_s;
     g2.sgate = gate;
     g2.zero_ptr = nullptr;
     g2.zero_n = 0;
+    g2.streamk_max = gemm_streamk_max(GM_FC2, bn2, sms);
+    g2.skp = nullptr;
+    g2.done = nullptr;
     if (!mark()) return MOE_ERR_CUDA;
     MOE_CK(launch_gemm(GM_FC2, bn2, g2, m2, sms, s, chain));
 
     // 6. finalize
     if (!mark()) return MOE_ERR_CUDA;
-    MOE_CK(launch_finalize(acc, Is ? ys : sh_out, out, (size_t)T * H, rscale, sms, s, chain));
+    MOE_CK(launch_finalize(acc, acc_s, sh_out, out, (size_t)T * H, rscale, sms, s, chain));
     if (!mark()) return MOE_ERR_CUDA;
     return MOE_OK;
 }

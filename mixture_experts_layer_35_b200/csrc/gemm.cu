@@ -17,10 +17,9 @@
 //       vector reductions, 4 consecutive features of one token per lane ("weighted output
 //       combination").
 //       The shared expert is one more group whose FC2 output is rounded to BF16 into ys.
-//   DENSE: router logits, A = Wr (128 experts per tile), B = x rows (TMA).  Four more
-//       warps read each A tile out of the ring as it arrives and sum the squares of its
-//       rows: the squared L2 norm of every router weight row, whose maximum bounds the
-//       tensor-core logits' accumulation error (used by the top-k kernels).
+//   DENSE: router logits, A = Wr (128 experts per tile), B = x rows (TMA).  It reads
+//       nothing an earlier kernel of the call writes, so it waits on the previous kernel
+//       (the call's prep kernel) only at its end and overlaps it.
 //
 // Warp roles (one CTA per SM, persistent over a group-major tile list):
 //   warp 0      TMA producer (weights; FC2/DENSE token rows)
@@ -30,7 +29,6 @@
 //               wide tiles eight (FC1) or twelve (FC2): the warps of a quarter take
 //               32-token column chunks in turn
 //   then        FC1 only: eight warps gathering token rows of x with cp.async
-//               DENSE only: four warps summing squares of the weight rows in the ring
 // Shared memory holds a ring of stages (full/empty mbarriers); TMEM holds two
 // accumulator buffers so the epilogue of one tile overlaps the mainloop of the next.
 #include "kernels.cuh"
@@ -83,9 +81,7 @@ struct Cfg {
     static constexpr int kGatherThreads = 32 * kGatherWarps;
     static constexpr int kGatherRowStep = kGather ? kGatherThreads / 8 : 16;  // (unused without a gather)
     static_assert(!kGather || kBN % kGatherRowStep == 0, "gather rows must tile the token tile");
-    // DENSE: one thread per A row (128) sums the squares of that weight row.
-    static constexpr int kNormWarps = (MODE == GM_DENSE) ? BM / 32 : 0;
-    static constexpr int kThreads = 64 + 32 * kEpiWarps + kGatherThreads + 32 * kNormWarps;
+    static constexpr int kThreads = 64 + 32 * kEpiWarps + kGatherThreads;
     // FC1 gather: stages of token rows in flight before the gather warps signal the oldest
     // one.  It must stay at most kStages - 2: the gather can only issue stage j + lag once
     // the MMA has freed that slot, so with lag = kStages - 1 the signal for stage j waits
@@ -156,6 +152,76 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmArgs& a, const int* s_
     return ti;
 }
 
+// One unit of a CTA's work: a whole tile, or (stream-K) a contiguous range of its k-blocks.
+enum SegKind { kWhole = 0, kFixer = 1, kPart = 2 };
+struct Seg {
+    int tile, kb0, kb1;
+    int kind;  // kWhole; kFixer: holds the tile's first k-blocks and adds the other CTAs' partial
+               // sums before the epilogue (FC1); kPart: a later k-block range (FC1: its partial
+               // sum goes to this CTA's scratch slot; FC2: reduced into the accumulator directly)
+    int last;  // kFixer: last CTA whose range holds k-blocks of this tile
+};
+
+// A CTA's work.  Without stream-K, tiles are dealt round-robin.  With stream-K (few tiles
+// for the grid: one wave or a few, where whole tiles would leave SMs idle at the end),
+// the iteration space -- every tile's k-blocks, tiles in group-major order, routed tiles
+// with nk_r k-blocks and the shared group's with nk_s -- is split into gridDim.x equal
+// contiguous ranges, cut at tile boundaries into segments.  Every role of the CTA walks
+// the same sequence.
+struct WorkWalk {
+    int total, R, nk_r, nk_s, streamk, next_tile;
+    long long N, hi, i;
+    __device__ void init(int total_, int R_, int nk_r_, int nk_s_, bool sk) {
+        total = total_;
+        R = R_;
+        nk_r = nk_r_;
+        nk_s = nk_s_;
+        streamk = sk ? 1 : 0;
+        N = (long long)R * nk_r + (long long)(total - R) * nk_s;
+        i = lo_of(blockIdx.x);
+        hi = lo_of(blockIdx.x + 1);
+        next_tile = blockIdx.x;
+    }
+    __device__ long long lo_of(int b) const { return N * b / gridDim.x; }
+    // CTA whose range holds iteration it: the largest b with lo_of(b) <= it.
+    __device__ int owner(long long it) const { return (int)(((it + 1) * gridDim.x - 1) / N); }
+    __device__ bool next(Seg& s) {
+        if (!streamk) {
+            if (next_tile >= total) return false;
+            s.tile = next_tile;
+            s.kb0 = 0;
+            s.kb1 = next_tile < R ? nk_r : nk_s;
+            s.kind = kWhole;
+            s.last = blockIdx.x;
+            next_tile += gridDim.x;
+            return true;
+        }
+        if (i >= hi) return false;
+        const long long rr = (long long)R * nk_r;
+        long long tb;
+        int nk;
+        if (i < rr) {
+            s.tile = (int)(i / nk_r);
+            tb = (long long)s.tile * nk_r;
+            nk = nk_r;
+        } else {
+            const int j = (int)((i - rr) / nk_s);
+            s.tile = R + j;
+            tb = rr + (long long)j * nk_s;
+            nk = nk_s;
+        }
+        const long long end = hi < tb + nk ? hi : tb + nk;
+        s.kb0 = (int)(i - tb);
+        s.kb1 = (int)(end - tb);
+        s.kind = (s.kb0 == 0 && s.kb1 == nk) ? kWhole : (s.kb0 == 0 ? kFixer : kPart);
+        s.last = s.kind == kFixer ? owner(tb + nk - 1) : (int)blockIdx.x;
+        i = end;
+        return true;
+    }
+    // CTA c holds iterations (its range is not empty).
+    __device__ bool active(int c) const { return lo_of(c) < lo_of(c + 1); }
+};
+
 template <int MODE, int BN>
 __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
     gemm_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ CUtensorMap tm_a_s,
@@ -183,7 +249,7 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kStages; ++s) {
             mbar_init(full_bar(s), 1 + C::kGatherThreads);
-            mbar_init(empty_bar(s), 1 + C::kNormWarps);
+            mbar_init(empty_bar(s), 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(tfull_bar(b), 1);
@@ -202,8 +268,9 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
     }
     if (warp == 1) tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
 
-    // Everything below reads what earlier kernels wrote (tile tables, perm, h).
-    pdl_wait();
+    // Everything below reads what earlier kernels wrote (tile tables, perm, h) -- except
+    // in DENSE mode, which reads only the caller's x and Wr and waits at its end.
+    if (MODE != GM_DENSE) pdl_wait();
     if (!a.dense) {
         for (int i = threadIdx.x; i <= G; i += blockDim.x) s_tiles[i] = a.tiles[i];
         for (int i = threadIdx.x; i <= a.E; i += blockDim.x) s_offs[i] = a.offsets[i];
@@ -213,18 +280,24 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     const int total = a.dense ? a.nfeat_r * cdiv(a.T, kDenseTokenTile) : s_tiles[G];
-    // Tiles are dealt round-robin over the persistent CTAs: at any moment the CTAs work on
-    // neighbouring tiles of the group-major list (one expert's feature and token tiles),
-    // which share that expert's weight rows and token rows in L2, and tiles of unequal
-    // cost (ragged token tails) spread evenly.
+    const int routed_tiles = (a.dense || !a.has_shared) ? total : s_tiles[a.E];
+    const bool streamk = total > 0 && total < a.streamk_max;
+    const int nk_r = cdiv(a.kdim, BK), nk_s = cdiv(a.kdim_s > 0 ? a.kdim_s : a.kdim, BK);
+    // Round-robin dealing keeps the CTAs on neighbouring tiles of the group-major list (one
+    // expert's feature and token tiles), which share that expert's weight and token rows in
+    // L2, and spreads tiles of unequal cost (ragged token tails) evenly.
+    WorkWalk work;
+    work.init(total, routed_tiles, nk_r, nk_s, streamk);
+    Seg sg;
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             const uint64_t wpol = l2_policy_evict_first();
             int it = 0;
-            for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
-                const TileInfo ti = decode_tile<C::kBN>(a, s_tiles, s_offs, G, tile);
+            while (!*abort_flag && work.next(sg)) {
+                const TileInfo ti = decode_tile<C::kBN>(a, s_tiles, s_offs, G, sg.tile);
+                if (ti.nk == 0) continue;
                 const bool sh = ti.shared;
                 const CUtensorMap* ta = sh ? &tm_a_s : &tm_a_r;
                 const CUtensorMap* tb = sh ? &tm_b_s : &tm_b_r;
@@ -232,10 +305,14 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
                 constexpr int BBOX = b_box_rows<MODE>();
                 const int nbox = cdiv(ti.n, BBOX);
                 const uint32_t bytes = C::kNA * A_BYTES + (C::kGather ? 0u : (uint32_t)nbox * BBOX * BK * 2);
-                for (int kb = 0; kb < ti.nk; ++kb, ++it) {
+                bool ok = true;
+                for (int kb = sg.kb0; kb < sg.kb1; ++kb, ++it) {
                     const int s = it % C::kStages;
                     const uint32_t ph = (uint32_t)(it / C::kStages) & 1u;
-                    if (!mbar_wait(empty_bar(s), ph ^ 1u, abort_flag, a.err)) break;
+                    if (!mbar_wait(empty_bar(s), ph ^ 1u, abort_flag, a.err)) {
+                        ok = false;
+                        break;
+                    }
                     const uint32_t st = base_u32 + (uint32_t)s * C::kStageBytes;
                     mbar_expect_tx(full_bar(s), bytes);
                     if (sh || a.dense) {
@@ -260,15 +337,16 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
                                         ti.row0 + q * BBOX);
                     }
                 }
+                if (!ok) break;
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             int it = 0, tcount = 0;
-            for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x, ++tcount) {
-                const TileInfo ti = decode_tile<C::kBN>(a, s_tiles, s_offs, G, tile);
-                const int nk = ti.nk;
+            while (!*abort_flag && work.next(sg)) {
+                const TileInfo ti = decode_tile<C::kBN>(a, s_tiles, s_offs, G, sg.tile);
+                if (ti.nk == 0) continue;
                 const int npad = cdiv(ti.n, 16) * 16;
                 const uint32_t idesc = idesc_bf16_f32(BM, npad);
                 const int buf = tcount % C::kAccBufs;
@@ -278,7 +356,7 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
                 const uint32_t d0 = tmem_base + (uint32_t)(buf * C::kAccStride);
                 const uint32_t d1 = d0 + C::kBN;
                 bool ok = true;
-                for (int kb = 0; kb < nk; ++kb, ++it) {
+                for (int kb = sg.kb0; kb < sg.kb1; ++kb, ++it) {
                     const int s = it % C::kStages;
                     const uint32_t ph = (uint32_t)(it / C::kStages) & 1u;
                     if (!mbar_wait(full_bar(s), ph, abort_flag, a.err)) {
@@ -290,7 +368,7 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
                     const uint32_t bsm = st + C::kNA * A_BYTES;
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk) {
-                        const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
+                        const uint32_t accum = (kb > sg.kb0 || kk > 0) ? 1u : 0u;
                         const uint64_t bdesc = sdesc_sw128(bsm + kk * 32);
                         tc_mma(d0, sdesc_sw128(st + kk * 32), bdesc, idesc, accum);
                         if (C::kSwiglu) tc_mma(d1, sdesc_sw128(st + A_BYTES + kk * 32), bdesc, idesc, accum);
@@ -299,12 +377,13 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
                 }
                 if (!ok) break;
                 tc_commit(tfull_bar(buf));
+                ++tcount;
             }
         }
     } else if (warp < 2 + C::kEpiWarps) {
         // ------------------------------------------------------------ epilogue
         const int q = warp & 3;                     // TMEM lane quarter of this warp
-        const int half = (warp - 2) >> 2;          // FC2: which token columns (chunk parity)
+        const int half = (warp - 2) >> 2;          // which token columns (chunk parity)
         const int nhalf = C::kEpiWarps / 4;
         const int et = threadIdx.x - 64;
         if (a.zero_ptr) {
@@ -314,16 +393,20 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
             for (size_t i = (size_t)blockIdx.x * ne + et; i < n4; i += (size_t)gridDim.x * ne)
                 z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
+        // FC1 stream-K scratch: one slot per CTA, [kNA][BN token columns][128 features] FP32.
+        constexpr size_t kSlotFloats = (size_t)C::kNA * C::kBN * BM;
         int tcount = 0;
-        // (the abort flag is checked through the per-tile wait below)
         // 32-token chunks per half of the epilogue warps (the last may lie past the tile)
         constexpr int kChunks = (C::kBN + 32 * (C::kEpiWarps / 4) - 1) / (32 * (C::kEpiWarps / 4));
-        for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++tcount) {
-            const TileInfo ti = decode_tile<C::kBN>(a, s_tiles, s_offs, G, tile);
+        while (work.next(sg)) {
+            const TileInfo ti = decode_tile<C::kBN>(a, s_tiles, s_offs, G, sg.tile);
+            if (ti.nk == 0) continue;
             const int buf = tcount % C::kAccBufs;
             const uint32_t tph = (uint32_t)(tcount / C::kAccBufs) & 1u;
-            // FC2: token and routing weight of each column this thread will scale, loaded
-            // before the accumulator is ready (hidden behind the tile's mainloop).
+            // FC2: token and weight of each column this thread will scale, loaded before the
+            // accumulator is ready (hidden behind the tile's mainloop).  Routed rows are
+            // permuted slots (token, routing weight); the shared expert's rows are the tokens
+            // in order (weight: the shared-expert gate, or 1).
             int mt[kChunks];
             float mw[kChunks];
 #pragma unroll
@@ -331,14 +414,19 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
                 mt[ci] = 0;
                 mw[ci] = 0.0f;
                 const int colm = 32 * half + 32 * nhalf * ci + lane;
-                if (MODE == GM_FC2 && !ti.shared && colm < ti.n && ti.row0 + ti.n <= a.T * a.K) {
-                    const int src = a.perm[ti.row0 + colm];
-                    if ((unsigned)src < (unsigned)(a.T * a.K)) {
-                        const int kk = src / a.T;
-                        mt[ci] = src - kk * a.T;
-                        mw[ci] = a.topk_w[(size_t)mt[ci] * a.K + kk];
-                    } else {  // never from a valid permutation: flag it, contribute nothing
-                        set_dev_error(a.err, MOE_DEVERR_BAD_INDEX);
+                if (MODE == GM_FC2 && colm < ti.n) {
+                    if (ti.shared) {
+                        mt[ci] = ti.row0 + colm;
+                        mw[ci] = a.sgate ? a.sgate[mt[ci]] : 1.0f;
+                    } else if (ti.row0 + ti.n <= a.T * a.K) {
+                        const int src = a.perm[ti.row0 + colm];
+                        if ((unsigned)src < (unsigned)(a.T * a.K)) {
+                            const int kk = src / a.T;
+                            mt[ci] = src - kk * a.T;
+                            mw[ci] = a.topk_w[(size_t)mt[ci] * a.K + kk];
+                        } else {  // never from a valid permutation: flag it, contribute nothing
+                            set_dev_error(a.err, MOE_DEVERR_BAD_INDEX);
+                        }
                     }
                 }
             }
@@ -353,6 +441,70 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
             const int feat = ti.shared ? a.feat_s : a.feat_r;
             const bool fok = f < feat;
             const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * C::kAccStride);
+            if (C::kGather && sg.kind == kPart) {
+                // ---- stream-K, FC1: a later k-block range; its partial sums go to this CTA's
+                // slot, then the tile's counter tells the fixer it is there.
+                float* slot = a.skp + (size_t)blockIdx.x * kSlotFloats;
+#pragma unroll
+                for (int ci = 0; ci < kChunks; ++ci) {
+                    const int c0 = 32 * half + 32 * nhalf * ci;
+                    if (c0 >= ti.n || !rows_ok) break;
+                    uint32_t v[32];
+                    tmem_ld32(tb + c0, v);
+                    uint32_t u[32];
+                    if (C::kSwiglu) tmem_ld32(tb + C::kBN + c0, u);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int col = c0 + j;
+                        if (col < ti.n) {
+                            slot[(size_t)col * BM + q * 32 + lane] = __uint_as_float(v[j]);
+                            if (C::kSwiglu) slot[(size_t)(C::kBN + col) * BM + q * 32 + lane] = __uint_as_float(u[j]);
+                        }
+                    }
+                }
+                // Each warp publishes its own rows: every lane's stores are fenced, then the
+                // warp's lane 0 counts it on the tile's counter (no barrier across warps).
+                __threadfence();
+                __syncwarp();
+                if (lane == 0) atomicAdd(a.done + sg.tile, 1);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(tempty_bar(buf));
+                ++tcount;
+                continue;
+            }
+            int ncontrib = 0;
+            if (C::kGather && sg.kind == kFixer) {
+                // ---- stream-K, FC1: this CTA holds the tile's first k-blocks.  Each warp waits
+                // (bounded) until every warp of every later range has published its partial,
+                // then adds them below.
+                for (int c = blockIdx.x + 1; c <= sg.last; ++c) ncontrib += work.active(c) ? 1 : 0;
+                int ok = 1;
+                if (lane == 0) {
+                    const volatile int* cnt = a.done + sg.tile;
+                    const int target = ncontrib * C::kEpiWarps;
+                    const uint64_t t0 = globaltimer_ns();
+                    uint32_t n = 0;
+                    while (*cnt < target) {
+                        if ((++n & 255u) == 0) {
+                            if (*abort_flag) {
+                                ok = 0;
+                                break;
+                            }
+                            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                                *abort_flag = 1;
+                                set_dev_error(a.err, MOE_DEVERR_WAIT_TIMEOUT);
+                                ok = 0;
+                                break;
+                            }
+                        }
+                    }
+                    __threadfence();
+                }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
+            }
 #pragma unroll
             for (int ci = 0; ci < kChunks; ++ci) {
                 const int c0 = 32 * half + 32 * nhalf * ci;
@@ -362,6 +514,23 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
                 uint32_t u[32];
                 if (C::kSwiglu) tmem_ld32(tb + C::kBN + c0, u);
                 tmem_ld_wait();
+                if (C::kGather && ncontrib > 0) {  // the later ranges' partial sums, in CTA order
+                    for (int c = blockIdx.x + 1; c <= sg.last; ++c) {
+                        if (!work.active(c)) continue;
+                        const float* slot = a.skp + (size_t)c * kSlotFloats;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const int col = c0 + j;
+                            if (col < ti.n) {
+                                v[j] = __float_as_uint(__uint_as_float(v[j]) +
+                                                       __ldcg(slot + (size_t)col * BM + q * 32 + lane));
+                                if (C::kSwiglu)
+                                    u[j] = __float_as_uint(__uint_as_float(u[j]) +
+                                                           __ldcg(slot + (size_t)(C::kBN + col) * BM + q * 32 + lane));
+                            }
+                        }
+                    }
+                }
                 if (C::kGather) {
                     bf16* dst = ti.shared ? a.hs : a.h;
                     const int ld = feat;
@@ -376,58 +545,49 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
                         }
                     }
                 } else if (MODE == GM_FC2) {
-                    if (ti.shared) {  // shared rows are the tokens in order; optional sigmoid gate
+                    // Column j of this chunk is token t_j with weight w_j; lane l holds feature
+                    // f0 + l.  Each block of 4 columns is transposed within groups of 4 lanes
+                    // (two XOR-shuffle stages), after which lane 4g+i holds features
+                    // f0+4g .. f0+4g+3 of token t_{j0+i}, scales them by w_{j0+i} (one shuffle
+                    // brings the token, one the weight) and adds them into the FP32
+                    // accumulator (routed rows: acc; the shared expert: acc_s) with one 16-byte
+                    // vector reduction (FP32 add in L2).  A stream-K range adds its partial
+                    // sum the same way.  No shared memory is staged, so the ring keeps it for
+                    // weights.
+                    float* dstacc = ti.shared ? a.acc_s : a.acc;
+                    const int i4 = lane & 3;
+                    const bool fok4 = f - i4 + 3 < feat;  // features of my group (feat % 8 == 0)
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            const int col = c0 + j;
-                            if (col < ti.n && fok) {
-                                float y = __uint_as_float(v[j]);
-                                if (a.sgate) y = __fmul_rn(a.sgate[ti.row0 + col], y);
-                                a.ys[(size_t)(ti.row0 + col) * a.feat_s + f] = __float2bfloat16_rn(y);
-                            }
+                    for (int j0 = 0; j0 < 32; j0 += 4) {
+                        float r[4];
+#pragma unroll
+                        for (int jj = 0; jj < 4; ++jj) r[jj] = __uint_as_float(v[j0 + jj]);
+                        // r[jj] = y[feature of this lane, token j0 + jj]; 4x4 transpose
+                        float t0 = (i4 & 1) ? r[0] : r[1], t1 = (i4 & 1) ? r[2] : r[3];
+                        t0 = __shfl_xor_sync(0xffffffffu, t0, 1);
+                        t1 = __shfl_xor_sync(0xffffffffu, t1, 1);
+                        if (i4 & 1) {
+                            r[0] = t0;
+                            r[2] = t1;
+                        } else {
+                            r[1] = t0;
+                            r[3] = t1;
                         }
-                    } else {
-                        // Column j of this chunk is token t_j with routing weight w_j; lane l
-                        // holds feature f0 + l.  Each block of 4 columns is transposed within
-                        // groups of 4 lanes (two XOR-shuffle stages), after which lane 4g+i
-                        // holds features f0+4g .. f0+4g+3 of token t_{j0+i}, scales them by
-                        // w_{j0+i} (one shuffle brings the token, one the weight) and adds
-                        // them into acc with one 16-byte vector reduction (FP32 add in L2).
-                        // No shared memory is staged, so the ring keeps it for weights.
-                        const int i4 = lane & 3;
-                        const bool fok4 = f - i4 + 3 < a.feat_r;  // features of my group (feat_r % 8 == 0)
-#pragma unroll
-                        for (int j0 = 0; j0 < 32; j0 += 4) {
-                            float r[4];
-#pragma unroll
-                            for (int jj = 0; jj < 4; ++jj) r[jj] = __uint_as_float(v[j0 + jj]);
-                            // r[jj] = y[feature of this lane, token j0 + jj]; 4x4 transpose
-                            float t0 = (i4 & 1) ? r[0] : r[1], t1 = (i4 & 1) ? r[2] : r[3];
-                            t0 = __shfl_xor_sync(0xffffffffu, t0, 1);
-                            t1 = __shfl_xor_sync(0xffffffffu, t1, 1);
-                            if (i4 & 1) {
-                                r[0] = t0;
-                                r[2] = t1;
-                            } else {
-                                r[1] = t0;
-                                r[3] = t1;
-                            }
-                            float u0 = (i4 & 2) ? r[0] : r[2], u1 = (i4 & 2) ? r[1] : r[3];
-                            u0 = __shfl_xor_sync(0xffffffffu, u0, 2);
-                            u1 = __shfl_xor_sync(0xffffffffu, u1, 2);
-                            if (i4 & 2) {
-                                r[0] = u0;
-                                r[1] = u1;
-                            } else {
-                                r[2] = u0;
-                                r[3] = u1;
-                            }
-                            const int tok = __shfl_sync(0xffffffffu, mt[ci], j0 + i4);
-                            const float wt = __shfl_sync(0xffffffffu, mw[ci], j0 + i4);
-                            if (c0 + j0 + i4 < ti.n && fok4 && (unsigned)tok < (unsigned)a.T)
-                                red_add_v4_f32(a.acc + (size_t)tok * a.feat_r + (f - i4), wt * r[0], wt * r[1],
-                                               wt * r[2], wt * r[3]);
+                        float u0 = (i4 & 2) ? r[0] : r[2], u1 = (i4 & 2) ? r[1] : r[3];
+                        u0 = __shfl_xor_sync(0xffffffffu, u0, 2);
+                        u1 = __shfl_xor_sync(0xffffffffu, u1, 2);
+                        if (i4 & 2) {
+                            r[0] = u0;
+                            r[1] = u1;
+                        } else {
+                            r[2] = u0;
+                            r[3] = u1;
                         }
+                        const int tok = __shfl_sync(0xffffffffu, mt[ci], j0 + i4);
+                        const float wt = __shfl_sync(0xffffffffu, mw[ci], j0 + i4);
+                        if (c0 + j0 + i4 < ti.n && fok4 && (unsigned)tok < (unsigned)a.T)
+                            red_add_v4_f32(dstacc + (size_t)tok * feat + (f - i4), wt * r[0], wt * r[1],
+                                           wt * r[2], wt * r[3]);
                     }
                 } else {  // GM_DENSE
 #pragma unroll
@@ -444,16 +604,17 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(tempty_bar(buf));
+            ++tcount;
         }
     } else if (C::kGather) {
         // ------------------------------------------------------------ FC1 token gather
         const int p = threadIdx.x - (64 + 32 * C::kEpiWarps);  // 0 .. kGatherThreads - 1
         const int chunk = p & 7, rsub = p >> 3;
         int it = 0;
-        for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
-            const TileInfo ti = decode_tile<C::kBN>(a, s_tiles, s_offs, G, tile);
+        while (!*abort_flag && work.next(sg)) {
+            const TileInfo ti = decode_tile<C::kBN>(a, s_tiles, s_offs, G, sg.tile);
+            if (ti.nk == 0) continue;
             const int kd = ti.shared ? a.kdim_s : a.kdim;
-            const int nk = ti.nk;
             const int npad = cdiv(ti.n, 16) * 16;
             int tok[C::kBN / C::kGatherRowStep];
 #pragma unroll
@@ -470,7 +631,7 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
                 }
             }
             bool ok = true;
-            for (int kb = 0; kb < nk; ++kb, ++it) {
+            for (int kb = sg.kb0; kb < sg.kb1; ++kb, ++it) {
                 const int s = it % C::kStages;
                 const uint32_t ph = (uint32_t)(it / C::kStages) & 1u;
                 if (!mbar_wait(empty_bar(s), ph ^ 1u, abort_flag, a.err)) {
@@ -501,40 +662,6 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
         cp_async_wait<0>();
         fence_proxy_async_smem();
         for (int j = max(0, it - C::kLag); j < it; ++j) mbar_arrive(full_bar(j % C::kStages));
-    } else if (C::kNormWarps) {
-        // ------------------------------------------------------------ DENSE: weight-row norms
-        // Thread r owns A row r of every stage: its 64 BF16 values occupy bytes
-        // [128 r, 128 r + 128) of the tile (the 128-byte swizzle only permutes the 16-byte
-        // chunks inside a row), so the sum of their squares needs no unswizzling.  Rows
-        // past E are zero-filled by TMA.  The FP32 sum of H squares is within a relative
-        // H * 2^-24 of the exact value; it is scaled up by (1 + 2^-8) (H <= 2^16), so the
-        // result is an upper bound.  The maximum over rows goes to a.wnorm2 (atomicMax on
-        // the bits of a non-negative float orders like the float).
-        const int r = threadIdx.x - (64 + 32 * C::kEpiWarps + C::kGatherThreads);
-        int it = 0;
-        for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
-            const TileInfo ti = decode_tile<C::kBN>(a, s_tiles, s_offs, G, tile);
-            float ss = 0.0f;
-            bool ok = true;
-            for (int kb = 0; kb < ti.nk; ++kb, ++it) {
-                const int s = it % C::kStages;
-                const uint32_t ph = (uint32_t)(it / C::kStages) & 1u;
-                if (!mbar_wait(full_bar(s), ph, abort_flag, a.err)) {
-                    ok = false;
-                    break;
-                }
-                const uint4* row = reinterpret_cast<const uint4*>(base + (size_t)s * C::kStageBytes + (size_t)r * 128);
-#pragma unroll
-                for (int c = 0; c < 8; ++c) ss = dot8(row[c], row[c], ss);
-                __syncwarp();
-                if (lane == 0) mbar_arrive(empty_bar(s));
-            }
-            if (!ok) break;
-            float m = ss * (1.0f + 0x1p-8f);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-            if (lane == 0 && a.wnorm2) atomicMax(reinterpret_cast<int*>(a.wnorm2), __float_as_int(m));
-        }
     }
 
     tc_fence_before();
@@ -546,14 +673,15 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
         }
     }
     if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
+    if (MODE == GM_DENSE) pdl_wait();  // the previous kernel is complete before this one is
     pdl_trigger();
 }
 
 // ---------------------------------------------------------------- finalize
-// `ys` may be the caller's shared output and `out` that same buffer: each thread reads
+// `sh_out` may be the caller's shared output and `out` that same buffer: each thread reads
 // its 8 elements before writing them, so the in-place form is safe (no __restrict__).
-__global__ void __launch_bounds__(256) finalize_kernel(const float* __restrict__ acc, const bf16* ys, bf16* out,
-                                                       size_t n, float scale) {
+__global__ void __launch_bounds__(256) finalize_kernel(const float* __restrict__ acc, const float* __restrict__ acc_s,
+                                                       const bf16* sh_out, bf16* out, size_t n, float scale) {
     pdl_wait();
     const size_t stride = (size_t)gridDim.x * blockDim.x * 8;
     for (size_t i = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) * 8; i < n; i += stride) {
@@ -564,8 +692,14 @@ __global__ void __launch_bounds__(256) finalize_kernel(const float* __restrict__
 #pragma unroll
             for (int j = 0; j < 8; ++j) r[j] = __fmul_rn(scale, r[j]);
         }
-        if (ys) {
-            const uint4 y = *reinterpret_cast<const uint4*>(ys + i);
+        if (acc_s) {  // routed -> BF16, shared -> BF16, BF16 add
+            const float4 s0 = *reinterpret_cast<const float4*>(acc_s + i);
+            const float4 s1 = *reinterpret_cast<const float4*>(acc_s + i + 4);
+            const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+#pragma unroll
+            for (int j = 0; j < 8; ++j) r[j] = __fadd_rn(bf_round(r[j]), bf_round(sv[j]));
+        } else if (sh_out) {
+            const uint4 y = *reinterpret_cast<const uint4*>(sh_out + i);
             const uint32_t yw[4] = {y.x, y.y, y.z, y.w};
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
@@ -637,12 +771,23 @@ cudaError_t launch_gemm(int mode, int bn, const GemmArgs& a, const GemmMaps& m, 
     return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_finalize(const float* acc, const bf16* ys, bf16* out, size_t n, float scale, int num_sms,
-                            cudaStream_t s, bool pdl) {
+cudaError_t launch_finalize(const float* acc, const float* acc_s, const bf16* sh_out, bf16* out, size_t n,
+                            float scale, int num_sms, cudaStream_t s, bool pdl) {
     const size_t groups = n / 8;
     int grid = (int)std::min<size_t>((groups + 255) / 256, (size_t)num_sms * 4);
     if (grid < 1) grid = 1;
-    return launch_k(finalize_kernel, dim3(grid), dim3(256), 0, s, pdl, acc, ys, out, n, scale);
+    return launch_k(finalize_kernel, dim3(grid), dim3(256), 0, s, pdl, acc, acc_s, sh_out, out, n, scale);
+}
+
+size_t fc1_streamk_bytes(int bn, bool swiglu, int grid) {
+    if (bn > kStreamKMaxBN) return 0;
+    return (size_t)grid * (swiglu ? 2 : 1) * bn * BM * sizeof(float);
+}
+
+int gemm_streamk_max(int mode, int bn, int grid) {
+    if (mode == GM_DENSE) return 0;
+    if (mode == GM_FC2) return kStreamKWaves * grid;
+    return bn <= kStreamKMaxBN ? std::min(kStreamKWaves * grid, kStreamKMaxTiles) : 0;
 }
 
 }  // namespace moe

@@ -33,7 +33,8 @@ struct RefineArgs {
     const bf16* wr;      // [E, H]
     int H;
     float* logits_rw;    // refined logits are written back here (the logits buffer)
-    const float* wnorm2; // max over experts of |Wr[e]|_2^2 (upper bound), from the router GEMM
+    const float* wpart;  // [nwpart] per-CTA upper bounds of max_e |Wr[e]|_2^2 (prep kernel)
+    int nwpart;
     int* err;            // device error word (MOE_DEVERR_ROUTER_BOUND)
 };
 // Shared-expert gate of each token, computed by the routing kernels (one exact dot
@@ -108,6 +109,13 @@ bool small_path_supported(int T, int H, int I, int Is);
 cudaError_t launch_small(const SmallArgs& a, int num_sms, cudaStream_t s, bool pdl_first,
                          const std::function<bool()>* mark);
 
+// First kernel of a many-token call: zeroes the call's counters (n ints) and, when wr is
+// given, writes per-CTA upper bounds of max_e |wr[e]|_2^2 into wpart[prep_grid(E, sms)]
+// (the bound on the tensor-core router's error uses their maximum).
+int prep_grid(int E, int num_sms);
+cudaError_t launch_prep(int* counters, int n, const bf16* wr, int E, int H, float* wpart, int num_sms,
+                        cudaStream_t s);
+
 // ---------------------------------------------------------------- permutation
 // Tile bookkeeping that the permute kernel writes for the grouped GEMMs (group g < E is
 // routed expert g; g == E is the shared expert when present, with T rows).
@@ -157,14 +165,15 @@ struct GemmArgs {
     bf16* h;                 // FC1 routed out [T*K, I]
     bf16* hs;                // FC1 shared out [T, I_s]
     float* acc;              // FC2 routed out [T, H] (FP32 red.add)
-    bf16* ys;                // FC2 shared out [T, H]
+    float* acc_s;            // FC2 shared-expert out [T, H] (FP32 red.add)
     float* logits;           // GM_DENSE out [T, E]
     float* logits_copy;      // GM_DENSE optional second output
     float* zero_ptr;         // FC1: buffer zeroed by the epilogue warps before their tiles
     size_t zero_n;           //      (floats, multiple of 4)
-    float* wnorm2;           // GM_DENSE: max over experts of |Wr[e]|_2^2 (upper bound), atomicMax;
-                             //           zero on entry, or null
-    const float* sgate;      // FC2: shared-expert gate per token (ys = bf16(gate[t] * y)), or null
+    const float* sgate;      // FC2: shared-expert gate per token (acc_s += gate[t] * y), or null
+    int streamk_max;         // stream-K when the call has fewer tiles than this (0: never)
+    float* skp;              // FC1 stream-K partial sums, one slot per CTA ([kNA][BN][128] FP32)
+    int* done;               // FC1 stream-K per-tile counters (zero on entry, >= streamk_max of them)
     int* err;
 };
 struct GemmMaps {
@@ -183,10 +192,21 @@ int gemm_token_tile(int mode, int T, int K, int E);
 constexpr int kFc2BoxRows = 32;
 cudaError_t launch_gemm(int mode, int bn, const GemmArgs& a, const GemmMaps& m, int grid, cudaStream_t s, bool pdl);
 
-// finalize: out = bf16(bf16(scale * acc) + ys) or bf16(scale * acc); out may equal ys
-// (each element is read before it is written, by the same thread).
-cudaError_t launch_finalize(const float* acc, const bf16* ys, bf16* out, size_t n, float scale, int num_sms,
-                            cudaStream_t s, bool pdl);
+// Stream-K limits: FC1 and FC2 run stream-K while a call has fewer tiles than
+// kStreamKWaves waves of the grid; FC1 only with token tiles of at most 64 rows (its
+// partial-sum slots) and at most kStreamKMaxTiles tiles (its counters).
+static constexpr int kStreamKWaves = 8;
+static constexpr int kStreamKMaxTiles = 1024;
+static constexpr int kStreamKMaxBN = 64;
+// Bytes of FC1's stream-K partial-sum slots for `grid` CTAs (0 when FC1 cannot use it).
+size_t fc1_streamk_bytes(int bn, bool swiglu, int grid);
+int gemm_streamk_max(int mode, int bn, int grid);
+
+// finalize: out = bf16(bf16(scale * acc) + shared) with shared = bf16(acc_s) (internal
+// shared expert) or sh_out (caller's), or bf16(scale * acc) without one.  out may equal
+// sh_out (each element is read before it is written, by the same thread).
+cudaError_t launch_finalize(const float* acc, const float* acc_s, const bf16* sh_out, bf16* out, size_t n,
+                            float scale, int num_sms, cudaStream_t s, bool pdl);
 
 // Driver entry point for tensor-map encoding (resolved once through the runtime).
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,

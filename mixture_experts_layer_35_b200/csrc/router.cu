@@ -57,6 +57,57 @@ __device__ __forceinline__ void shared_gate_row(const GateArgs& g, int row, int 
     if (lane == 0) g.out[row] = sigmoid_f32_rn(l);
 }
 
+// ---------------------------------------------------------------- call prep
+// First kernel of a many-token call.  CTA 0 zeroes the call's counters.  With a router
+// weight, every CTA also bounds the squared L2 norms of its share of the router rows (one
+// warp per row): the FP32 sum of H squares lies within a relative H * 2^-24 of the exact
+// value and is scaled up by (1 + 2^-8) (H <= 2^16), so it is an upper bound; the CTA's
+// maximum goes to wpart[blockIdx.x].  Consumers take the maximum over the grid's entries
+// (no atomics, so nothing needs zeroing first).
+__global__ void __launch_bounds__(256) prep_kernel(int* __restrict__ counters, int n, const bf16* __restrict__ wr,
+                                                   int E, int H, float* __restrict__ wpart) {
+    const int tid = threadIdx.x, lane = tid & 31;
+    if (blockIdx.x == 0)
+        for (int i = tid; i < n; i += blockDim.x) counters[i] = 0;
+    if (wr) {
+        __shared__ float s_max[8];
+        float m = 0.0f;
+        const int nw = (gridDim.x * blockDim.x) >> 5;
+        for (int e = (blockIdx.x * blockDim.x + tid) >> 5; e < E; e += nw) {
+            const bf16* row = wr + (size_t)e * H;
+            float ss = 0.0f;
+            for (int c = lane; c < (H >> 3); c += 32) {
+                const uint4 v = ld_nc16(row + (size_t)c * 8);
+                ss = dot8(v, v, ss);
+            }
+            m = fmaxf(m, warp_sum(ss) * (1.0f + 0x1p-8f));
+        }
+        if (lane == 0) s_max[tid >> 5] = m;
+        __syncthreads();
+        if (tid == 0) {
+            for (int w = 1; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, s_max[w]);
+            wpart[blockIdx.x] = m;
+        }
+    }
+    pdl_trigger();
+}
+
+int prep_grid(int E, int num_sms) { return std::max(1, std::min(num_sms, cdiv(E, 8))); }
+
+cudaError_t launch_prep(int* counters, int n, const bf16* wr, int E, int H, float* wpart, int num_sms,
+                        cudaStream_t s) {
+    return launch_k(prep_kernel, dim3(prep_grid(E, num_sms)), dim3(256), 0, s, false, counters, n, wr, E, H, wpart);
+}
+
+// Upper bound of max_e |Wr[e]|_2^2 from the prep kernel's per-CTA maxima (warp-collective).
+__device__ __forceinline__ float wnorm2_max(const float* __restrict__ wpart, int n, int lane) {
+    float m = 0.0f;
+    for (int i = lane; i < n; i += 32) m = fmaxf(m, wpart[i]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    return m;
+}
+
 // ---------------------------------------------------------------- top-k, one warp per row
 static constexpr int kTopkRowsPerBlock = 4;  // small blocks: the SM fills up to its register limit
 
@@ -67,7 +118,7 @@ __global__ void __launch_bounds__(32 * kTopkRowsPerBlock) topk_kernel(const void
                                                    int32_t* __restrict__ src_idx, float* __restrict__ w_copy,
                                                    int32_t* __restrict__ id_copy, const bf16* __restrict__ x,
                                                    const bf16* __restrict__ wr, int H, float* logits_rw,
-                                                   const float* __restrict__ wnorm2, int* err,
+                                                   const float* __restrict__ wpart, int nwpart, int* err,
                                                    int* __restrict__ counts, const GateArgs gate) {
     __shared__ float s_wbuf[kTopkRowsPerBlock][32];
     pdl_wait();
@@ -84,7 +135,7 @@ __global__ void __launch_bounds__(32 * kTopkRowsPerBlock) topk_kernel(const void
         float w, lg;
         if (REFINE) {
             const bf16* xr = x + (size_t)row * H;
-            const float eps = tc_logit_bound(xr, H, *wnorm2, lane);
+            const float eps = tc_logit_bound(xr, H, wnorm2_max(wpart, nwpart, lane), lane);
             const RowRefine rf{xr, wr, H, E, row, lane, logits_rw, eps, err};
             warp_route_row<V>(l, E, K, score, bias, renorm, lane, eps, rf, wbuf, id, w, lg);
         } else {
@@ -115,20 +166,21 @@ cudaError_t launch_topk(const void* logits, bool bf16_in, int M, int E, int K, i
     const bf16* wr = refine ? refine->wr : nullptr;
     const int H = refine ? refine->H : 0;
     float* lrw = refine ? refine->logits_rw : nullptr;
-    const float* wn2 = refine ? refine->wnorm2 : nullptr;
+    const float* wn2 = refine ? refine->wpart : nullptr;
+    const int nwp = refine ? refine->nwpart : 0;
     int* err = refine ? refine->err : nullptr;
 #define MOE_L(VV)                                                                                              \
     if (v == VV) {                                                                                             \
         if (refine)                                                                                            \
             return launch_k(topk_kernel<VV, false, true>, grid, block, 0, s, pdl, logits, M, E, K, score, bias, \
-                            renorm, topk_w, topk_ids, src_idx, w_copy, id_copy, x, wr, H, lrw, wn2, err,       \
+                            renorm, topk_w, topk_ids, src_idx, w_copy, id_copy, x, wr, H, lrw, wn2, nwp, err,  \
                             counts, gate);                                                                     \
         return bf16_in ? launch_k(topk_kernel<VV, true, false>, grid, block, 0, s, pdl, logits, M, E, K, score, \
                                   bias, renorm, topk_w, topk_ids, src_idx, w_copy, id_copy, x, wr, H, lrw, wn2, \
-                                  err, counts, gate)                                                           \
+                                  nwp, err, counts, gate)                                                           \
                        : launch_k(topk_kernel<VV, false, false>, grid, block, 0, s, pdl, logits, M, E, K, score, \
                                   bias, renorm, topk_w, topk_ids, src_idx, w_copy, id_copy, x, wr, H, lrw, wn2, \
-                                  err, counts, gate);                                                          \
+                                  nwp, err, counts, gate);                                                          \
     }
     MOE_L(1) MOE_L(2) MOE_L(4) MOE_L(8) MOE_L(16) MOE_L(32)
 #undef MOE_L
@@ -155,7 +207,8 @@ __global__ void __launch_bounds__(32 * kTopkRowsPerBlock) topk_screen_kernel(con
                                                                               const float* __restrict__ bias,
                                                                               const CandList cl,
                                                                               const bf16* __restrict__ x, int H,
-                                                                              const float* __restrict__ wnorm2) {
+                                                                              const float* __restrict__ wpart,
+                                                                              int nwpart) {
     pdl_wait();
     const int lane = threadIdx.x & 31;
     const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -163,7 +216,7 @@ __global__ void __launch_bounds__(32 * kTopkRowsPerBlock) topk_screen_kernel(con
         const bool sig = score == MOE_SCORE_SIGMOID;
         float l[V], key[V];
         load_row_f32<V>(logits + (size_t)row * E, E, lane, l);
-        const float eps = tc_logit_bound(x + (size_t)row * H, H, *wnorm2, lane);
+        const float eps = tc_logit_bound(x + (size_t)row * H, H, wnorm2_max(wpart, nwpart, lane), lane);
         if (lane == 0) cl.row_eps[row] = eps;
         screening_keys<V>(l, key, E, sig, bias, lane);
         float kth, ua, ub;
@@ -312,7 +365,7 @@ cudaError_t launch_topk_split(const float* logits, int M, int E, int K, int scor
 #define MOE_S(VV)                                                                                           \
     if (v == VV)                                                                                            \
         st = launch_k(topk_screen_kernel<VV>, grid, block, 0, s, pdl, logits, M, E, K, score, bias, cl, ra.x, \
-                      ra.H, ra.wnorm2);
+                      ra.H, ra.wpart, ra.nwpart);
     MOE_S(1) MOE_S(2) MOE_S(4) MOE_S(8) MOE_S(16) MOE_S(32)
 #undef MOE_S
     if (st != cudaSuccess) return st;

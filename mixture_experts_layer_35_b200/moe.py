@@ -67,7 +67,7 @@ _lib.moe_fused_forward_timed.argtypes = [ctypes.POINTER(LayerDesc), _vp, _vp, _v
 _lib.moe_fused_forward_timed.restype = _ci
 _lib.moe_fused_forward_noalloc.argtypes = [ctypes.POINTER(LayerDesc), _vp, _vp, _vp, _vp, _vp, _vp]
 _lib.moe_fused_forward_noalloc.restype = _ci
-NOALLOC_SCRATCH_BYTES = 4 << 20  # MOE_NOALLOC_SCRATCH_BYTES
+NOALLOC_SCRATCH_BYTES = 16 << 20  # MOE_NOALLOC_SCRATCH_BYTES
 _lib.moe_noalloc_get_error.argtypes = [ctypes.POINTER(_ci), _vp]
 _lib.moe_noalloc_get_error.restype = _ci
 _lib.moe_get_error.argtypes = [_vp, ctypes.POINTER(_ci), _vp]

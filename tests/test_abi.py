@@ -101,16 +101,16 @@ def test_path_selection_and_launch_counts():
     assert moe.launches(d) == 4
     d = _desc(T=4096)
     assert moe.select_path(d) == "large"
-    assert moe.launches(d) == 6
+    assert moe.launches(d) == 7  # prep, router, top-k, permute, fc1, fc2, finalize
     d = _desc(T=4096, E=512, top_k=10)
-    assert moe.launches(d) == 8  # router, top-k in three kernels, permute, fc1, fc2, finalize
+    assert moe.launches(d) == 9  # prep, router, top-k in three kernels, permute, fc1, fc2, finalize
     d = _desc(T=4096, E=512, top_k=10, score="softmax", renorm=False)
-    assert moe.launches(d) == 6  # full softmax keeps the one-kernel top-k
+    assert moe.launches(d) == 7  # full softmax keeps the one-kernel top-k
     d = _desc(T=4, path="large")
     assert moe.select_path(d) == "large"
-    assert moe.launches(d) == 6
+    assert moe.launches(d) == 7
     d.router_logits = FAKE * 8
-    assert moe.launches(d) == 5  # logits given: no router launch
+    assert moe.launches(d) == 6  # logits given: no router launch
     d = _desc(T=64, path="small")
     assert moe.select_path(d) == "small"
     assert _fwd(d, ws=FAKE * 8, ws_bytes=moe.workspace_size(d)) == moe.MOE_ERR_UNSUPPORTED
