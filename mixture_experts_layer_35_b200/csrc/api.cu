@@ -519,7 +519,13 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
     g1.hs = hs;
     g1.zero_ptr = acc;
     g1.zero_n = (size_t)T * H * (Is ? 2 : 1);
-    g1.streamk_max = gemm_streamk_max(fc1_mode, bn1, sms);
+    // Upper bound of a grouped GEMM's tiles: at most min(E, T*K) experts have rows, and each
+    // expert's token tiles add at most one beyond its share of T*K / bn; plus the shared group.
+    auto max_tiles = [&](int bn, int nf_r, int nf_s) {
+        const long long TK = (long long)T * K;
+        return (long long)nf_r * (std::min<long long>(E, TK) + TK / bn) + (long long)nf_s * cdiv(T, bn);
+    };
+    g1.streamk_max = gemm_streamk_max(fc1_mode, bn1, sms, max_tiles(bn1, g1.nfeat_r, Is ? g1.nfeat_s : 0));
     g1.skp = reinterpret_cast<float*>(w8 + L.skp);
     g1.done = counts + done_int(E);
     g1.err = err;
@@ -549,7 +555,7 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
     g2.sgate = gate;
     g2.zero_ptr = nullptr;
     g2.zero_n = 0;
-    g2.streamk_max = gemm_streamk_max(GM_FC2, bn2, sms);
+    g2.streamk_max = gemm_streamk_max(GM_FC2, bn2, sms, max_tiles(bn2, g2.nfeat_r, Is ? g2.nfeat_s : 0));
     g2.skp = nullptr;
     g2.done = nullptr;
     if (!mark()) return MOE_ERR_CUDA;

@@ -222,11 +222,15 @@ struct WorkWalk {
     __device__ bool active(int c) const { return lo_of(c) < lo_of(c + 1); }
 };
 
-template <int MODE, int BN>
+// SK: the stream-K variant (the host launches it for calls with few tiles per SM); the
+// other variant deals whole tiles only, and compiles without the stream-K bookkeeping.
+template <int MODE, int BN, bool SK>
 __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
     gemm_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ CUtensorMap tm_a_s,
                 const __grid_constant__ CUtensorMap tm_b_r, const __grid_constant__ CUtensorMap tm_b_s) {
     using C = Cfg<MODE, BN>;
+    // FC1's stream-K fix-up keeps [kNA][BN][128] partial sums per CTA: BN <= 64 only.
+    constexpr bool kFix = SK && C::kGather && BN <= kStreamKMaxBN;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_u32 = smem_u32(smem_raw);
     const uint32_t base_u32 = (raw_u32 + 1023u) & ~1023u;
@@ -281,7 +285,7 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
     const uint32_t tmem_base = *tmem_slot;
     const int total = a.dense ? a.nfeat_r * cdiv(a.T, kDenseTokenTile) : s_tiles[G];
     const int routed_tiles = (a.dense || !a.has_shared) ? total : s_tiles[a.E];
-    const bool streamk = total > 0 && total < a.streamk_max;
+    const bool streamk = SK && total > 0 && total < a.streamk_max;
     const int nk_r = cdiv(a.kdim, BK), nk_s = cdiv(a.kdim_s > 0 ? a.kdim_s : a.kdim, BK);
     // Round-robin dealing keeps the CTAs on neighbouring tiles of the group-major list (one
     // expert's feature and token tiles), which share that expert's weight and token rows in
@@ -441,7 +445,7 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
             const int feat = ti.shared ? a.feat_s : a.feat_r;
             const bool fok = f < feat;
             const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * C::kAccStride);
-            if (C::kGather && sg.kind == kPart) {
+            if (kFix && sg.kind == kPart) {
                 // ---- stream-K, FC1: a later k-block range; its partial sums go to this CTA's
                 // slot, then the tile's counter tells the fixer it is there.
                 float* slot = a.skp + (size_t)blockIdx.x * kSlotFloats;
@@ -475,7 +479,7 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
                 continue;
             }
             int ncontrib = 0;
-            if (C::kGather && sg.kind == kFixer) {
+            if (kFix && sg.kind == kFixer) {
                 // ---- stream-K, FC1: this CTA holds the tile's first k-blocks.  Each warp waits
                 // (bounded) until every warp of every later range has published its partial,
                 // then adds them below.
@@ -514,7 +518,7 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
                 uint32_t u[32];
                 if (C::kSwiglu) tmem_ld32(tb + C::kBN + c0, u);
                 tmem_ld_wait();
-                if (C::kGather && ncontrib > 0) {  // the later ranges' partial sums, in CTA order
+                if (kFix && ncontrib > 0) {  // the later ranges' partial sums, in CTA order
                     for (int c = blockIdx.x + 1; c <= sg.last; ++c) {
                         if (!work.active(c)) continue;
                         const float* slot = a.skp + (size_t)c * kSlotFloats;
@@ -719,14 +723,22 @@ __global__ void __launch_bounds__(256) finalize_kernel(const float* __restrict__
 
 }  // namespace
 
-template <int MODE, int BN>
-static cudaError_t launch_mode(const GemmArgs& a, const GemmMaps& m, int grid, cudaStream_t s, bool pdl) {
+template <int MODE, int BN, bool SK>
+static cudaError_t launch_mode_sk(const GemmArgs& a, const GemmMaps& m, int grid, cudaStream_t s, bool pdl) {
     using C = Cfg<MODE, BN>;
     cudaError_t e =
-        cudaFuncSetAttribute(gemm_kernel<MODE, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
+        cudaFuncSetAttribute(gemm_kernel<MODE, BN, SK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
     if (e != cudaSuccess) return e;
-    return launch_k(gemm_kernel<MODE, BN>, dim3(grid), dim3(C::kThreads), C::kSmem, s, pdl, a, m.a_r, m.a_s, m.b_r,
-                    m.b_s);
+    return launch_k(gemm_kernel<MODE, BN, SK>, dim3(grid), dim3(C::kThreads), C::kSmem, s, pdl, a, m.a_r, m.a_s,
+                    m.b_r, m.b_s);
+}
+// The stream-K variant exists for the token tiles of few-token calls (32 and 64 rows for
+// FC1, 32 and 128 for FC2); a.streamk_max == 0 selects the whole-tile variant.
+template <int MODE, int BN>
+static cudaError_t launch_mode(const GemmArgs& a, const GemmMaps& m, int grid, cudaStream_t s, bool pdl) {
+    constexpr bool kHasSK = MODE == GM_FC2 ? (BN == 32 || BN == 128) : (MODE != GM_DENSE && BN <= kStreamKMaxBN);
+    if (kHasSK && a.streamk_max > 0) return launch_mode_sk<MODE, BN, kHasSK>(a, m, grid, s, pdl);
+    return launch_mode_sk<MODE, BN, false>(a, m, grid, s, pdl);
 }
 
 int gemm_token_tile(int mode, int T, int K, int E) {
@@ -784,10 +796,15 @@ size_t fc1_streamk_bytes(int bn, bool swiglu, int grid) {
     return (size_t)grid * (swiglu ? 2 : 1) * bn * BM * sizeof(float);
 }
 
-int gemm_streamk_max(int mode, int bn, int grid) {
+int gemm_streamk_max(int mode, int bn, int grid, long long max_tiles) {
     if (mode == GM_DENSE) return 0;
-    if (mode == GM_FC2) return kStreamKWaves * grid;
-    return bn <= kStreamKMaxBN ? std::min(kStreamKWaves * grid, kStreamKMaxTiles) : 0;
+    if (mode == GM_FC2) {
+        if (bn != 32 && bn != 128) return 0;
+    } else if (bn > kStreamKMaxBN) {
+        return 0;
+    }
+    const int limit = mode == GM_FC2 ? kStreamKWaves * grid : std::min(kStreamKWaves * grid, kStreamKMaxTiles);
+    return max_tiles < limit ? limit : 0;  // the call can have fewer tiles than the limit
 }
 
 }  // namespace moe

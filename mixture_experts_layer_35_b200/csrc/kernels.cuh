@@ -200,7 +200,8 @@ static constexpr int kStreamKMaxTiles = 1024;
 static constexpr int kStreamKMaxBN = 64;
 // Bytes of FC1's stream-K partial-sum slots for `grid` CTAs (0 when FC1 cannot use it).
 size_t fc1_streamk_bytes(int bn, bool swiglu, int grid);
-int gemm_streamk_max(int mode, int bn, int grid);
+// Stream-K tile limit for a call whose tile count is at most max_tiles (0: whole tiles).
+int gemm_streamk_max(int mode, int bn, int grid, long long max_tiles);
 
 // finalize: out = bf16(bf16(scale * acc) + shared) with shared = bf16(acc_s) (internal
 // shared expert) or sh_out (caller's), or bf16(scale * acc) without one.  out may equal

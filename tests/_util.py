@@ -13,9 +13,10 @@ OUT_MEAN_REL = 1e-3
 W_REL = 1e-6
 
 
-def device_layer(shape, T, seed=0, routing="router", device="cuda", x_mode="normal"):
-    """Inputs drawn on the device (fast for full-size weights)."""
-    return inp_mod.make_layer(shape, T, seed=seed, device=device, routing=routing, x_mode=x_mode)
+def device_layer(shape, T, seed=0, routing="router", device="cuda", **kw):
+    """Inputs drawn on the device (fast for full-size weights); ``kw``: the generator's
+    x_mode / shared_gate / shared_out options."""
+    return inp_mod.make_layer(shape, T, seed=seed, device=device, routing=routing, **kw)
 
 
 def host_copy(d):
