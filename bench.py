@@ -209,7 +209,8 @@ def kernel_names(path: str, router: bool, launches: int = 0):
     names = ["router"] if router else []
     if path == "small":
         return names + ["route", "fc1", "fc2"]
-    names = ["prep"] + names
+    if launches in (len(names) + 6, len(names) + 8) or not router:  # a prep kernel leads
+        names = ["prep"] + names
     if launches == len(names) + 7:  # top-k after the tensor-core router: screen, refine, final
         return names + ["topk", "refine", "select", "permute", "fc1", "fc2", "finalize"]
     return names + ["topk", "permute", "fc1", "fc2", "finalize"]

@@ -307,12 +307,17 @@ static bool split_topk_mode(const moe_layer_desc* d) {
     return d->E > 256 && (d->score == MOE_SCORE_SIGMOID || d->renorm);
 }
 
+// The many-token path's prep kernel runs before the tensor-core router and when the
+// logits are given; the few-token router zeroes the counters itself.
+static bool prep_kernel_for(const moe_layer_desc* d) { return d->router_logits || dense_router_for(d); }
+
 int moe_fused_forward_launches(const moe_layer_desc* d) {
     if (validate_desc(d) != MOE_OK || d->T == 0) return 0;
     const int router = d->router_logits ? 0 : 1;
     if (resolve_path(d) == MOE_PATH_SMALL) return router + 3;  // route table, fc1, fc2
-    if (dense_router_for(d) && split_topk_mode(d)) return router + 8;  // prep, screen, refine, final, ...
-    return router + 6;                                          // prep, topk, permute, fc1, fc2, finalize
+    const int prep = prep_kernel_for(d) ? 1 : 0;
+    if (dense_router_for(d) && split_topk_mode(d)) return prep + router + 7;  // screen, refine, final, ...
+    return prep + router + 5;                                   // topk, permute, fc1, fc2, finalize
 }
 
 static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, void* out_, float* topk_w_out,
@@ -358,7 +363,7 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
     const bool dense_router = path == MOE_PATH_LARGE && dense_router_for(d);
     float* wpart = reinterpret_cast<float*>(w8 + L.wpart);
     bool pdl = false;
-    if (path == MOE_PATH_LARGE) {
+    if (path == MOE_PATH_LARGE && prep_kernel_for(d)) {
         if (!mark()) return MOE_ERR_CUDA;
         MOE_CK(launch_prep(reinterpret_cast<int*>(w8 + L.counts), (int)counter_ints(E),
                            dense_router ? static_cast<const bf16*>(d->router_w) : nullptr, E, H, wpart, sms, s));
@@ -372,7 +377,10 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
         float* lg = logits_out ? logits_out : reinterpret_cast<float*>(w8 + L.logits);
         if (!mark()) return MOE_ERR_CUDA;
         if (!dense_router && T <= 64 && router_small_supported(H)) {
-            MOE_CK(launch_router_small(x, static_cast<const bf16*>(d->router_w), T, H, E, lg, nullptr, err, s, pdl));
+            // the many-token path without a prep kernel: this first kernel zeroes the counters
+            int* zc = path == MOE_PATH_LARGE ? reinterpret_cast<int*>(w8 + L.counts) : nullptr;
+            MOE_CK(launch_router_small(x, static_cast<const bf16*>(d->router_w), T, H, E, lg, nullptr, err, s, pdl,
+                                       zc, zc ? (int)counter_ints(E) : 0));
         } else {
             st = run_router_dense(d, x, lg, nullptr, sms, s, err, pdl);
             if (st != MOE_OK) return st;

@@ -98,6 +98,10 @@ struct Cfg {
     // dynamic smem: alignment slack, stages, barriers, flags, tile and offset tables
     static constexpr size_t kSmem = 1024 + (size_t)kStages * kStageBytes + kEpiBytes + kMeta;
     static constexpr int kLag = (kStages - 2) < kLagMax ? (kStages - 2) : kLagMax;
+    // Weight k-blocks prefetched into L2 ahead of the load that uses them (the producer).
+    // Eight blocks of weights (128 or 256 KB per SM) keep each SM's share of the stream in
+    // flight without crowding the activations and accumulator out of L2.
+    static constexpr int kPrefetch = 8;
     static_assert(kStages >= 3, "ring too shallow");
     static_assert(kGather || kBN % b_box_rows<MODE>() == 0, "a tile's boxes must fit its stage");
     static_assert(8 * (2 * kStages + 4) + 8 <= 256, "barrier block");
@@ -298,6 +302,33 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             const uint64_t wpol = l2_policy_evict_first();
+            // Weight tiles are also prefetched into L2 kPrefetch k-blocks ahead of the ring: a
+            // stage's round trip from HBM takes several microseconds under load, and the
+            // ring alone (its stages / that latency) caps an SM's weight stream well below
+            // its share of HBM bandwidth.  A second walker runs ahead over the same work.
+            WorkWalk ahead = work;
+            Seg sa;
+            TileInfo tia;
+            int a_kb = 0, a_end = 0;
+            auto prefetch_next = [&]() {
+                while (a_kb >= a_end) {
+                    if (!ahead.next(sa)) return;
+                    tia = decode_tile<C::kBN>(a, s_tiles, s_offs, G, sa.tile);
+                    a_kb = sa.kb0;
+                    a_end = tia.nk == 0 ? sa.kb0 : sa.kb1;
+                }
+                const int fr = tia.ft * BM;
+                if (tia.shared || a.dense) {
+                    const CUtensorMap* t = tia.shared ? &tm_a_s : &tm_a_r;
+                    tma_prefetch_l2_2d(t, a_kb * BK, fr);
+                    if (C::kSwiglu) tma_prefetch_l2_2d(t, a_kb * BK, a.up_s + fr);
+                } else {
+                    tma_prefetch_l2_3d(&tm_a_r, a_kb * BK, fr, tia.g);
+                    if (C::kSwiglu) tma_prefetch_l2_3d(&tm_a_r, a_kb * BK, a.up_r + fr, tia.g);
+                }
+                ++a_kb;
+            };
+            for (int d = 0; d < C::kPrefetch; ++d) prefetch_next();
             int it = 0;
             while (!*abort_flag && work.next(sg)) {
                 const TileInfo ti = decode_tile<C::kBN>(a, s_tiles, s_offs, G, sg.tile);
@@ -340,6 +371,7 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
                             tma_load_2d(bs + (uint32_t)q * (BBOX * BK * 2), tb, full_bar(s), kb * BK,
                                         ti.row0 + q * BBOX);
                     }
+                    prefetch_next();
                 }
                 if (!ok) break;
             }

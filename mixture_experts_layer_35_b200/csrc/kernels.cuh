@@ -66,8 +66,10 @@ cudaError_t launch_topk_split(const float* logits, int M, int E, int K, int scor
                               const RefineArgs& ra, int* counts, int* err, int num_sms, cudaStream_t s, bool pdl,
                               const std::function<bool()>* mark, const GateArgs& gate);
 bool router_small_supported(int H);
+// zero_ints (optional, n_zero ints): counters the kernel zeroes as a call's first kernel.
 cudaError_t launch_router_small(const bf16* x, const bf16* wr, int T, int H, int E, float* logits,
-                                float* logits_copy, int* err, cudaStream_t s, bool pdl);
+                                float* logits_copy, int* err, cudaStream_t s, bool pdl, int* zero_ints = nullptr,
+                                int n_zero = 0);
 
 // ---------------------------------------------------------------- few-token path
 static constexpr int kSmallMaxT = 16;

@@ -397,11 +397,15 @@ static constexpr int kRouterTokBlock = 4;
 template <int VH>
 __global__ void __launch_bounds__(64) router_logits_small(const bf16* __restrict__ x, const bf16* __restrict__ wr,
                                                           int T, int H, int E, float* __restrict__ logits,
-                                                          float* __restrict__ logits_copy, int* err) {
+                                                          float* __restrict__ logits_copy, int* err,
+                                                          int* __restrict__ zero_ints, int n_zero) {
     extern __shared__ uint4 xs[];  // [kRouterTokBlock][H / 8]
     __shared__ __align__(8) uint64_t s_bar;
     __shared__ int s_abort;
     const int tid = threadIdx.x, lane = tid & 31;
+    // As the first kernel of a many-token call, CTA (0, 0) also zeroes the call's counters.
+    if (zero_ints && blockIdx.x == 0 && blockIdx.y == 0)
+        for (int i = tid; i < n_zero; i += blockDim.x) zero_ints[i] = 0;
     const uint32_t bar = smem_u32(&s_bar);
     if (tid == 0) {
         mbar_init(bar, 1);
@@ -468,7 +472,7 @@ __global__ void __launch_bounds__(64) router_logits_small(const bf16* __restrict
 bool router_small_supported(int H) { return (H >> 3) <= 32 * 16; }
 
 cudaError_t launch_router_small(const bf16* x, const bf16* wr, int T, int H, int E, float* logits,
-                                float* logits_copy, int* err, cudaStream_t s, bool pdl) {
+                                float* logits_copy, int* err, cudaStream_t s, bool pdl, int* zero_ints, int n_zero) {
     dim3 grid(cdiv(E, 2), cdiv(T, kRouterTokBlock)), block(64);
     const size_t smem = (size_t)kRouterTokBlock * H * 2;
     const int need = cdiv(H >> 3, 32);
@@ -477,7 +481,8 @@ cudaError_t launch_router_small(const bf16* x, const bf16* wr, int T, int H, int
         cudaError_t st = cudaFuncSetAttribute(router_logits_small<VV>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
                                                (int)smem);                                                       \
         if (st != cudaSuccess) return st;                                                                        \
-        return launch_k(router_logits_small<VV>, grid, block, smem, s, pdl, x, wr, T, H, E, logits, logits_copy, err); \
+        return launch_k(router_logits_small<VV>, grid, block, smem, s, pdl, x, wr, T, H, E, logits, logits_copy, err, \
+                        zero_ints, n_zero);                                                                      \
     }
     MOE_R(4) MOE_R(8) MOE_R(12) MOE_R(16)
 #undef MOE_R

@@ -108,9 +108,9 @@ def test_path_selection_and_launch_counts():
     assert moe.launches(d) == 7  # full softmax keeps the one-kernel top-k
     d = _desc(T=4, path="large")
     assert moe.select_path(d) == "large"
-    assert moe.launches(d) == 7
+    assert moe.launches(d) == 6  # few-token router (it zeroes the counters), top-k, permute, fc1, fc2, finalize
     d.router_logits = FAKE * 8
-    assert moe.launches(d) == 6  # logits given: no router launch
+    assert moe.launches(d) == 6  # logits given: prep, no router launch
     d = _desc(T=64, path="small")
     assert moe.select_path(d) == "small"
     assert _fwd(d, ws=FAKE * 8, ws_bytes=moe.workspace_size(d)) == moe.MOE_ERR_UNSUPPORTED

@@ -41,6 +41,7 @@ def test_kernel_names_follow_launch_order():
     assert bench.kernel_names("large", True, 9) == ["prep", "router", "topk", "refine", "select", "permute", "fc1",
                                                     "fc2", "finalize"]
     assert bench.kernel_names("large", True, 7) == ["prep", "router", "topk", "permute", "fc1", "fc2", "finalize"]
+    assert bench.kernel_names("large", True, 6) == ["router", "topk", "permute", "fc1", "fc2", "finalize"]
     assert bench.kernel_names("large", False, 6) == ["prep", "topk", "permute", "fc1", "fc2", "finalize"]
     assert bench.kernel_names("large", False) == ["prep", "topk", "permute", "fc1", "fc2", "finalize"]
 
