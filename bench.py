@@ -202,20 +202,6 @@ def accounting(shape, T: int, U: int, router: bool, Is: int):
     return {"layer": {"bytes": layer_bytes, "flops": layer_flops}, "kernels": k}
 
 
-def kernel_names(path: str, router: bool, launches: int = 0):
-    """Names of a forward's kernels in launch order: the streaming path's route table,
-    the three-kernel top-k after the tensor-core router (more than 256 experts), or the
-    one-kernel top-k + permute of the other cases."""
-    names = ["router"] if router else []
-    if path == "small":
-        return names + ["route", "fc1", "fc2"]
-    if launches in (len(names) + 6, len(names) + 8) or not router:  # a prep kernel leads
-        names = ["prep"] + names
-    if launches == len(names) + 7:  # top-k after the tensor-core router: screen, refine, final
-        return names + ["topk", "refine", "select", "permute", "fc1", "fc2", "finalize"]
-    return names + ["topk", "permute", "fc1", "fc2", "finalize"]
-
-
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu
 # capture of the default workload (seed 0, one GPU), keyed by (config, T, routing, kernel).
 # The capture and its command are summarised in profiles/; an entry is removed whenever
@@ -466,7 +452,7 @@ def run_ours(args, rank, local, world):
     router = b.logits is None
     acc = accounting(shape, args.T, U, router, b.Is)
     kt = b.per_kernel(max(3, min(args.steps, 10)))
-    names = kernel_names(b.path, router, b.launches)
+    names = b.moe.kernel_plan(b.desc)
     dom = int(np.argmax(kt))
     dom_name = names[dom]
     roof = roofline_of(acc["kernels"][dom_name], kt[dom] / 1e3, peaks)

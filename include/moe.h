@@ -189,6 +189,19 @@ moe_status_t moe_fused_forward(const moe_layer_desc* d, const void* x, void* out
 /* Number of kernels moe_fused_forward enqueues for this description (for accounting). */
 int moe_fused_forward_launches(const moe_layer_desc* d);
 
+/* The kernels moe_fused_forward enqueues for this description, in launch order: writes up
+ * to max_kernels MOE_K_* values to `kernels` (may be NULL) and returns their number (0
+ * for an invalid description or T == 0).  The path, the router used and the folding of
+ * the finalize into FC2 (few tokens) decide the list. */
+enum { MOE_K_PREP = 0,        /* zero the call's counters; bound the router rows' norms */
+       MOE_K_ROUTER = 1,      /* router logits */
+       MOE_K_ROUTE_TABLE = 2, /* few-token path: routing and the distinct-expert table */
+       MOE_K_TOPK = 3,        /* top-k (screening, exact re-evaluation, selection), or its screen */
+       MOE_K_TOPK_REFINE = 4, /* split top-k: exact re-evaluation of the candidates */
+       MOE_K_TOPK_SELECT = 5, /* split top-k: selection on exact keys */
+       MOE_K_PERMUTE = 6, MOE_K_FC1 = 7, MOE_K_FC2 = 8, MOE_K_FINALIZE = 9 };
+int moe_fused_forward_plan(const moe_layer_desc* d, int* kernels, int max_kernels);
+
 /* Token rows per tile of the many-token path's grouped GEMMs for this description (the
  * MMA N of one tile: FC1 and FC2 each pick one width per call from T * top_k / E).
  * Returns MOE_OK, or the description's validation error. */

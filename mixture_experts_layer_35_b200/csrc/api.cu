@@ -27,10 +27,18 @@ struct WsLayout {
 };
 // Candidate-list capacity per token of the three-kernel top-k (rows with more fall back).
 constexpr size_t kCandPerRow = 32;
-// Counters zeroed at the start of each many-token call (prep kernel): per-expert counts,
-// per-expert cursors, the candidate count, then FC1's stream-K per-tile counters.
-inline size_t counter_ints(size_t E) { return 2 * (E + 2) + 4 + kStreamKMaxTiles; }
+// Counters zeroed at the start of each many-token call (by its first kernel): per-expert
+// counts, per-expert cursors, the candidate count, FC1's stream-K per-tile counters, then
+// the per-feature-block counters of FC2's folded finalize.
+constexpr int kFinMaxBlocks = 64;  // H <= 8192
+inline size_t counter_ints(size_t E) { return 2 * (E + 2) + 4 + kStreamKMaxTiles + kFinMaxBlocks; }
 inline size_t done_int(size_t E) { return 2 * (E + 2) + 4; }
+inline size_t fin_int(size_t E) { return done_int(E) + kStreamKMaxTiles; }
+// Few tokens: FC2's last warp per 128-feature block writes the output (no finalize launch).
+constexpr int kFoldFinalizeMaxT = 64;
+inline bool fold_finalize(const moe_layer_desc* d) {
+    return d->T <= kFoldFinalizeMaxT && (d->H + 127) / 128 <= kFinMaxBlocks;
+}
 inline size_t cand_count_int(size_t E) { return 2 * (E + 2); }
 // Per-CTA router weight-norm bounds of the prep kernel (its grid is at most E / 8 <= 128).
 constexpr size_t kMaxPrepGrid = (MOE_MAX_EXPERTS + 7) / 8;
@@ -311,14 +319,32 @@ static bool split_topk_mode(const moe_layer_desc* d) {
 // logits are given; the few-token router zeroes the counters itself.
 static bool prep_kernel_for(const moe_layer_desc* d) { return d->router_logits || dense_router_for(d); }
 
-int moe_fused_forward_launches(const moe_layer_desc* d) {
+int moe_fused_forward_plan(const moe_layer_desc* d, int* kernels, int max_kernels) {
     if (validate_desc(d) != MOE_OK || d->T == 0) return 0;
-    const int router = d->router_logits ? 0 : 1;
-    if (resolve_path(d) == MOE_PATH_SMALL) return router + 3;  // route table, fc1, fc2
-    const int prep = prep_kernel_for(d) ? 1 : 0;
-    if (dense_router_for(d) && split_topk_mode(d)) return prep + router + 7;  // screen, refine, final, ...
-    return prep + router + 5;                                   // topk, permute, fc1, fc2, finalize
+    int k[16], n = 0;
+    if (resolve_path(d) == MOE_PATH_SMALL) {
+        if (!d->router_logits) k[n++] = MOE_K_ROUTER;
+        k[n++] = MOE_K_ROUTE_TABLE;
+        k[n++] = MOE_K_FC1;
+        k[n++] = MOE_K_FC2;
+    } else {
+        if (prep_kernel_for(d)) k[n++] = MOE_K_PREP;
+        if (!d->router_logits) k[n++] = MOE_K_ROUTER;
+        k[n++] = MOE_K_TOPK;
+        if (dense_router_for(d) && split_topk_mode(d)) {
+            k[n++] = MOE_K_TOPK_REFINE;
+            k[n++] = MOE_K_TOPK_SELECT;
+        }
+        k[n++] = MOE_K_PERMUTE;
+        k[n++] = MOE_K_FC1;
+        k[n++] = MOE_K_FC2;
+        if (!fold_finalize(d)) k[n++] = MOE_K_FINALIZE;
+    }
+    for (int i = 0; kernels && i < n && i < max_kernels; ++i) kernels[i] = k[i];
+    return n;
 }
+
+int moe_fused_forward_launches(const moe_layer_desc* d) { return moe_fused_forward_plan(d, nullptr, 0); }
 
 static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, void* out_, float* topk_w_out,
                                        int32_t* topk_ids_out, float* logits_out, void* ws, size_t ws_bytes,
@@ -566,12 +592,19 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
     g2.streamk_max = gemm_streamk_max(GM_FC2, bn2, sms, max_tiles(bn2, g2.nfeat_r, Is ? g2.nfeat_s : 0));
     g2.skp = nullptr;
     g2.done = nullptr;
+    const bool fold = fold_finalize(d);
+    g2.fin_out = fold ? out : nullptr;
+    g2.fin_sh = fold ? sh_out : nullptr;
+    g2.fin_scale = rscale;
+    g2.fin_cnt = counts + fin_int(E);
     if (!mark()) return MOE_ERR_CUDA;
     MOE_CK(launch_gemm(GM_FC2, bn2, g2, m2, sms, s, chain));
 
-    // 6. finalize
-    if (!mark()) return MOE_ERR_CUDA;
-    MOE_CK(launch_finalize(acc, acc_s, sh_out, out, (size_t)T * H, rscale, sms, s, chain));
+    // 6. finalize (folded into FC2 for few tokens)
+    if (!fold) {
+        if (!mark()) return MOE_ERR_CUDA;
+        MOE_CK(launch_finalize(acc, acc_s, sh_out, out, (size_t)T * H, rscale, sms, s, chain));
+    }
     if (!mark()) return MOE_ERR_CUDA;
     return MOE_OK;
 }

@@ -98,10 +98,6 @@ struct Cfg {
     // dynamic smem: alignment slack, stages, barriers, flags, tile and offset tables
     static constexpr size_t kSmem = 1024 + (size_t)kStages * kStageBytes + kEpiBytes + kMeta;
     static constexpr int kLag = (kStages - 2) < kLagMax ? (kStages - 2) : kLagMax;
-    // Weight k-blocks prefetched into L2 ahead of the load that uses them (the producer).
-    // Eight blocks of weights (128 or 256 KB per SM) keep each SM's share of the stream in
-    // flight without crowding the activations and accumulator out of L2.
-    static constexpr int kPrefetch = 8;
     static_assert(kStages >= 3, "ring too shallow");
     static_assert(kGather || kBN % b_box_rows<MODE>() == 0, "a tile's boxes must fit its stage");
     static_assert(8 * (2 * kStages + 4) + 8 <= 256, "barrier block");
@@ -297,38 +293,19 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
     WorkWalk work;
     work.init(total, routed_tiles, nk_r, nk_s, streamk);
     Seg sg;
+    // FC2 with the finalize folded in: every epilogue warp adds the k-blocks of each of its
+    // segments to its feature block's counter; the warp that completes the block's total
+    // (all tiles of that block, all their k-blocks, times the epilogue warps) finalizes it.
+    const int fin_target =
+        (MODE == GM_FC2 && a.fin_out)
+            ? ((routed_tiles / max(1, a.nfeat_r)) * nk_r +
+               (a.has_shared ? ((total - routed_tiles) / max(1, a.nfeat_s)) * nk_s : 0)) * C::kEpiWarps
+            : 0;
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             const uint64_t wpol = l2_policy_evict_first();
-            // Weight tiles are also prefetched into L2 kPrefetch k-blocks ahead of the ring: a
-            // stage's round trip from HBM takes several microseconds under load, and the
-            // ring alone (its stages / that latency) caps an SM's weight stream well below
-            // its share of HBM bandwidth.  A second walker runs ahead over the same work.
-            WorkWalk ahead = work;
-            Seg sa;
-            TileInfo tia;
-            int a_kb = 0, a_end = 0;
-            auto prefetch_next = [&]() {
-                while (a_kb >= a_end) {
-                    if (!ahead.next(sa)) return;
-                    tia = decode_tile<C::kBN>(a, s_tiles, s_offs, G, sa.tile);
-                    a_kb = sa.kb0;
-                    a_end = tia.nk == 0 ? sa.kb0 : sa.kb1;
-                }
-                const int fr = tia.ft * BM;
-                if (tia.shared || a.dense) {
-                    const CUtensorMap* t = tia.shared ? &tm_a_s : &tm_a_r;
-                    tma_prefetch_l2_2d(t, a_kb * BK, fr);
-                    if (C::kSwiglu) tma_prefetch_l2_2d(t, a_kb * BK, a.up_s + fr);
-                } else {
-                    tma_prefetch_l2_3d(&tm_a_r, a_kb * BK, fr, tia.g);
-                    if (C::kSwiglu) tma_prefetch_l2_3d(&tm_a_r, a_kb * BK, a.up_r + fr, tia.g);
-                }
-                ++a_kb;
-            };
-            for (int d = 0; d < C::kPrefetch; ++d) prefetch_next();
             int it = 0;
             while (!*abort_flag && work.next(sg)) {
                 const TileInfo ti = decode_tile<C::kBN>(a, s_tiles, s_offs, G, sg.tile);
@@ -371,7 +348,6 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
                             tma_load_2d(bs + (uint32_t)q * (BBOX * BK * 2), tb, full_bar(s), kb * BK,
                                         ti.row0 + q * BBOX);
                     }
-                    prefetch_next();
                 }
                 if (!ok) break;
             }
@@ -641,6 +617,54 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(tempty_bar(buf));
             ++tcount;
+            if (MODE == GM_FC2 && a.fin_out) {
+                // This warp's reductions for the segment are issued; fence them, count them.
+                __threadfence();
+                __syncwarp();
+                int last = 0;
+                if (lane == 0) {
+                    const int add = sg.kb1 - sg.kb0;
+                    last = atomicAdd(a.fin_cnt + ti.ft, add) + add == fin_target;
+                }
+                last = __shfl_sync(0xffffffffu, last, 0);
+                if (last) {  // every addition into this feature block is done: finalize it
+                    __threadfence();
+                    const int f4 = ti.ft * BM + 4 * lane;  // 4 features per lane
+                    const int H = a.feat_r;
+                    if (f4 < H) {
+                        for (int t = 0; t < a.T; ++t) {
+                            const size_t o = (size_t)t * H + f4;
+                            const float4 r4 = __ldcg(reinterpret_cast<const float4*>(a.acc + o));
+                            float r[4] = {r4.x, r4.y, r4.z, r4.w};
+                            float sv[4] = {0.f, 0.f, 0.f, 0.f};
+                            const bool has_s = a.has_shared || a.fin_sh;
+                            if (a.has_shared) {
+                                const float4 s4 = __ldcg(reinterpret_cast<const float4*>(a.acc_s + o));
+                                sv[0] = bf_round(s4.x);
+                                sv[1] = bf_round(s4.y);
+                                sv[2] = bf_round(s4.z);
+                                sv[3] = bf_round(s4.w);
+                            } else if (a.fin_sh) {  // read before the write below (in-place form)
+                                const uint2 y = *reinterpret_cast<const uint2*>(a.fin_sh + o);
+                                sv[0] = bf16lo(y.x);
+                                sv[1] = bf16hi(y.x);
+                                sv[2] = bf16lo(y.y);
+                                sv[3] = bf16hi(y.y);
+                            }
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                float q = bf_round(__fmul_rn(a.fin_scale, r[j]));
+                                if (has_s) q = __fadd_rn(q, sv[j]);
+                                r[j] = q;
+                            }
+                            uint2 ob;
+                            ob.x = (uint32_t)f2bf_bits(r[0]) | ((uint32_t)f2bf_bits(r[1]) << 16);
+                            ob.y = (uint32_t)f2bf_bits(r[2]) | ((uint32_t)f2bf_bits(r[3]) << 16);
+                            *reinterpret_cast<uint2*>(a.fin_out + o) = ob;
+                        }
+                    }
+                }
+            }
         }
     } else if (C::kGather) {
         // ------------------------------------------------------------ FC1 token gather

@@ -173,6 +173,11 @@ struct GemmArgs {
     float* zero_ptr;         // FC1: buffer zeroed by the epilogue warps before their tiles
     size_t zero_n;           //      (floats, multiple of 4)
     const float* sgate;      // FC2: shared-expert gate per token (acc_s += gate[t] * y), or null
+    bf16* fin_out;           // FC2, few tokens: the layer output, written by the last warp to add into
+                             // each 128-feature block (no finalize kernel); null = finalize kernel
+    const bf16* fin_sh;      //   the caller's shared output (with fin_out), or null
+    float fin_scale;         //   routed scale (with fin_out)
+    int* fin_cnt;            //   per-feature-block counters, zero on entry (with fin_out)
     int streamk_max;         // stream-K when the call has fewer tiles than this (0: never)
     float* skp;              // FC1 stream-K partial sums, one slot per CTA ([kNA][BN][128] FP32)
     int* done;               // FC1 stream-K per-tile counters (zero on entry, >= streamk_max of them)

@@ -155,12 +155,159 @@ __global__ void __launch_bounds__(32 * kTopkRowsPerBlock) topk_kernel(const void
     pdl_trigger();
 }
 
+// ---------------------------------------------------------------- top-k, several warps per row
+// For many experts and exact logits (few-token router, given or BF16 logits), one warp per
+// row walks a long chain (V keys per lane, K rounds, rescans).  Here W warps share a row:
+// warp w takes experts [w * Ew, (w + 1) * Ew) and selects their top K with the same
+// screening and exact keys as a whole-row warp.  Every member of the row's top K is in its
+// own warp's top K, so warp 0 then selects the row's top K from the W * K entries -- two per
+// lane, compared by (exact key desc, expert id asc) with explicit ids -- and computes the
+// weights (sigmoid: s_k / sum s; softmax with renorm: exp(l_k - l_max) / sum over the K).
+static constexpr int kWideWarps = 4;
+static constexpr int kWideMaxK = 16;  // W * K entries fit two per lane
+template <int V, bool BF16_IN>
+__global__ void __launch_bounds__(32 * kWideWarps) topk_wide_kernel(const void* __restrict__ logits, int M, int E,
+                                                                    int K, int score, const float* __restrict__ bias,
+                                                                    int renorm, float* __restrict__ topk_w,
+                                                                    int32_t* __restrict__ topk_ids,
+                                                                    int32_t* __restrict__ src_idx,
+                                                                    float* __restrict__ w_copy,
+                                                                    int32_t* __restrict__ id_copy,
+                                                                    int* __restrict__ counts, const GateArgs gate) {
+    __shared__ float s_wbuf[kWideWarps][32];
+    __shared__ int s_id[kWideWarps][32];
+    __shared__ float s_l[kWideWarps][32], s_s[kWideWarps][32];
+    __shared__ int s_k[kWideWarps];
+    pdl_wait();
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const int row = blockIdx.x;
+    const bool sig = score == MOE_SCORE_SIGMOID;
+    const int ew = cdiv(cdiv(E, kWideWarps), 32) * 32;  // experts per warp (whole lanes)
+    const int e0 = w * ew;
+    const int en = max(0, min(ew, E - e0));
+    const int kw = min(K, en);
+    if (en > 0) {
+        float l[V], key[V], sx[V];
+        if (BF16_IN)
+            load_row_bf16<V>(static_cast<const uint16_t*>(logits) + (size_t)row * E + e0, en, lane, l);
+        else
+            load_row_f32<V>(static_cast<const float*>(logits) + (size_t)row * E + e0, en, lane, l);
+        const float* bw = bias ? bias + e0 : nullptr;
+        screening_keys<V>(l, key, en, sig, bw, lane);
+#pragma unroll
+        for (int c = 0; c < V; ++c) sx[c] = 0.0f;
+        if (sig) route_refine_keys<V>(l, key, sx, en, kw, sig, bw, lane, 0.0f, NoRefine{}, s_wbuf[w]);
+        float kth, sel_l, sel_s;
+        const int id = warp_select<V, true>(key, l, sx, en, kw, lane, kth, sel_l, sel_s);
+        if (lane < kw) {
+            s_id[w][lane] = e0 + id;
+            s_l[w][lane] = sel_l;
+            s_s[w][lane] = sel_s;
+        }
+    }
+    if (lane == 0) s_k[w] = kw;
+    __syncthreads();
+    if (w == 1 && gate.w) shared_gate_row(gate, row, lane);  // alongside warp 0's merge
+    if (w != 0) {
+        pdl_trigger();
+        return;
+    }
+    // ---- warp 0: the row's top K from the warps' entries, two per lane
+    const float NEG_INF = __int_as_float(0xff800000);
+    uint32_t code[2];
+    int eid[2];
+    float el[2], es[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int j = lane + 32 * h;  // entry j: warp j / K, slot j % K
+        const int ww = j / K, kk = j - ww * K;
+        code[h] = 0u;
+        eid[h] = 0x7fffffff;
+        el[h] = es[h] = 0.0f;
+        if (ww < kWideWarps && kk < s_k[ww]) {
+            eid[h] = s_id[ww][kk];
+            el[h] = s_l[ww][kk];
+            es[h] = s_s[ww][kk];
+            float k = sig ? es[h] : el[h];
+            if (bias) k = __fadd_rn(k, bias[eid[h]]);
+            code[h] = key_code((k != k) ? NEG_INF : k);
+        }
+    }
+    int my_id = 0;
+    float my_l = 0.0f, my_s = 0.0f;
+    for (int r = 0; r < K; ++r) {
+        // this lane's better entry under (code desc, id asc); code 0 = none
+        const bool second = code[1] > code[0] || (code[1] == code[0] && code[1] != 0u && eid[1] < eid[0]);
+        const uint32_t c = second ? code[1] : code[0];
+        const int id = second ? eid[1] : eid[0];
+        const uint32_t best = __reduce_max_sync(0xffffffffu, c);
+        const uint32_t mine = (c != 0u && c == best) ? (uint32_t)id : 0x7fffffffu;
+        const int win = (int)__reduce_min_sync(0xffffffffu, mine);
+        const int src = __ffs(__ballot_sync(0xffffffffu, c != 0u && c == best && id == win)) - 1;
+        const float wl = __shfl_sync(0xffffffffu, second ? el[1] : el[0], src & 31);
+        const float ws = __shfl_sync(0xffffffffu, second ? es[1] : es[0], src & 31);
+        if (lane == r) {
+            my_id = win;
+            my_l = wl;
+            my_s = ws;
+        }
+        if (lane == src) {
+            if (second) code[1] = 0u;
+            else code[0] = 0u;
+        }
+    }
+    float wgt;
+    if (sig) {
+        const float sk = (lane < K) ? my_s : 0.0f;
+        double sum = 0.0;
+        for (int r = 0; r < K; ++r) sum += (double)__shfl_sync(0xffffffffu, sk, r);
+        wgt = renorm ? __double2float_rn((double)sk / sum) : sk;
+    } else {  // softmax with renorm (the only softmax mode routed here)
+        float lmax = (lane < K) ? my_l : NEG_INF;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) lmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
+        const double ex = (lane < K) ? exp_f64((double)my_l - (double)lmax) : 0.0;
+        double sum = 0.0;
+        for (int r = 0; r < K; ++r) sum += __shfl_sync(0xffffffffu, ex, r);
+        wgt = __double2float_rn(ex / sum);
+    }
+    if (lane < K) {
+        const size_t o = (size_t)row * K + lane;
+        topk_w[o] = wgt;
+        topk_ids[o] = my_id;
+        if (src_idx) src_idx[o] = lane * M + row;
+        if (w_copy) w_copy[o] = wgt;
+        if (id_copy) id_copy[o] = my_id;
+        if (counts) atomicAdd(counts + my_id, 1);
+    }
+    pdl_trigger();
+}
+
+// The several-warp top-k serves exact logits with many experts (at least 8 keys per lane
+// in the one-warp form) when the weights need only the selected experts.
+static bool use_wide_topk(int E, int K, int score, int renorm) {
+    return E > 256 && K <= kWideMaxK && (score == MOE_SCORE_SIGMOID || renorm);
+}
+
 cudaError_t launch_topk(const void* logits, bool bf16_in, int M, int E, int K, int score, const float* bias,
                         int renorm, float* topk_w, int32_t* topk_ids, int32_t* src_idx, float* w_copy,
                         int32_t* id_copy, cudaStream_t s, bool pdl, const RefineArgs* refine, int* counts,
                         const GateArgs* gate_in) {
     dim3 grid(cdiv(M, kTopkRowsPerBlock)), block(32 * kTopkRowsPerBlock);
     const GateArgs gate = gate_in ? *gate_in : GateArgs{nullptr, nullptr, 0, nullptr};
+    if (!refine && use_wide_topk(E, K, score, renorm)) {
+        const int vw = topk_v(cdiv(E, kWideWarps));
+#define MOE_W(VV)                                                                                                   \
+        if (vw == VV)                                                                                               \
+            return bf16_in ? launch_k(topk_wide_kernel<VV, true>, dim3(M), dim3(32 * kWideWarps), 0, s, pdl, logits, \
+                                      M, E, K, score, bias, renorm, topk_w, topk_ids, src_idx, w_copy, id_copy,      \
+                                      counts, gate)                                                                 \
+                           : launch_k(topk_wide_kernel<VV, false>, dim3(M), dim3(32 * kWideWarps), 0, s, pdl, logits,\
+                                      M, E, K, score, bias, renorm, topk_w, topk_ids, src_idx, w_copy, id_copy,      \
+                                      counts, gate);
+        MOE_W(4) MOE_W(8)
+#undef MOE_W
+    }
     const int v = topk_v(E);
     const bf16* x = refine ? refine->x : nullptr;
     const bf16* wr = refine ? refine->wr : nullptr;

@@ -25,7 +25,8 @@ WS_TOPK_IDS, WS_TOPK_W, WS_OFFSETS, WS_PERM = range(4)
 
 # Every symbol include/moe.h declares.
 EXPORTS = ("moe_router_topk", "moe_permute_workspace_size", "moe_permute", "moe_workspace_size",
-           "moe_select_path", "moe_fused_forward", "moe_fused_forward_launches", "moe_token_tiles",
+           "moe_select_path", "moe_fused_forward", "moe_fused_forward_launches", "moe_fused_forward_plan",
+           "moe_token_tiles",
            "moe_workspace_region", "moe_fused_forward_timed", "moe_fused_forward_noalloc",
            "moe_noalloc_get_error", "moe_get_error", "moe_status_string")
 
@@ -56,6 +57,9 @@ _lib.moe_select_path.argtypes = [ctypes.POINTER(LayerDesc)]
 _lib.moe_select_path.restype = _ci
 _lib.moe_fused_forward_launches.argtypes = [ctypes.POINTER(LayerDesc)]
 _lib.moe_fused_forward_launches.restype = _ci
+_lib.moe_fused_forward_plan.argtypes = [ctypes.POINTER(LayerDesc), ctypes.POINTER(_ci), _ci]
+_lib.moe_fused_forward_plan.restype = _ci
+KERNEL_NAMES = ("prep", "router", "route", "topk", "refine", "select", "permute", "fc1", "fc2", "finalize")
 _lib.moe_token_tiles.argtypes = [ctypes.POINTER(LayerDesc), ctypes.POINTER(_ci), ctypes.POINTER(_ci)]
 _lib.moe_token_tiles.restype = _ci
 _lib.moe_workspace_region.argtypes = [ctypes.POINTER(LayerDesc), _ci, ctypes.POINTER(_sz), ctypes.POINTER(_sz)]
@@ -183,6 +187,13 @@ def select_path(desc: LayerDesc) -> str:
 
 def launches(desc: LayerDesc) -> int:
     return _lib.moe_fused_forward_launches(ctypes.byref(desc))
+
+
+def kernel_plan(desc: LayerDesc):
+    """Names of the kernels moe_fused_forward launches for this description, in order."""
+    buf = (_ci * 16)()
+    n = _lib.moe_fused_forward_plan(ctypes.byref(desc), buf, 16)
+    return [KERNEL_NAMES[buf[i]] for i in range(n)]
 
 
 def token_tiles(desc: LayerDesc):

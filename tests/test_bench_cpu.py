@@ -36,16 +36,6 @@ def test_roofline_bound_choice():
     assert r["bound"] == "tensor" and abs(r["frac"] - 0.5) < 1e-12
 
 
-def test_kernel_names_follow_launch_order():
-    assert bench.kernel_names("small", True) == ["router", "route", "fc1", "fc2"]
-    assert bench.kernel_names("large", True, 9) == ["prep", "router", "topk", "refine", "select", "permute", "fc1",
-                                                    "fc2", "finalize"]
-    assert bench.kernel_names("large", True, 7) == ["prep", "router", "topk", "permute", "fc1", "fc2", "finalize"]
-    assert bench.kernel_names("large", True, 6) == ["router", "topk", "permute", "fc1", "fc2", "finalize"]
-    assert bench.kernel_names("large", False, 6) == ["prep", "topk", "permute", "fc1", "fc2", "finalize"]
-    assert bench.kernel_names("large", False) == ["prep", "topk", "permute", "fc1", "fc2", "finalize"]
-
-
 def _free_port():
     s = socket.socket()
     s.bind(("127.0.0.1", 0))
