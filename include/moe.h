@@ -191,8 +191,7 @@ int moe_fused_forward_launches(const moe_layer_desc* d);
 
 /* The kernels moe_fused_forward enqueues for this description, in launch order: writes up
  * to max_kernels MOE_K_* values to `kernels` (may be NULL) and returns their number (0
- * for an invalid description or T == 0).  The path, the router used and the folding of
- * the finalize into FC2 (few tokens) decide the list. */
+ * for an invalid description or T == 0).  The path and the router used decide the list. */
 enum { MOE_K_PREP = 0,        /* zero the call's counters; bound the router rows' norms */
        MOE_K_ROUTER = 1,      /* router logits */
        MOE_K_ROUTE_TABLE = 2, /* few-token path: routing and the distinct-expert table */

@@ -22,26 +22,18 @@ int num_sms() {
 
 // Workspace carve-up of moe_fused_forward, 256-byte aligned regions after the header.
 struct WsLayout {
-    size_t logits, route, topk_w, topk_ids, offsets, tiles1, tiles2, counts, wpart, perm, cand, h, hs, acc, skp, gate,
-        total;
+    size_t logits, route, topk_w, topk_ids, offsets, tiles1, tiles2, counts, wpart, xn2, perm, cand, h, hs, acc, skp,
+        gate, total;
 };
 // Candidate-list capacity per token of the three-kernel top-k (rows with more fall back).
 constexpr size_t kCandPerRow = 32;
 // Counters zeroed at the start of each many-token call (by its first kernel): per-expert
-// counts, per-expert cursors, the candidate count, FC1's stream-K per-tile counters, then
-// the per-feature-block counters of FC2's folded finalize.
-constexpr int kFinMaxBlocks = 64;  // H <= 8192
-inline size_t counter_ints(size_t E) { return 2 * (E + 2) + 4 + kStreamKMaxTiles + kFinMaxBlocks; }
+// counts, per-expert cursors, the candidate count, then FC1's stream-K per-tile counters.
+inline size_t counter_ints(size_t E) { return 2 * (E + 2) + 4 + kStreamKMaxTiles; }
 inline size_t done_int(size_t E) { return 2 * (E + 2) + 4; }
-inline size_t fin_int(size_t E) { return done_int(E) + kStreamKMaxTiles; }
-// Few tokens: FC2's last warp per 128-feature block writes the output (no finalize launch).
-constexpr int kFoldFinalizeMaxT = 64;
-inline bool fold_finalize(const moe_layer_desc* d) {
-    return d->T <= kFoldFinalizeMaxT && (d->H + 127) / 128 <= kFinMaxBlocks;
-}
 inline size_t cand_count_int(size_t E) { return 2 * (E + 2); }
-// Per-CTA router weight-norm bounds of the prep kernel (its grid is at most E / 8 <= 128).
-constexpr size_t kMaxPrepGrid = (MOE_MAX_EXPERTS + 7) / 8;
+// Per-CTA router weight-norm bounds of the prep kernel (one per SM at most).
+constexpr size_t kMaxPrepGrid = 1024;
 WsLayout layout(const moe_layer_desc* d) {
     const size_t T = (size_t)d->T, E = (size_t)d->E, K = (size_t)d->top_k, H = (size_t)d->H, I = (size_t)d->I,
                  Is = (size_t)d->I_shared;
@@ -61,6 +53,7 @@ WsLayout layout(const moe_layer_desc* d) {
     L.tiles2 = take((E + 2) * 4);
     L.counts = take(counter_ints(E) * 4);
     L.wpart = take(kMaxPrepGrid * 4);
+    L.xn2 = take(T * 4);
     L.perm = take(T * K * 4);
     L.cand = take(T * (3 + 3 * kCandPerRow) * 4);  // row_base, row_n, row_eps, cand_row, cand_e, cand_val
     L.h = take(T * K * I * 2);
@@ -338,7 +331,7 @@ int moe_fused_forward_plan(const moe_layer_desc* d, int* kernels, int max_kernel
         k[n++] = MOE_K_PERMUTE;
         k[n++] = MOE_K_FC1;
         k[n++] = MOE_K_FC2;
-        if (!fold_finalize(d)) k[n++] = MOE_K_FINALIZE;
+        k[n++] = MOE_K_FINALIZE;
     }
     for (int i = 0; kernels && i < n && i < max_kernels; ++i) kernels[i] = k[i];
     return n;
@@ -392,7 +385,8 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
     if (path == MOE_PATH_LARGE && prep_kernel_for(d)) {
         if (!mark()) return MOE_ERR_CUDA;
         MOE_CK(launch_prep(reinterpret_cast<int*>(w8 + L.counts), (int)counter_ints(E),
-                           dense_router ? static_cast<const bf16*>(d->router_w) : nullptr, E, H, wpart, sms, s));
+                           dense_router ? static_cast<const bf16*>(d->router_w) : nullptr, E, H, wpart, x, T,
+                           reinterpret_cast<float*>(w8 + L.xn2), sms, s));
         pdl = !timed;
     }
 
@@ -476,7 +470,8 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
     const int bn1 = gemm_token_tile(fc1_mode, T, K, E), bn2 = gemm_token_tile(GM_FC2, T, K, E);
     // 2. top-k (also counts the slots per expert; the counters were cleared in step 0)
     if (!mark()) return MOE_ERR_CUDA;
-    RefineArgs ra = {x, static_cast<const bf16*>(d->router_w), H, logits_rw, wpart, prep_grid(E, sms), err};
+    RefineArgs ra = {x, static_cast<const bf16*>(d->router_w), H, logits_rw, wpart, prep_grid(E, T, sms),
+                     reinterpret_cast<const float*>(w8 + L.xn2), err};
     if (dense_router && split_topk_mode(d)) {  // screen, refine, final
         int* cbase = reinterpret_cast<int*>(w8 + L.cand);
         CandList cl;
@@ -592,19 +587,13 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
     g2.streamk_max = gemm_streamk_max(GM_FC2, bn2, sms, max_tiles(bn2, g2.nfeat_r, Is ? g2.nfeat_s : 0));
     g2.skp = nullptr;
     g2.done = nullptr;
-    const bool fold = fold_finalize(d);
-    g2.fin_out = fold ? out : nullptr;
-    g2.fin_sh = fold ? sh_out : nullptr;
-    g2.fin_scale = rscale;
-    g2.fin_cnt = counts + fin_int(E);
+
     if (!mark()) return MOE_ERR_CUDA;
     MOE_CK(launch_gemm(GM_FC2, bn2, g2, m2, sms, s, chain));
 
-    // 6. finalize (folded into FC2 for few tokens)
-    if (!fold) {
-        if (!mark()) return MOE_ERR_CUDA;
-        MOE_CK(launch_finalize(acc, acc_s, sh_out, out, (size_t)T * H, rscale, sms, s, chain));
-    }
+    // 6. finalize
+    if (!mark()) return MOE_ERR_CUDA;
+    MOE_CK(launch_finalize(acc, acc_s, sh_out, out, (size_t)T * H, rscale, sms, s, chain));
     if (!mark()) return MOE_ERR_CUDA;
     return MOE_OK;
 }

@@ -168,6 +168,7 @@ struct Seg {
 // with nk_r k-blocks and the shared group's with nk_s -- is split into gridDim.x equal
 // contiguous ranges, cut at tile boundaries into segments.  Every role of the CTA walks
 // the same sequence.
+template <bool SK>
 struct WorkWalk {
     int total, R, nk_r, nk_s, streamk, next_tile;
     long long N, hi, i;
@@ -176,7 +177,7 @@ struct WorkWalk {
         R = R_;
         nk_r = nk_r_;
         nk_s = nk_s_;
-        streamk = sk ? 1 : 0;
+        streamk = (SK && sk) ? 1 : 0;
         N = (long long)R * nk_r + (long long)(total - R) * nk_s;
         i = lo_of(blockIdx.x);
         hi = lo_of(blockIdx.x + 1);
@@ -186,7 +187,7 @@ struct WorkWalk {
     // CTA whose range holds iteration it: the largest b with lo_of(b) <= it.
     __device__ int owner(long long it) const { return (int)(((it + 1) * gridDim.x - 1) / N); }
     __device__ bool next(Seg& s) {
-        if (!streamk) {
+        if (!SK || !streamk) {
             if (next_tile >= total) return false;
             s.tile = next_tile;
             s.kb0 = 0;
@@ -221,6 +222,44 @@ struct WorkWalk {
     // CTA c holds iterations (its range is not empty).
     __device__ bool active(int c) const { return lo_of(c) < lo_of(c + 1); }
 };
+
+// FC2 epilogue of one 32-column chunk (see the comment at its call).
+__device__ __forceinline__ void combine_chunk(const uint32_t (&v)[32], int mt, float mw, int c0, int n, int f,
+                                              int feat, int T, float* __restrict__ acc, int lane) {
+    const int i4 = lane & 3;
+    const bool fok4 = f - i4 + 3 < feat;  // features of my group (feat % 8 == 0)
+#pragma unroll
+    for (int j0 = 0; j0 < 32; j0 += 4) {
+        float r[4];
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) r[jj] = __uint_as_float(v[j0 + jj]);
+        // r[jj] = y[feature of this lane, token j0 + jj]; 4x4 transpose
+        float t0 = (i4 & 1) ? r[0] : r[1], t1 = (i4 & 1) ? r[2] : r[3];
+        t0 = __shfl_xor_sync(0xffffffffu, t0, 1);
+        t1 = __shfl_xor_sync(0xffffffffu, t1, 1);
+        if (i4 & 1) {
+            r[0] = t0;
+            r[2] = t1;
+        } else {
+            r[1] = t0;
+            r[3] = t1;
+        }
+        float u0 = (i4 & 2) ? r[0] : r[2], u1 = (i4 & 2) ? r[1] : r[3];
+        u0 = __shfl_xor_sync(0xffffffffu, u0, 2);
+        u1 = __shfl_xor_sync(0xffffffffu, u1, 2);
+        if (i4 & 2) {
+            r[0] = u0;
+            r[1] = u1;
+        } else {
+            r[2] = u0;
+            r[3] = u1;
+        }
+        const int tok = __shfl_sync(0xffffffffu, mt, j0 + i4);
+        const float wt = __shfl_sync(0xffffffffu, mw, j0 + i4);
+        if (c0 + j0 + i4 < n && fok4 && (unsigned)tok < (unsigned)T)
+            red_add_v4_f32(acc + (size_t)tok * feat + (f - i4), wt * r[0], wt * r[1], wt * r[2], wt * r[3]);
+    }
+}
 
 // SK: the stream-K variant (the host launches it for calls with few tiles per SM); the
 // other variant deals whole tiles only, and compiles without the stream-K bookkeeping.
@@ -285,22 +324,20 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
     const uint32_t tmem_base = *tmem_slot;
     const int total = a.dense ? a.nfeat_r * cdiv(a.T, kDenseTokenTile) : s_tiles[G];
     const int routed_tiles = (a.dense || !a.has_shared) ? total : s_tiles[a.E];
-    const bool streamk = SK && total > 0 && total < a.streamk_max;
+    // Stream-K only where dealing whole tiles would leave the last wave mostly idle: more
+    // tiles than CTAs, but under three quarters of the whole-tile waves' slots filled
+    // (measured: with fewer tiles than SMs, or with several full waves, whole tiles are as
+    // fast or faster).
+    const int waves = cdiv(total, (int)gridDim.x);
+    const bool streamk = SK && total > (int)gridDim.x && total < a.streamk_max &&
+                         4 * total < 3 * waves * (int)gridDim.x;
     const int nk_r = cdiv(a.kdim, BK), nk_s = cdiv(a.kdim_s > 0 ? a.kdim_s : a.kdim, BK);
     // Round-robin dealing keeps the CTAs on neighbouring tiles of the group-major list (one
     // expert's feature and token tiles), which share that expert's weight and token rows in
     // L2, and spreads tiles of unequal cost (ragged token tails) evenly.
-    WorkWalk work;
+    WorkWalk<SK> work;
     work.init(total, routed_tiles, nk_r, nk_s, streamk);
     Seg sg;
-    // FC2 with the finalize folded in: every epilogue warp adds the k-blocks of each of its
-    // segments to its feature block's counter; the warp that completes the block's total
-    // (all tiles of that block, all their k-blocks, times the epilogue warps) finalizes it.
-    const int fin_target =
-        (MODE == GM_FC2 && a.fin_out)
-            ? ((routed_tiles / max(1, a.nfeat_r)) * nk_r +
-               (a.has_shared ? ((total - routed_tiles) / max(1, a.nfeat_s)) * nk_s : 0)) * C::kEpiWarps
-            : 0;
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
@@ -426,20 +463,18 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
                 mt[ci] = 0;
                 mw[ci] = 0.0f;
                 const int colm = 32 * half + 32 * nhalf * ci + lane;
-                if (MODE == GM_FC2 && colm < ti.n) {
-                    if (ti.shared) {
-                        mt[ci] = ti.row0 + colm;
-                        mw[ci] = a.sgate ? a.sgate[mt[ci]] : 1.0f;
-                    } else if (ti.row0 + ti.n <= a.T * a.K) {
-                        const int src = a.perm[ti.row0 + colm];
-                        if ((unsigned)src < (unsigned)(a.T * a.K)) {
-                            const int kk = src / a.T;
-                            mt[ci] = src - kk * a.T;
-                            mw[ci] = a.topk_w[(size_t)mt[ci] * a.K + kk];
-                        } else {  // never from a valid permutation: flag it, contribute nothing
-                            set_dev_error(a.err, MOE_DEVERR_BAD_INDEX);
-                        }
+                if (MODE == GM_FC2 && !ti.shared && colm < ti.n && ti.row0 + ti.n <= a.T * a.K) {
+                    const int src = a.perm[ti.row0 + colm];
+                    if ((unsigned)src < (unsigned)(a.T * a.K)) {
+                        const int kk = src / a.T;
+                        mt[ci] = src - kk * a.T;
+                        mw[ci] = a.topk_w[(size_t)mt[ci] * a.K + kk];
+                    } else {  // never from a valid permutation: flag it, contribute nothing
+                        set_dev_error(a.err, MOE_DEVERR_BAD_INDEX);
                     }
+                } else if (MODE == GM_FC2 && ti.shared && colm < ti.n) {
+                    mt[ci] = ti.row0 + colm;
+                    mw[ci] = a.sgate ? a.sgate[mt[ci]] : 1.0f;
                 }
             }
             const bool waited = mbar_wait(tfull_bar(buf), tph, abort_flag, a.err);
@@ -566,41 +601,8 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
                     // vector reduction (FP32 add in L2).  A stream-K range adds its partial
                     // sum the same way.  No shared memory is staged, so the ring keeps it for
                     // weights.
-                    float* dstacc = ti.shared ? a.acc_s : a.acc;
-                    const int i4 = lane & 3;
-                    const bool fok4 = f - i4 + 3 < feat;  // features of my group (feat % 8 == 0)
-#pragma unroll
-                    for (int j0 = 0; j0 < 32; j0 += 4) {
-                        float r[4];
-#pragma unroll
-                        for (int jj = 0; jj < 4; ++jj) r[jj] = __uint_as_float(v[j0 + jj]);
-                        // r[jj] = y[feature of this lane, token j0 + jj]; 4x4 transpose
-                        float t0 = (i4 & 1) ? r[0] : r[1], t1 = (i4 & 1) ? r[2] : r[3];
-                        t0 = __shfl_xor_sync(0xffffffffu, t0, 1);
-                        t1 = __shfl_xor_sync(0xffffffffu, t1, 1);
-                        if (i4 & 1) {
-                            r[0] = t0;
-                            r[2] = t1;
-                        } else {
-                            r[1] = t0;
-                            r[3] = t1;
-                        }
-                        float u0 = (i4 & 2) ? r[0] : r[2], u1 = (i4 & 2) ? r[1] : r[3];
-                        u0 = __shfl_xor_sync(0xffffffffu, u0, 2);
-                        u1 = __shfl_xor_sync(0xffffffffu, u1, 2);
-                        if (i4 & 2) {
-                            r[0] = u0;
-                            r[1] = u1;
-                        } else {
-                            r[2] = u0;
-                            r[3] = u1;
-                        }
-                        const int tok = __shfl_sync(0xffffffffu, mt[ci], j0 + i4);
-                        const float wt = __shfl_sync(0xffffffffu, mw[ci], j0 + i4);
-                        if (c0 + j0 + i4 < ti.n && fok4 && (unsigned)tok < (unsigned)a.T)
-                            red_add_v4_f32(dstacc + (size_t)tok * feat + (f - i4), wt * r[0], wt * r[1],
-                                           wt * r[2], wt * r[3]);
-                    }
+                    if (ti.shared) combine_chunk(v, mt[ci], mw[ci], c0, ti.n, f, a.feat_s, a.T, a.acc_s, lane);
+                    else combine_chunk(v, mt[ci], mw[ci], c0, ti.n, f, a.feat_r, a.T, a.acc, lane);
                 } else {  // GM_DENSE
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
@@ -617,54 +619,6 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(tempty_bar(buf));
             ++tcount;
-            if (MODE == GM_FC2 && a.fin_out) {
-                // This warp's reductions for the segment are issued; fence them, count them.
-                __threadfence();
-                __syncwarp();
-                int last = 0;
-                if (lane == 0) {
-                    const int add = sg.kb1 - sg.kb0;
-                    last = atomicAdd(a.fin_cnt + ti.ft, add) + add == fin_target;
-                }
-                last = __shfl_sync(0xffffffffu, last, 0);
-                if (last) {  // every addition into this feature block is done: finalize it
-                    __threadfence();
-                    const int f4 = ti.ft * BM + 4 * lane;  // 4 features per lane
-                    const int H = a.feat_r;
-                    if (f4 < H) {
-                        for (int t = 0; t < a.T; ++t) {
-                            const size_t o = (size_t)t * H + f4;
-                            const float4 r4 = __ldcg(reinterpret_cast<const float4*>(a.acc + o));
-                            float r[4] = {r4.x, r4.y, r4.z, r4.w};
-                            float sv[4] = {0.f, 0.f, 0.f, 0.f};
-                            const bool has_s = a.has_shared || a.fin_sh;
-                            if (a.has_shared) {
-                                const float4 s4 = __ldcg(reinterpret_cast<const float4*>(a.acc_s + o));
-                                sv[0] = bf_round(s4.x);
-                                sv[1] = bf_round(s4.y);
-                                sv[2] = bf_round(s4.z);
-                                sv[3] = bf_round(s4.w);
-                            } else if (a.fin_sh) {  // read before the write below (in-place form)
-                                const uint2 y = *reinterpret_cast<const uint2*>(a.fin_sh + o);
-                                sv[0] = bf16lo(y.x);
-                                sv[1] = bf16hi(y.x);
-                                sv[2] = bf16lo(y.y);
-                                sv[3] = bf16hi(y.y);
-                            }
-#pragma unroll
-                            for (int j = 0; j < 4; ++j) {
-                                float q = bf_round(__fmul_rn(a.fin_scale, r[j]));
-                                if (has_s) q = __fadd_rn(q, sv[j]);
-                                r[j] = q;
-                            }
-                            uint2 ob;
-                            ob.x = (uint32_t)f2bf_bits(r[0]) | ((uint32_t)f2bf_bits(r[1]) << 16);
-                            ob.y = (uint32_t)f2bf_bits(r[2]) | ((uint32_t)f2bf_bits(r[3]) << 16);
-                            *reinterpret_cast<uint2*>(a.fin_out + o) = ob;
-                        }
-                    }
-                }
-            }
         }
     } else if (C::kGather) {
         // ------------------------------------------------------------ FC1 token gather

@@ -35,6 +35,7 @@ struct RefineArgs {
     float* logits_rw;    // refined logits are written back here (the logits buffer)
     const float* wpart;  // [nwpart] per-CTA upper bounds of max_e |Wr[e]|_2^2 (prep kernel)
     int nwpart;
+    const float* xn2;    // [M] upper bounds of |x_t|_2^2 (prep kernel)
     int* err;            // device error word (MOE_DEVERR_ROUTER_BOUND)
 };
 // Shared-expert gate of each token, computed by the routing kernels (one exact dot
@@ -112,11 +113,11 @@ cudaError_t launch_small(const SmallArgs& a, int num_sms, cudaStream_t s, bool p
                          const std::function<bool()>* mark);
 
 // First kernel of a many-token call: zeroes the call's counters (n ints) and, when wr is
-// given, writes per-CTA upper bounds of max_e |wr[e]|_2^2 into wpart[prep_grid(E, sms)]
-// (the bound on the tensor-core router's error uses their maximum).
-int prep_grid(int E, int num_sms);
-cudaError_t launch_prep(int* counters, int n, const bf16* wr, int E, int H, float* wpart, int num_sms,
-                        cudaStream_t s);
+// given, writes per-CTA upper bounds of max_e |wr[e]|_2^2 into wpart[prep_grid(E, T, sms)]
+// and upper bounds of |x_t|_2^2 into xn2[T] (the bound on the tensor-core router's error).
+int prep_grid(int E, int T, int num_sms);
+cudaError_t launch_prep(int* counters, int n, const bf16* wr, int E, int H, float* wpart, const bf16* x, int T,
+                        float* xn2, int num_sms, cudaStream_t s);
 
 // ---------------------------------------------------------------- permutation
 // Tile bookkeeping that the permute kernel writes for the grouped GEMMs (group g < E is
@@ -173,11 +174,6 @@ struct GemmArgs {
     float* zero_ptr;         // FC1: buffer zeroed by the epilogue warps before their tiles
     size_t zero_n;           //      (floats, multiple of 4)
     const float* sgate;      // FC2: shared-expert gate per token (acc_s += gate[t] * y), or null
-    bf16* fin_out;           // FC2, few tokens: the layer output, written by the last warp to add into
-                             // each 128-feature block (no finalize kernel); null = finalize kernel
-    const bf16* fin_sh;      //   the caller's shared output (with fin_out), or null
-    float fin_scale;         //   routed scale (with fin_out)
-    int* fin_cnt;            //   per-feature-block counters, zero on entry (with fin_out)
     int streamk_max;         // stream-K when the call has fewer tiles than this (0: never)
     float* skp;              // FC1 stream-K partial sums, one slot per CTA ([kNA][BN][128] FP32)
     int* done;               // FC1 stream-K per-tile counters (zero on entry, >= streamk_max of them)

@@ -13,20 +13,12 @@ namespace moe {
 // 17 addends to the largest one and truncates them, within one such unit per addend --
 // the computed logit lies within H * 2^-22 * sum_h |x_h w_h| of the exact sum.  Cauchy-
 // Schwarz bounds the sum by |x_t|_2 * max_e |Wr[e]|_2; the router GEMM supplies an upper
-// bound of max_e |Wr[e]|_2^2, and |x_t|_2^2 is summed here in FP32 and scaled up by
-// (1 + 2^-8) to cover its own rounding (H <= 2^16).  A final factor (1 + 2^-8) covers the
-// roundings of this product.  Hmax = the padded reduction length, a multiple of 64.
-__device__ __forceinline__ float tc_logit_bound(const bf16* __restrict__ xr, int H, float wnorm2, int lane) {
-    float ss = 0.0f;
-    for (int c = lane; c < (H >> 3); c += 32) {
-        const uint4 v = ld_nc16(xr + (size_t)c * 8);
-        ss = dot8(v, v, ss);
-    }
-    ss = warp_sum(ss);
+// bound of max_e |Wr[e]|_2^2 and of every |x_t|_2^2 (FP32 sums of squares scaled up by
+// (1 + 2^-8) to cover their own rounding, H <= 2^16).  A final factor (1 + 2^-8) covers the
+// roundings of this product.  The reduction length is padded to a multiple of 64.
+__device__ __forceinline__ float tc_logit_bound(float xnorm2, int H, float wnorm2) {
     const float hpad = (float)(((H + 63) / 64) * 64);
-    const float xn = sqrtf(ss * (1.0f + 0x1p-8f));
-    const float wn = sqrtf(wnorm2);
-    return hpad * 0x1p-22f * xn * wn * (1.0f + 0x1p-8f);
+    return hpad * 0x1p-22f * sqrtf(xnorm2) * sqrtf(wnorm2) * (1.0f + 0x1p-8f);
 }
 
 // Exact re-evaluation of one candidate's logit (warp-collective), written back into the
@@ -58,14 +50,16 @@ __device__ __forceinline__ void shared_gate_row(const GateArgs& g, int row, int 
 }
 
 // ---------------------------------------------------------------- call prep
-// First kernel of a many-token call.  CTA 0 zeroes the call's counters.  With a router
-// weight, every CTA also bounds the squared L2 norms of its share of the router rows (one
-// warp per row): the FP32 sum of H squares lies within a relative H * 2^-24 of the exact
-// value and is scaled up by (1 + 2^-8) (H <= 2^16), so it is an upper bound; the CTA's
-// maximum goes to wpart[blockIdx.x].  Consumers take the maximum over the grid's entries
-// (no atomics, so nothing needs zeroing first).
+// First kernel of a many-token call.  CTA 0 zeroes the call's counters.  Before the
+// tensor-core router (wr given), the grid's warps also take the E router rows and the T
+// token rows of x, one row each: the FP32 sum of the H squares lies within a relative
+// H * 2^-24 of the exact value and is scaled up by (1 + 2^-8) (H <= 2^16), so it is an
+// upper bound.  Each CTA's maximum over router rows goes to wpart[blockIdx.x] (consumers
+// take the maximum over the grid's entries: no atomics, nothing to zero first); a token
+// row's bound goes to xn2[t].
 __global__ void __launch_bounds__(256) prep_kernel(int* __restrict__ counters, int n, const bf16* __restrict__ wr,
-                                                   int E, int H, float* __restrict__ wpart) {
+                                                   int E, int H, float* __restrict__ wpart,
+                                                   const bf16* __restrict__ x, int T, float* __restrict__ xn2) {
     const int tid = threadIdx.x, lane = tid & 31;
     if (blockIdx.x == 0)
         for (int i = tid; i < n; i += blockDim.x) counters[i] = 0;
@@ -73,14 +67,16 @@ __global__ void __launch_bounds__(256) prep_kernel(int* __restrict__ counters, i
         __shared__ float s_max[8];
         float m = 0.0f;
         const int nw = (gridDim.x * blockDim.x) >> 5;
-        for (int e = (blockIdx.x * blockDim.x + tid) >> 5; e < E; e += nw) {
-            const bf16* row = wr + (size_t)e * H;
+        for (int r = (blockIdx.x * blockDim.x + tid) >> 5; r < E + T; r += nw) {
+            const bf16* row = r < E ? wr + (size_t)r * H : x + (size_t)(r - E) * H;
             float ss = 0.0f;
             for (int c = lane; c < (H >> 3); c += 32) {
                 const uint4 v = ld_nc16(row + (size_t)c * 8);
                 ss = dot8(v, v, ss);
             }
-            m = fmaxf(m, warp_sum(ss) * (1.0f + 0x1p-8f));
+            const float b = warp_sum(ss) * (1.0f + 0x1p-8f);
+            if (r < E) m = fmaxf(m, b);
+            else if (lane == 0) xn2[r - E] = b;
         }
         if (lane == 0) s_max[tid >> 5] = m;
         __syncthreads();
@@ -92,11 +88,12 @@ __global__ void __launch_bounds__(256) prep_kernel(int* __restrict__ counters, i
     pdl_trigger();
 }
 
-int prep_grid(int E, int num_sms) { return std::max(1, std::min(num_sms, cdiv(E, 8))); }
+int prep_grid(int E, int T, int num_sms) { return std::max(1, std::min(num_sms, cdiv(E + T, 8))); }
 
-cudaError_t launch_prep(int* counters, int n, const bf16* wr, int E, int H, float* wpart, int num_sms,
-                        cudaStream_t s) {
-    return launch_k(prep_kernel, dim3(prep_grid(E, num_sms)), dim3(256), 0, s, false, counters, n, wr, E, H, wpart);
+cudaError_t launch_prep(int* counters, int n, const bf16* wr, int E, int H, float* wpart, const bf16* x, int T,
+                        float* xn2, int num_sms, cudaStream_t s) {
+    return launch_k(prep_kernel, dim3(prep_grid(E, wr ? T : 0, num_sms)), dim3(256), 0, s, false, counters, n, wr, E,
+                    H, wpart, x, T, xn2);
 }
 
 // Upper bound of max_e |Wr[e]|_2^2 from the prep kernel's per-CTA maxima (warp-collective).
@@ -118,7 +115,8 @@ __global__ void __launch_bounds__(32 * kTopkRowsPerBlock) topk_kernel(const void
                                                    int32_t* __restrict__ src_idx, float* __restrict__ w_copy,
                                                    int32_t* __restrict__ id_copy, const bf16* __restrict__ x,
                                                    const bf16* __restrict__ wr, int H, float* logits_rw,
-                                                   const float* __restrict__ wpart, int nwpart, int* err,
+                                                   const float* __restrict__ wpart, int nwpart,
+                                                   const float* __restrict__ xn2, int* err,
                                                    int* __restrict__ counts, const GateArgs gate) {
     __shared__ float s_wbuf[kTopkRowsPerBlock][32];
     pdl_wait();
@@ -135,7 +133,7 @@ __global__ void __launch_bounds__(32 * kTopkRowsPerBlock) topk_kernel(const void
         float w, lg;
         if (REFINE) {
             const bf16* xr = x + (size_t)row * H;
-            const float eps = tc_logit_bound(xr, H, wnorm2_max(wpart, nwpart, lane), lane);
+            const float eps = tc_logit_bound(xn2[row], H, wnorm2_max(wpart, nwpart, lane));
             const RowRefine rf{xr, wr, H, E, row, lane, logits_rw, eps, err};
             warp_route_row<V>(l, E, K, score, bias, renorm, lane, eps, rf, wbuf, id, w, lg);
         } else {
@@ -315,19 +313,20 @@ cudaError_t launch_topk(const void* logits, bool bf16_in, int M, int E, int K, i
     float* lrw = refine ? refine->logits_rw : nullptr;
     const float* wn2 = refine ? refine->wpart : nullptr;
     const int nwp = refine ? refine->nwpart : 0;
+    const float* xn2 = refine ? refine->xn2 : nullptr;
     int* err = refine ? refine->err : nullptr;
 #define MOE_L(VV)                                                                                              \
     if (v == VV) {                                                                                             \
         if (refine)                                                                                            \
             return launch_k(topk_kernel<VV, false, true>, grid, block, 0, s, pdl, logits, M, E, K, score, bias, \
-                            renorm, topk_w, topk_ids, src_idx, w_copy, id_copy, x, wr, H, lrw, wn2, nwp, err,  \
-                            counts, gate);                                                                     \
+                            renorm, topk_w, topk_ids, src_idx, w_copy, id_copy, x, wr, H, lrw, wn2, nwp, xn2,  \
+                            err, counts, gate);                                                                \
         return bf16_in ? launch_k(topk_kernel<VV, true, false>, grid, block, 0, s, pdl, logits, M, E, K, score, \
                                   bias, renorm, topk_w, topk_ids, src_idx, w_copy, id_copy, x, wr, H, lrw, wn2, \
-                                  nwp, err, counts, gate)                                                           \
+                                  nwp, xn2, err, counts, gate)                                                           \
                        : launch_k(topk_kernel<VV, false, false>, grid, block, 0, s, pdl, logits, M, E, K, score, \
                                   bias, renorm, topk_w, topk_ids, src_idx, w_copy, id_copy, x, wr, H, lrw, wn2, \
-                                  nwp, err, counts, gate);                                                          \
+                                  nwp, xn2, err, counts, gate);                                                          \
     }
     MOE_L(1) MOE_L(2) MOE_L(4) MOE_L(8) MOE_L(16) MOE_L(32)
 #undef MOE_L
@@ -355,7 +354,8 @@ __global__ void __launch_bounds__(32 * kTopkRowsPerBlock) topk_screen_kernel(con
                                                                               const CandList cl,
                                                                               const bf16* __restrict__ x, int H,
                                                                               const float* __restrict__ wpart,
-                                                                              int nwpart) {
+                                                                              int nwpart,
+                                                                              const float* __restrict__ xn2) {
     pdl_wait();
     const int lane = threadIdx.x & 31;
     const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -363,7 +363,7 @@ __global__ void __launch_bounds__(32 * kTopkRowsPerBlock) topk_screen_kernel(con
         const bool sig = score == MOE_SCORE_SIGMOID;
         float l[V], key[V];
         load_row_f32<V>(logits + (size_t)row * E, E, lane, l);
-        const float eps = tc_logit_bound(x + (size_t)row * H, H, wnorm2_max(wpart, nwpart, lane), lane);
+        const float eps = tc_logit_bound(xn2[row], H, wnorm2_max(wpart, nwpart, lane));
         if (lane == 0) cl.row_eps[row] = eps;
         screening_keys<V>(l, key, E, sig, bias, lane);
         float kth, ua, ub;
@@ -512,7 +512,7 @@ cudaError_t launch_topk_split(const float* logits, int M, int E, int K, int scor
 #define MOE_S(VV)                                                                                           \
     if (v == VV)                                                                                            \
         st = launch_k(topk_screen_kernel<VV>, grid, block, 0, s, pdl, logits, M, E, K, score, bias, cl, ra.x, \
-                      ra.H, ra.wpart, ra.nwpart);
+                      ra.H, ra.wpart, ra.nwpart, ra.xn2);
     MOE_S(1) MOE_S(2) MOE_S(4) MOE_S(8) MOE_S(16) MOE_S(32)
 #undef MOE_S
     if (st != cudaSuccess) return st;

@@ -108,9 +108,9 @@ def test_path_selection_and_launch_counts():
     assert moe.launches(d) == 7  # full softmax keeps the one-kernel top-k
     d = _desc(T=4, path="large")
     assert moe.select_path(d) == "large"
-    assert moe.launches(d) == 5  # few-token router (it zeroes the counters), top-k, permute, fc1, fc2 (+finalize)
+    assert moe.launches(d) == 6  # few-token router (it zeroes the counters), top-k, permute, fc1, fc2, finalize
     d.router_logits = FAKE * 8
-    assert moe.launches(d) == 5  # logits given: prep, no router launch
+    assert moe.launches(d) == 6  # logits given: prep, no router launch
     d = _desc(T=64, path="small")
     assert moe.select_path(d) == "small"
     assert _fwd(d, ws=FAKE * 8, ws_bytes=moe.workspace_size(d)) == moe.MOE_ERR_UNSUPPORTED
@@ -207,12 +207,12 @@ def test_kernel_plan_lists_the_launches_in_order():
     assert moe.kernel_plan(_desc(T=4096)) == ["prep", "router", "topk", "permute", "fc1", "fc2", "finalize"]
     assert moe.kernel_plan(_desc(T=4096, E=512, top_k=10)) == ["prep", "router", "topk", "refine", "select",
                                                               "permute", "fc1", "fc2", "finalize"]
-    assert moe.kernel_plan(_desc(T=64, path="large")) == ["router", "topk", "permute", "fc1", "fc2"]
+    assert moe.kernel_plan(_desc(T=64, path="large")) == ["router", "topk", "permute", "fc1", "fc2", "finalize"]
     assert moe.kernel_plan(_desc(T=65, path="large")) == ["prep", "router", "topk", "permute", "fc1", "fc2",
                                                          "finalize"]
     d = _desc(T=16, path="large")
     d.router_logits = FAKE * 8
-    assert moe.kernel_plan(d) == ["prep", "topk", "permute", "fc1", "fc2"]
+    assert moe.kernel_plan(d) == ["prep", "topk", "permute", "fc1", "fc2", "finalize"]
     for T in (1, 16, 64, 300, 4096):
         d = _desc(T=T, path="large")
         assert len(moe.kernel_plan(d)) == moe.launches(d)
