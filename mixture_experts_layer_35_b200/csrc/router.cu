@@ -60,6 +60,9 @@ __device__ __forceinline__ void shared_gate_row(const GateArgs& g, int row, int 
 __global__ void __launch_bounds__(256) prep_kernel(int* __restrict__ counters, int n, const bf16* __restrict__ wr,
                                                    int E, int H, float* __restrict__ wpart,
                                                    const bf16* __restrict__ x, int T, float* __restrict__ xn2) {
+    // The router GEMM that follows reads nothing written here and waits for this kernel
+    // only at its end: let it start now and run alongside.
+    pdl_trigger();
     const int tid = threadIdx.x, lane = tid & 31;
     if (blockIdx.x == 0)
         for (int i = tid; i < n; i += blockDim.x) counters[i] = 0;
@@ -85,7 +88,6 @@ __global__ void __launch_bounds__(256) prep_kernel(int* __restrict__ counters, i
             wpart[blockIdx.x] = m;
         }
     }
-    pdl_trigger();
 }
 
 int prep_grid(int E, int T, int num_sms) { return std::max(1, std::min(num_sms, cdiv(E + T, 8))); }
