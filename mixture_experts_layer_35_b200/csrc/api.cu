@@ -22,15 +22,15 @@ int num_sms() {
 
 // Workspace carve-up of moe_fused_forward, 256-byte aligned regions after the header.
 struct WsLayout {
-    size_t logits, route, topk_w, topk_ids, offsets, tiles1, tiles2, counts, wpart, xn2, perm, cand, h, hs, acc, skp,
-        gate, total;
+    size_t logits, route, topk_w, topk_ids, offsets, tiles1, tiles2, counts, perm, cand, h, hs, acc, done, wpart, xn2,
+        roweps, skp, gate, total;
 };
 // Candidate-list capacity per token of the three-kernel top-k (rows with more fall back).
 constexpr size_t kCandPerRow = 32;
 // Counters zeroed at the start of each many-token call (by its first kernel): per-expert
-// counts, per-expert cursors, the candidate count, then FC1's stream-K per-tile counters.
-inline size_t counter_ints(size_t E) { return 2 * (E + 2) + 4 + kStreamKMaxTiles; }
-inline size_t done_int(size_t E) { return 2 * (E + 2) + 4; }
+// counts, per-expert cursors, the candidate count; and, in a region of their own, FC1's
+// stream-K per-tile counters.
+inline size_t counter_ints(size_t E) { return 2 * (E + 2) + 4; }
 inline size_t cand_count_int(size_t E) { return 2 * (E + 2); }
 // Per-CTA router weight-norm bounds of the prep kernel (one per SM at most).
 constexpr size_t kMaxPrepGrid = 1024;
@@ -52,13 +52,16 @@ WsLayout layout(const moe_layer_desc* d) {
     L.tiles1 = take((E + 2) * 4);
     L.tiles2 = take((E + 2) * 4);
     L.counts = take(counter_ints(E) * 4);
-    L.wpart = take(kMaxPrepGrid * 4);
-    L.xn2 = take(T * 4);
     L.perm = take(T * K * 4);
-    L.cand = take(T * (3 + 3 * kCandPerRow) * 4);  // row_base, row_n, row_eps, cand_row, cand_e, cand_val
+    L.cand = take(T * (2 + 3 * kCandPerRow) * 4);  // row_base, row_n, cand_row, cand_e, cand_val
     L.h = take(T * K * I * 2);
     L.hs = take(T * Is * 2);
     L.acc = take(T * H * 4 * (Is ? 2 : 1));  // routed sum, then the shared expert's (FP32)
+    // Small regions after the large ones, so that the large buffers keep their offsets.
+    L.done = take((size_t)kStreamKMaxTiles * 4);
+    L.wpart = take(kMaxPrepGrid * 4);
+    L.xn2 = take(T * 4);
+    L.roweps = take(T * 4);
     const int fc1_mode = d->act == MOE_ACT_SWIGLU ? GM_FC1_SWIGLU : GM_FC1_RELU2;
     L.skp = take(fc1_streamk_bytes(gemm_token_tile(fc1_mode, d->T, d->top_k, d->E), d->act == MOE_ACT_SWIGLU,
                                    num_sms()));
@@ -385,6 +388,7 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
     if (path == MOE_PATH_LARGE && prep_kernel_for(d)) {
         if (!mark()) return MOE_ERR_CUDA;
         MOE_CK(launch_prep(reinterpret_cast<int*>(w8 + L.counts), (int)counter_ints(E),
+                           reinterpret_cast<int*>(w8 + L.done), kStreamKMaxTiles,
                            dense_router ? static_cast<const bf16*>(d->router_w) : nullptr, E, H, wpart, x, T,
                            reinterpret_cast<float*>(w8 + L.xn2), sms, s));
         pdl = !timed;
@@ -398,9 +402,11 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
         if (!mark()) return MOE_ERR_CUDA;
         if (!dense_router && T <= 64 && router_small_supported(H)) {
             // the many-token path without a prep kernel: this first kernel zeroes the counters
-            int* zc = path == MOE_PATH_LARGE ? reinterpret_cast<int*>(w8 + L.counts) : nullptr;
+            const bool lp = path == MOE_PATH_LARGE;
             MOE_CK(launch_router_small(x, static_cast<const bf16*>(d->router_w), T, H, E, lg, nullptr, err, s, pdl,
-                                       zc, zc ? (int)counter_ints(E) : 0));
+                                       lp ? reinterpret_cast<int*>(w8 + L.counts) : nullptr,
+                                       lp ? (int)counter_ints(E) : 0, lp ? reinterpret_cast<int*>(w8 + L.done) : nullptr,
+                                       lp ? kStreamKMaxTiles : 0));
         } else {
             st = run_router_dense(d, x, lg, nullptr, sms, s, err, pdl);
             if (st != MOE_OK) return st;
@@ -478,8 +484,8 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
         cl.count = counts + cand_count_int(E);
         cl.row_base = cbase;
         cl.row_n = cbase + T;
-        cl.row_eps = reinterpret_cast<float*>(cbase + 2 * (size_t)T);
-        cl.cand_row = cbase + 3 * (size_t)T;
+        cl.row_eps = reinterpret_cast<float*>(w8 + L.roweps);
+        cl.cand_row = cbase + 2 * (size_t)T;
         cl.cand_e = cl.cand_row + kCandPerRow * (size_t)T;
         cl.cand_val = reinterpret_cast<float*>(cl.cand_e + kCandPerRow * (size_t)T);
         cl.cap = (int)(kCandPerRow * (size_t)T);
@@ -556,7 +562,7 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
     };
     g1.streamk_max = gemm_streamk_max(fc1_mode, bn1, sms, max_tiles(bn1, g1.nfeat_r, Is ? g1.nfeat_s : 0));
     g1.skp = reinterpret_cast<float*>(w8 + L.skp);
-    g1.done = counts + done_int(E);
+    g1.done = reinterpret_cast<int*>(w8 + L.done);
     g1.err = err;
     if (!mark()) return MOE_ERR_CUDA;
     MOE_CK(launch_gemm(fc1_mode, bn1, g1, m1, sms, s, chain));

@@ -464,17 +464,17 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
                 mw[ci] = 0.0f;
                 const int colm = 32 * half + 32 * nhalf * ci + lane;
                 if (MODE == GM_FC2 && !ti.shared && colm < ti.n && ti.row0 + ti.n <= a.T * a.K) {
-                    const int src = a.perm[ti.row0 + colm];
+                    const int src = ld_nc_pinned_s32(a.perm + ti.row0 + colm);
                     if ((unsigned)src < (unsigned)(a.T * a.K)) {
                         const int kk = src / a.T;
                         mt[ci] = src - kk * a.T;
-                        mw[ci] = a.topk_w[(size_t)mt[ci] * a.K + kk];
+                        mw[ci] = ld_nc_pinned_f32(a.topk_w + (size_t)mt[ci] * a.K + kk);
                     } else {  // never from a valid permutation: flag it, contribute nothing
                         set_dev_error(a.err, MOE_DEVERR_BAD_INDEX);
                     }
                 } else if (MODE == GM_FC2 && ti.shared && colm < ti.n) {
                     mt[ci] = ti.row0 + colm;
-                    mw[ci] = a.sgate ? a.sgate[mt[ci]] : 1.0f;
+                    mw[ci] = a.sgate ? ld_nc_pinned_f32(a.sgate + mt[ci]) : 1.0f;
                 }
             }
             const bool waited = mbar_wait(tfull_bar(buf), tph, abort_flag, a.err);

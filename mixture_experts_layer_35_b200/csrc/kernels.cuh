@@ -67,10 +67,11 @@ cudaError_t launch_topk_split(const float* logits, int M, int E, int K, int scor
                               const RefineArgs& ra, int* counts, int* err, int num_sms, cudaStream_t s, bool pdl,
                               const std::function<bool()>* mark, const GateArgs& gate);
 bool router_small_supported(int H);
-// zero_ints (optional, n_zero ints): counters the kernel zeroes as a call's first kernel.
+// zero_ints / zero_ints2 (optional, n_zero / n_zero2 ints): counters the kernel zeroes as a
+// call's first kernel.
 cudaError_t launch_router_small(const bf16* x, const bf16* wr, int T, int H, int E, float* logits,
                                 float* logits_copy, int* err, cudaStream_t s, bool pdl, int* zero_ints = nullptr,
-                                int n_zero = 0);
+                                int n_zero = 0, int* zero_ints2 = nullptr, int n_zero2 = 0);
 
 // ---------------------------------------------------------------- few-token path
 static constexpr int kSmallMaxT = 16;
@@ -112,12 +113,12 @@ bool small_path_supported(int T, int H, int I, int Is);
 cudaError_t launch_small(const SmallArgs& a, int num_sms, cudaStream_t s, bool pdl_first,
                          const std::function<bool()>* mark);
 
-// First kernel of a many-token call: zeroes the call's counters (n ints) and, when wr is
+// First kernel of a many-token call: zeroes the call's counters (n and n2 ints) and, when wr is
 // given, writes per-CTA upper bounds of max_e |wr[e]|_2^2 into wpart[prep_grid(E, T, sms)]
 // and upper bounds of |x_t|_2^2 into xn2[T] (the bound on the tensor-core router's error).
 int prep_grid(int E, int T, int num_sms);
-cudaError_t launch_prep(int* counters, int n, const bf16* wr, int E, int H, float* wpart, const bf16* x, int T,
-                        float* xn2, int num_sms, cudaStream_t s);
+cudaError_t launch_prep(int* counters, int n, int* counters2, int n2, const bf16* wr, int E, int H, float* wpart,
+                        const bf16* x, int T, float* xn2, int num_sms, cudaStream_t s);
 
 // ---------------------------------------------------------------- permutation
 // Tile bookkeeping that the permute kernel writes for the grouped GEMMs (group g < E is

@@ -73,6 +73,18 @@ __device__ __forceinline__ uint4 ld_stream16(const void* p) {
     return r;
 }
 __device__ __forceinline__ uint4 ld_nc16(const void* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
+// Read-only 4-byte loads that stay where they are written (volatile asm is not moved past
+// other volatile asm such as a barrier wait), so that a load issued before a wait overlaps it.
+__device__ __forceinline__ int ld_nc_pinned_s32(const int* p) {
+    int v;
+    asm volatile("ld.global.nc.s32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+__device__ __forceinline__ float ld_nc_pinned_f32(const float* p) {
+    float v;
+    asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(v) : "l"(p));
+    return v;
+}
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll

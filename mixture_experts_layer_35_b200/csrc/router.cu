@@ -57,15 +57,18 @@ __device__ __forceinline__ void shared_gate_row(const GateArgs& g, int row, int 
 // upper bound.  Each CTA's maximum over router rows goes to wpart[blockIdx.x] (consumers
 // take the maximum over the grid's entries: no atomics, nothing to zero first); a token
 // row's bound goes to xn2[t].
-__global__ void __launch_bounds__(256) prep_kernel(int* __restrict__ counters, int n, const bf16* __restrict__ wr,
-                                                   int E, int H, float* __restrict__ wpart,
-                                                   const bf16* __restrict__ x, int T, float* __restrict__ xn2) {
+__global__ void __launch_bounds__(256) prep_kernel(int* __restrict__ counters, int n, int* __restrict__ counters2,
+                                                   int n2, const bf16* __restrict__ wr, int E, int H,
+                                                   float* __restrict__ wpart, const bf16* __restrict__ x, int T,
+                                                   float* __restrict__ xn2) {
     // The router GEMM that follows reads nothing written here and waits for this kernel
     // only at its end: let it start now and run alongside.
     pdl_trigger();
     const int tid = threadIdx.x, lane = tid & 31;
-    if (blockIdx.x == 0)
+    if (blockIdx.x == 0) {
         for (int i = tid; i < n; i += blockDim.x) counters[i] = 0;
+        for (int i = tid; i < n2; i += blockDim.x) counters2[i] = 0;
+    }
     if (wr) {
         __shared__ float s_max[8];
         float m = 0.0f;
@@ -92,10 +95,10 @@ __global__ void __launch_bounds__(256) prep_kernel(int* __restrict__ counters, i
 
 int prep_grid(int E, int T, int num_sms) { return std::max(1, std::min(num_sms, cdiv(E + T, 8))); }
 
-cudaError_t launch_prep(int* counters, int n, const bf16* wr, int E, int H, float* wpart, const bf16* x, int T,
-                        float* xn2, int num_sms, cudaStream_t s) {
-    return launch_k(prep_kernel, dim3(prep_grid(E, wr ? T : 0, num_sms)), dim3(256), 0, s, false, counters, n, wr, E,
-                    H, wpart, x, T, xn2);
+cudaError_t launch_prep(int* counters, int n, int* counters2, int n2, const bf16* wr, int E, int H, float* wpart,
+                        const bf16* x, int T, float* xn2, int num_sms, cudaStream_t s) {
+    return launch_k(prep_kernel, dim3(prep_grid(E, wr ? T : 0, num_sms)), dim3(256), 0, s, false, counters, n,
+                    counters2, n2, wr, E, H, wpart, x, T, xn2);
 }
 
 // Upper bound of max_e |Wr[e]|_2^2 from the prep kernel's per-CTA maxima (warp-collective).
@@ -547,14 +550,17 @@ template <int VH>
 __global__ void __launch_bounds__(64) router_logits_small(const bf16* __restrict__ x, const bf16* __restrict__ wr,
                                                           int T, int H, int E, float* __restrict__ logits,
                                                           float* __restrict__ logits_copy, int* err,
-                                                          int* __restrict__ zero_ints, int n_zero) {
+                                                          int* __restrict__ zero_ints, int n_zero,
+                                                          int* __restrict__ zero_ints2, int n_zero2) {
     extern __shared__ uint4 xs[];  // [kRouterTokBlock][H / 8]
     __shared__ __align__(8) uint64_t s_bar;
     __shared__ int s_abort;
     const int tid = threadIdx.x, lane = tid & 31;
     // As the first kernel of a many-token call, CTA (0, 0) also zeroes the call's counters.
-    if (zero_ints && blockIdx.x == 0 && blockIdx.y == 0)
+    if (zero_ints && blockIdx.x == 0 && blockIdx.y == 0) {
         for (int i = tid; i < n_zero; i += blockDim.x) zero_ints[i] = 0;
+        for (int i = tid; i < n_zero2; i += blockDim.x) zero_ints2[i] = 0;
+    }
     const uint32_t bar = smem_u32(&s_bar);
     if (tid == 0) {
         mbar_init(bar, 1);
@@ -621,7 +627,8 @@ __global__ void __launch_bounds__(64) router_logits_small(const bf16* __restrict
 bool router_small_supported(int H) { return (H >> 3) <= 32 * 16; }
 
 cudaError_t launch_router_small(const bf16* x, const bf16* wr, int T, int H, int E, float* logits,
-                                float* logits_copy, int* err, cudaStream_t s, bool pdl, int* zero_ints, int n_zero) {
+                                float* logits_copy, int* err, cudaStream_t s, bool pdl, int* zero_ints, int n_zero,
+                                int* zero_ints2, int n_zero2) {
     dim3 grid(cdiv(E, 2), cdiv(T, kRouterTokBlock)), block(64);
     const size_t smem = (size_t)kRouterTokBlock * H * 2;
     const int need = cdiv(H >> 3, 32);
@@ -631,7 +638,7 @@ cudaError_t launch_router_small(const bf16* x, const bf16* wr, int T, int H, int
                                                (int)smem);                                                       \
         if (st != cudaSuccess) return st;                                                                        \
         return launch_k(router_logits_small<VV>, grid, block, smem, s, pdl, x, wr, T, H, E, logits, logits_copy, err, \
-                        zero_ints, n_zero);                                                                      \
+                        zero_ints, n_zero, zero_ints2, n_zero2);                                                 \
     }
     MOE_R(4) MOE_R(8) MOE_R(12) MOE_R(16)
 #undef MOE_R
