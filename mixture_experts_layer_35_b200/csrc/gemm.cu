@@ -261,11 +261,375 @@ __device__ __forceinline__ void combine_chunk(const uint32_t (&v)[32], int mt, f
     }
 }
 
-// SK: the stream-K variant (the host launches it for calls with few tiles per SM); the
-// other variant deals whole tiles only, and compiles without the stream-K bookkeeping.
-template <int MODE, int BN, bool SK>
+// Whole tiles dealt round-robin over persistent CTAs (every call except few-token ones,
+// which take gemm_sk_kernel below).
+template <int MODE, int BN>
 __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
     gemm_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ CUtensorMap tm_a_s,
+                const __grid_constant__ CUtensorMap tm_b_r, const __grid_constant__ CUtensorMap tm_b_s) {
+    using C = Cfg<MODE, BN>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_u32 = smem_u32(smem_raw);
+    const uint32_t base_u32 = (raw_u32 + 1023u) & ~1023u;
+    uint8_t* base = smem_raw + (base_u32 - raw_u32);
+    uint8_t* meta = base + (size_t)C::kStages * C::kStageBytes + C::kEpiBytes;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(meta);  // full[S], empty[S], tfull[2], tempty[2]
+    const uint32_t bar_u32 = smem_u32(bars);
+    auto full_bar = [&](int s) { return bar_u32 + 8u * s; };
+    auto empty_bar = [&](int s) { return bar_u32 + 8u * (C::kStages + s); };
+    auto tfull_bar = [&](int b) { return bar_u32 + 8u * (2 * C::kStages + b); };
+    auto tempty_bar = [&](int b) { return bar_u32 + 8u * (2 * C::kStages + 2 + b); };
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(meta + 8 * (2 * C::kStages + 4));
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int* s_tiles = reinterpret_cast<int*>(meta + 256);
+    int* s_offs = s_tiles + C::kMaxGroups + 1;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int G = a.E + (a.has_shared ? 1 : 0);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(full_bar(s), 1 + C::kGatherThreads);
+            mbar_init(empty_bar(s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(tfull_bar(b), 1);
+            mbar_init(tempty_bar(b), C::kEpiWarps);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tm_a_r);
+        if (a.has_shared) tma_prefetch_desc(&tm_a_s);
+        if (!C::kGather) {
+            tma_prefetch_desc(&tm_b_r);
+            if (a.has_shared) tma_prefetch_desc(&tm_b_s);
+        }
+    }
+    if (warp == 1) tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+
+    // Everything below reads what earlier kernels wrote (tile tables, perm, h) -- except
+    // in DENSE mode, which reads only the caller's x and Wr and waits at its end.
+    if (MODE != GM_DENSE) pdl_wait();
+    if (!a.dense) {
+        for (int i = threadIdx.x; i <= G; i += blockDim.x) s_tiles[i] = a.tiles[i];
+        for (int i = threadIdx.x; i <= a.E; i += blockDim.x) s_offs[i] = a.offsets[i];
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int total = a.dense ? a.nfeat_r * cdiv(a.T, kDenseTokenTile) : s_tiles[G];
+    // Tiles are dealt round-robin over the persistent CTAs: at any moment the CTAs work on
+    // neighbouring tiles of the group-major list (one expert's feature and token tiles),
+    // which share that expert's weight rows and token rows in L2, and tiles of unequal
+    // cost (ragged token tails) spread evenly.
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            const uint64_t wpol = l2_policy_evict_first();
+            int it = 0;
+            for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
+                const TileInfo ti = decode_tile<C::kBN>(a, s_tiles, s_offs, G, tile);
+                const bool sh = ti.shared;
+                const CUtensorMap* ta = sh ? &tm_a_s : &tm_a_r;
+                const CUtensorMap* tb = sh ? &tm_b_s : &tm_b_r;
+                const int frow = ti.ft * BM;
+                constexpr int BBOX = b_box_rows<MODE>();
+                const int nbox = cdiv(ti.n, BBOX);
+                const uint32_t bytes = C::kNA * A_BYTES + (C::kGather ? 0u : (uint32_t)nbox * BBOX * BK * 2);
+                for (int kb = 0; kb < ti.nk; ++kb, ++it) {
+                    const int s = it % C::kStages;
+                    const uint32_t ph = (uint32_t)(it / C::kStages) & 1u;
+                    if (!mbar_wait(empty_bar(s), ph ^ 1u, abort_flag, a.err)) break;
+                    const uint32_t st = base_u32 + (uint32_t)s * C::kStageBytes;
+                    mbar_expect_tx(full_bar(s), bytes);
+                    if (sh || a.dense) {
+                        tma_load_2d(st, ta, full_bar(s), kb * BK, frow);
+                        if (C::kSwiglu) tma_load_2d(st + A_BYTES, ta, full_bar(s), kb * BK, a.up_s + frow);
+                    } else if (MODE == GM_FC2 || ti.ntok == 1) {
+                        // Weights that no other tile of this call reads: evict first, so that
+                        // they do not push the token rows, h and the accumulator out of L2
+                        // (measured on FC1: -9 % at 16 tokens, -6 % at 4096 tokens of the
+                        // Qwen3.6-shaped layer).
+                        tma_load_3d_hint(st, ta, full_bar(s), kb * BK, frow, ti.g, wpol);
+                        if (C::kSwiglu)
+                            tma_load_3d_hint(st + A_BYTES, ta, full_bar(s), kb * BK, a.up_r + frow, ti.g, wpol);
+                    } else {  // a second token tile of this expert streams the same slice
+                        tma_load_3d(st, ta, full_bar(s), kb * BK, frow, ti.g);
+                        if (C::kSwiglu) tma_load_3d(st + A_BYTES, ta, full_bar(s), kb * BK, a.up_r + frow, ti.g);
+                    }
+                    if (!C::kGather) {
+                        const uint32_t bs = st + C::kNA * A_BYTES;
+                        for (int q = 0; q < nbox; ++q)
+                            tma_load_2d(bs + (uint32_t)q * (BBOX * BK * 2), tb, full_bar(s), kb * BK,
+                                        ti.row0 + q * BBOX);
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int it = 0, tcount = 0;
+            for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x, ++tcount) {
+                const TileInfo ti = decode_tile<C::kBN>(a, s_tiles, s_offs, G, tile);
+                const int nk = ti.nk;
+                const int npad = cdiv(ti.n, 16) * 16;
+                const uint32_t idesc = idesc_bf16_f32(BM, npad);
+                const int buf = tcount % C::kAccBufs;
+                const uint32_t tph = (uint32_t)(tcount / C::kAccBufs) & 1u;
+                if (!mbar_wait(tempty_bar(buf), tph ^ 1u, abort_flag, a.err)) break;
+                tc_fence_after();
+                const uint32_t d0 = tmem_base + (uint32_t)(buf * C::kAccStride);
+                const uint32_t d1 = d0 + C::kBN;
+                bool ok = true;
+                for (int kb = 0; kb < nk; ++kb, ++it) {
+                    const int s = it % C::kStages;
+                    const uint32_t ph = (uint32_t)(it / C::kStages) & 1u;
+                    if (!mbar_wait(full_bar(s), ph, abort_flag, a.err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t st = base_u32 + (uint32_t)s * C::kStageBytes;
+                    const uint32_t bsm = st + C::kNA * A_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
+                        const uint64_t bdesc = sdesc_sw128(bsm + kk * 32);
+                        tc_mma(d0, sdesc_sw128(st + kk * 32), bdesc, idesc, accum);
+                        if (C::kSwiglu) tc_mma(d1, sdesc_sw128(st + A_BYTES + kk * 32), bdesc, idesc, accum);
+                    }
+                    tc_commit(empty_bar(s));
+                }
+                if (!ok) break;
+                tc_commit(tfull_bar(buf));
+            }
+        }
+    } else if (warp < 2 + C::kEpiWarps) {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;                     // TMEM lane quarter of this warp
+        const int half = (warp - 2) >> 2;          // FC2: which token columns (chunk parity)
+        const int nhalf = C::kEpiWarps / 4;
+        const int et = threadIdx.x - 64;
+        if (a.zero_ptr) {
+            float4* z = reinterpret_cast<float4*>(a.zero_ptr);
+            const size_t n4 = a.zero_n / 4;
+            const int ne = 32 * C::kEpiWarps;
+            for (size_t i = (size_t)blockIdx.x * ne + et; i < n4; i += (size_t)gridDim.x * ne)
+                z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        int tcount = 0;
+        // (the abort flag is checked through the per-tile wait below)
+        // 32-token chunks per half of the epilogue warps (the last may lie past the tile)
+        constexpr int kChunks = (C::kBN + 32 * (C::kEpiWarps / 4) - 1) / (32 * (C::kEpiWarps / 4));
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++tcount) {
+            const TileInfo ti = decode_tile<C::kBN>(a, s_tiles, s_offs, G, tile);
+            const int buf = tcount % C::kAccBufs;
+            const uint32_t tph = (uint32_t)(tcount / C::kAccBufs) & 1u;
+            // FC2: token and routing weight of each column this thread will scale, loaded
+            // before the accumulator is ready (hidden behind the tile's mainloop).
+            int mt[kChunks];
+            float mw[kChunks];
+#pragma unroll
+            for (int ci = 0; ci < kChunks; ++ci) {
+                mt[ci] = 0;
+                mw[ci] = 0.0f;
+                const int colm = 32 * half + 32 * nhalf * ci + lane;
+                if (MODE == GM_FC2 && !ti.shared && colm < ti.n && ti.row0 + ti.n <= a.T * a.K) {
+                    const int src = a.perm[ti.row0 + colm];
+                    if ((unsigned)src < (unsigned)(a.T * a.K)) {
+                        const int kk = src / a.T;
+                        mt[ci] = src - kk * a.T;
+                        mw[ci] = a.topk_w[(size_t)mt[ci] * a.K + kk];
+                    } else {  // never from a valid permutation: flag it, contribute nothing
+                        set_dev_error(a.err, MOE_DEVERR_BAD_INDEX);
+                    }
+                }
+            }
+            const bool waited = mbar_wait(tfull_bar(buf), tph, abort_flag, a.err);
+            if (!waited) break;
+            tc_fence_after();
+            // The tile's rows must lie inside their buffer (they do for any permutation the
+            // permute kernel writes); otherwise flag it and store nothing for this tile.
+            const bool rows_ok = a.dense || ti.row0 + ti.n <= (ti.shared ? a.T : a.T * a.K);
+            if (!rows_ok && lane == 0) set_dev_error(a.err, MOE_DEVERR_BAD_INDEX);
+            const int f = ti.ft * BM + q * 32 + lane;
+            const int feat = ti.shared ? a.feat_s : a.feat_r;
+            const bool fok = f < feat;
+            const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * C::kAccStride);
+#pragma unroll
+            for (int ci = 0; ci < kChunks; ++ci) {
+                const int c0 = 32 * half + 32 * nhalf * ci;
+                if (c0 >= ti.n || !rows_ok) break;
+                uint32_t v[32];
+                tmem_ld32(tb + c0, v);
+                uint32_t u[32];
+                if (C::kSwiglu) tmem_ld32(tb + C::kBN + c0, u);
+                tmem_ld_wait();
+                if (C::kGather) {
+                    bf16* dst = ti.shared ? a.hs : a.h;
+                    const int ld = feat;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int col = c0 + j;
+                        if (col < ti.n && fok) {
+                            float val;
+                            if (C::kSwiglu) val = act_swiglu(__uint_as_float(v[j]), __uint_as_float(u[j]));
+                            else val = act_relu2(__uint_as_float(v[j]));
+                            dst[(size_t)(ti.row0 + col) * ld + f] = __float2bfloat16_rn(val);
+                        }
+                    }
+                } else if (MODE == GM_FC2) {
+                    if (ti.shared) {  // shared rows are the tokens in order; optional sigmoid gate
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const int col = c0 + j;
+                            if (col < ti.n && fok) {
+                                float y = __uint_as_float(v[j]);
+                                if (a.sgate) y = __fmul_rn(a.sgate[ti.row0 + col], y);
+                                a.acc_s[(size_t)(ti.row0 + col) * a.feat_s + f] = y;
+                            }
+                        }
+                    } else {
+                        // Column j of this chunk is token t_j with routing weight w_j; lane l
+                        // holds feature f0 + l.  Each block of 4 columns is transposed within
+                        // groups of 4 lanes (two XOR-shuffle stages), after which lane 4g+i
+                        // holds features f0+4g .. f0+4g+3 of token t_{j0+i}, scales them by
+                        // w_{j0+i} (one shuffle brings the token, one the weight) and adds
+                        // them into acc with one 16-byte vector reduction (FP32 add in L2).
+                        // No shared memory is staged, so the ring keeps it for weights.
+                        const int i4 = lane & 3;
+                        const bool fok4 = f - i4 + 3 < a.feat_r;  // features of my group (feat_r % 8 == 0)
+#pragma unroll
+                        for (int j0 = 0; j0 < 32; j0 += 4) {
+                            float r[4];
+#pragma unroll
+                            for (int jj = 0; jj < 4; ++jj) r[jj] = __uint_as_float(v[j0 + jj]);
+                            // r[jj] = y[feature of this lane, token j0 + jj]; 4x4 transpose
+                            float t0 = (i4 & 1) ? r[0] : r[1], t1 = (i4 & 1) ? r[2] : r[3];
+                            t0 = __shfl_xor_sync(0xffffffffu, t0, 1);
+                            t1 = __shfl_xor_sync(0xffffffffu, t1, 1);
+                            if (i4 & 1) {
+                                r[0] = t0;
+                                r[2] = t1;
+                            } else {
+                                r[1] = t0;
+                                r[3] = t1;
+                            }
+                            float u0 = (i4 & 2) ? r[0] : r[2], u1 = (i4 & 2) ? r[1] : r[3];
+                            u0 = __shfl_xor_sync(0xffffffffu, u0, 2);
+                            u1 = __shfl_xor_sync(0xffffffffu, u1, 2);
+                            if (i4 & 2) {
+                                r[0] = u0;
+                                r[1] = u1;
+                            } else {
+                                r[2] = u0;
+                                r[3] = u1;
+                            }
+                            const int tok = __shfl_sync(0xffffffffu, mt[ci], j0 + i4);
+                            const float wt = __shfl_sync(0xffffffffu, mw[ci], j0 + i4);
+                            if (c0 + j0 + i4 < ti.n && fok4 && (unsigned)tok < (unsigned)a.T)
+                                red_add_v4_f32(a.acc + (size_t)tok * a.feat_r + (f - i4), wt * r[0], wt * r[1],
+                                               wt * r[2], wt * r[3]);
+                        }
+                    }
+                } else {  // GM_DENSE
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int col = c0 + j;
+                        if (col < ti.n && fok) {
+                            const float val = __uint_as_float(v[j]);
+                            a.logits[(size_t)(ti.row0 + col) * a.feat_r + f] = val;
+                            if (a.logits_copy) a.logits_copy[(size_t)(ti.row0 + col) * a.feat_r + f] = val;
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tempty_bar(buf));
+        }
+    } else if (C::kGather) {
+        // ------------------------------------------------------------ FC1 token gather
+        const int p = threadIdx.x - (64 + 32 * C::kEpiWarps);  // 0 .. kGatherThreads - 1
+        const int chunk = p & 7, rsub = p >> 3;
+        int it = 0;
+        for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
+            const TileInfo ti = decode_tile<C::kBN>(a, s_tiles, s_offs, G, tile);
+            const int kd = ti.shared ? a.kdim_s : a.kdim;
+            const int nk = ti.nk;
+            const int npad = cdiv(ti.n, 16) * 16;
+            int tok[C::kBN / C::kGatherRowStep];
+#pragma unroll
+            for (int j = 0; j < C::kBN / C::kGatherRowStep; ++j) {
+                const int r = rsub + C::kGatherRowStep * j;
+                tok[j] = -1;
+                if (r < ti.n && (ti.shared || ti.row0 + ti.n <= a.T * a.K)) {
+                    const int src = ti.shared ? ti.row0 + r : a.perm[ti.row0 + r];
+                    if ((unsigned)src < (unsigned)(ti.shared ? a.T : a.T * a.K)) {
+                        tok[j] = ti.shared ? src : src % a.T;
+                    } else {  // never from a valid permutation: flag it, gather zeros
+                        set_dev_error(a.err, MOE_DEVERR_BAD_INDEX);
+                    }
+                }
+            }
+            bool ok = true;
+            for (int kb = 0; kb < nk; ++kb, ++it) {
+                const int s = it % C::kStages;
+                const uint32_t ph = (uint32_t)(it / C::kStages) & 1u;
+                if (!mbar_wait(empty_bar(s), ph ^ 1u, abort_flag, a.err)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t bs = base_u32 + (uint32_t)s * C::kStageBytes + C::kNA * A_BYTES;
+                const int kcol = kb * BK + chunk * 8;
+#pragma unroll
+                for (int j = 0; j < C::kBN / C::kGatherRowStep; ++j) {
+                    const int r = rsub + C::kGatherRowStep * j;
+                    if (r < npad) {
+                        const uint32_t dst = bs + (uint32_t)r * 128u + ((uint32_t)(chunk ^ (r & 7)) << 4);
+                        const bool v = tok[j] >= 0 && kcol < kd;
+                        const bf16* src = v ? a.xsrc + (size_t)tok[j] * a.kdim + kcol : a.xsrc;
+                        cp_async16(dst, src, v ? 16u : 0u);
+                    }
+                }
+                cp_async_commit();
+                if (it >= C::kLag) {
+                    cp_async_wait<C::kLag>();
+                    fence_proxy_async_smem();
+                    mbar_arrive(full_bar((it - C::kLag) % C::kStages));
+                }
+            }
+            if (!ok) break;
+        }
+        cp_async_wait<0>();
+        fence_proxy_async_smem();
+        for (int j = max(0, it - C::kLag); j < it; ++j) mbar_arrive(full_bar(j % C::kStages));
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (*abort_flag) {  // let in-flight bulk copies and MMAs land before the CTA retires
+        const uint64_t t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 50000ull) {
+        }
+    }
+    if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
+    if (MODE == GM_DENSE) pdl_wait();  // the previous kernel is complete before this one is
+    pdl_trigger();
+}
+
+// The stream-K kernel, launched for few-token calls (FC1 token tiles of 32 or 64 rows, FC2
+// of 32 or 128): it decides on the device, from the call's tile count, between stream-K
+// and whole tiles.  SK is always true here; it keeps the walker's whole-tile path compiled.
+template <int MODE, int BN, bool SK>
+__global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
+    gemm_sk_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ CUtensorMap tm_a_s,
                 const __grid_constant__ CUtensorMap tm_b_r, const __grid_constant__ CUtensorMap tm_b_s) {
     using C = Cfg<MODE, BN>;
     // FC1's stream-K fix-up keeps [kNA][BN][128] partial sums per CTA: BN <= 64 only.
@@ -733,22 +1097,24 @@ __global__ void __launch_bounds__(256) finalize_kernel(const float* __restrict__
 
 }  // namespace
 
-template <int MODE, int BN, bool SK>
-static cudaError_t launch_mode_sk(const GemmArgs& a, const GemmMaps& m, int grid, cudaStream_t s, bool pdl) {
-    using C = Cfg<MODE, BN>;
-    cudaError_t e =
-        cudaFuncSetAttribute(gemm_kernel<MODE, BN, SK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
+template <typename Kern>
+static cudaError_t launch_gemm_kernel(Kern kern, size_t smem, int threads, const GemmArgs& a, const GemmMaps& m,
+                                      int grid, cudaStream_t s, bool pdl) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    return launch_k(gemm_kernel<MODE, BN, SK>, dim3(grid), dim3(C::kThreads), C::kSmem, s, pdl, a, m.a_r, m.a_s,
-                    m.b_r, m.b_s);
+    return launch_k(kern, dim3(grid), dim3(threads), smem, s, pdl, a, m.a_r, m.a_s, m.b_r, m.b_s);
 }
-// The stream-K variant exists for the token tiles of few-token calls (32 and 64 rows for
-// FC1, 32 and 128 for FC2); a.streamk_max == 0 selects the whole-tile variant.
+// The stream-K kernel exists for the token tiles of few-token calls (32 and 64 rows for
+// FC1, 32 and 128 for FC2); a.streamk_max == 0 selects the whole-tile kernel.
 template <int MODE, int BN>
 static cudaError_t launch_mode(const GemmArgs& a, const GemmMaps& m, int grid, cudaStream_t s, bool pdl) {
+    using C = Cfg<MODE, BN>;
     constexpr bool kHasSK = MODE == GM_FC2 ? (BN == 32 || BN == 128) : (MODE != GM_DENSE && BN <= kStreamKMaxBN);
-    if (kHasSK && a.streamk_max > 0) return launch_mode_sk<MODE, BN, kHasSK>(a, m, grid, s, pdl);
-    return launch_mode_sk<MODE, BN, false>(a, m, grid, s, pdl);
+    if constexpr (kHasSK) {
+        if (a.streamk_max > 0)
+            return launch_gemm_kernel(gemm_sk_kernel<MODE, BN, true>, C::kSmem, C::kThreads, a, m, grid, s, pdl);
+    }
+    return launch_gemm_kernel(gemm_kernel<MODE, BN>, C::kSmem, C::kThreads, a, m, grid, s, pdl);
 }
 
 int gemm_token_tile(int mode, int T, int K, int E) {
