@@ -5,20 +5,22 @@
 
 namespace moe {
 
-// Error bound of the tensor-core router logits of one token row (warp-collective).
-// The MMA forms every BF16 x BF16 product exactly in FP32 and sums the H products of a
-// logit (zero padding included) in FP32.  Whatever the association order and whether
-// each addition rounds or truncates, as long as every addition step is within 2 units
-// in the last place of an FP32 result -- or, for a multi-operand adder that aligns up to
-// 17 addends to the largest one and truncates them, within one such unit per addend --
-// the computed logit lies within H * 2^-22 * sum_h |x_h w_h| of the exact sum.  Cauchy-
-// Schwarz bounds the sum by |x_t|_2 * max_e |Wr[e]|_2; the router GEMM supplies an upper
-// bound of max_e |Wr[e]|_2^2 and of every |x_t|_2^2 (FP32 sums of squares scaled up by
+// Error bound of the tensor-core router logits of one token row.  The MMA forms every
+// BF16 x BF16 product exactly in FP32 and accumulates a logit's H products (zero padding
+// included) sixteen at a time: each tcgen05.mma of K = 16 adds its 16 products to the
+// FP32 accumulator.  Model: one such step aligns its 17 addends to the largest and keeps
+// at least 24 significant bits of it, truncating the rest, then rounds or truncates the
+// sum to FP32 -- an error below 17 units of the largest addend plus one unit of the
+// result, i.e. below 18 * 2^-23 * (|C| + sum |p|) for accumulator C.  Over the H / 16
+// steps (each |C| <= sum_h |x_h w_h| =: S) the logit lies within 18 * 2^-23 * (H/16 + 1) * S
+// = 1.125 * 2^-23 * (H + 16) * S of the exact sum; 1.25 is taken for margin.  Cauchy-
+// Schwarz bounds S by |x_t|_2 * max_e |Wr[e]|_2; the prep kernel supplies upper bounds
+// of max_e |Wr[e]|_2^2 and of every |x_t|_2^2 (FP32 sums of squares scaled up by
 // (1 + 2^-8) to cover their own rounding, H <= 2^16).  A final factor (1 + 2^-8) covers the
-// roundings of this product.  The reduction length is padded to a multiple of 64.
+// roundings of this product.  Each re-evaluated logit is checked against the bound.
 __device__ __forceinline__ float tc_logit_bound(float xnorm2, int H, float wnorm2) {
     const float hpad = (float)(((H + 63) / 64) * 64);
-    return hpad * 0x1p-22f * sqrtf(xnorm2) * sqrtf(wnorm2) * (1.0f + 0x1p-8f);
+    return 1.25f * (hpad + 16.0f) * 0x1p-23f * sqrtf(xnorm2) * sqrtf(wnorm2) * (1.0f + 0x1p-8f);
 }
 
 // Exact re-evaluation of one candidate's logit (warp-collective), written back into the

@@ -1,7 +1,8 @@
 """Exact routing after the tensor-core router on activations far from N(0, 1).
 
 With more than 64 tokens the router logits come from a tensor-core GEMM whose FP32
-accumulation error is bounded per token by H * 2^-22 * |x_t|_2 * max_e |Wr[e]|_2; every
+accumulation error is bounded per token by about 1.25 * 2^-23 * (H + 16) * |x_t|_2 *
+max_e |Wr[e]|_2 (a per-instruction alignment-and-truncation model of the MMA); every
 expert whose key lies within twice that bound of the K-th key is re-evaluated exactly
 ("Laguna exact M=8 BF16-input router top-k preregistration", "Question and arithmetic
 contract": the selection is that of the exact FP32 logits).  The bound scales with the
