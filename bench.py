@@ -291,6 +291,16 @@ class Bench:
         self.last_step_s = statistics.median(per) / 1e3 + 2e-5
         return per, clk
 
+    def telemetry(self):
+        """Phase trace of one eager forward behind an L2 flush (moe_layer_desc.trace):
+        per tensor-core kernel, launch skew, input wait, load span, tail."""
+        trace = self.moe.trace_buffer(self.device)
+        desc = self.layer.desc(self.T, self.logits, trace=trace)
+        self.flush()
+        self.moe.fused_forward_raw(desc, self.d["x"], self.out, self.ws, stream=self.stream)
+        torch.cuda.synchronize(self.device)
+        return self.moe.trace_summary(trace, torch.cuda.get_device_properties(self.device).multi_processor_count)
+
     def clock_soak(self, seconds: float):
         """Clocks while the same step (L2 flush + graph replay) repeats back to back for
         about ``seconds``: a longer window than a short timed region gives the sampler."""
@@ -467,6 +477,7 @@ def run_ours(args, rank, local, world):
     e2e_serial = max_over_ranks(e2e_serial, world, device)
     e2e_value = world * args.T / (e2e_pipe / 1e3)
 
+    telem = b.telemetry() if b.path == "large" else None
     clk_soak = b.clock_soak(args.soak_s) if args.soak_s > 0 else None
     dev_err = b.moe.get_error(b.ws)
     line = {
@@ -482,6 +493,7 @@ def run_ours(args, rank, local, world):
         "roofline": roof,
         "layer_roofline": layer_roof,
         "kernel_ms": {n: round(float(v), 5) for n, v in zip(names, kt)},
+        "telemetry": telem,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo,
                 "timing": "public forward call per step, pinned H2D of x and D2H of out inside each step; "
                           "copy-in, forward and read-back on three streams with double buffers, steps "

@@ -156,7 +156,23 @@ typedef struct {
     float routed_scale;
     const void* shared_gate_w;
     const void* shared_out;
+    /* Optional phase trace (NULL = none): a device buffer of moe_trace_size() bytes that the
+     * tensor-core kernels of the many-token path fill, one block per kernel (MOE_TRACE_ROUTER,
+     * _FC1, _FC2), one row of MOE_TRACE_FIELDS 64-bit values per CTA: %globaltimer (ns) at
+     * kernel entry, when its inputs are ready (after the wait on the previous kernel and the
+     * tile tables), when its producer issued its last load, when its first epilogue warp
+     * finished, and at exit; and the number of work units (tiles, or stream-K segments) the
+     * CTA took.  Rows of CTAs a kernel did not launch, and blocks of kernels the call did
+     * not run, are left as they were.  16-byte aligned. */
+    unsigned long long* trace;
 } moe_layer_desc;
+
+enum { MOE_TRACE_ENTRY = 0, MOE_TRACE_READY = 1, MOE_TRACE_LOADS_DONE = 2, MOE_TRACE_STORES_DONE = 3,
+       MOE_TRACE_EXIT = 4, MOE_TRACE_UNITS = 5, MOE_TRACE_FIELDS = 8 };
+enum { MOE_TRACE_ROUTER = 0, MOE_TRACE_FC1 = 1, MOE_TRACE_FC2 = 2, MOE_TRACE_KERNELS = 3 };
+#define MOE_TRACE_MAX_CTAS 1024
+/* Bytes of the phase-trace buffer: MOE_TRACE_KERNELS blocks of MOE_TRACE_MAX_CTAS rows. */
+size_t moe_trace_size(void);
 
 /* Bytes of workspace moe_fused_forward needs for this description (either path). */
 size_t moe_workspace_size(const moe_layer_desc* d);

@@ -89,7 +89,7 @@ moe_status_t validate_desc(const moe_layer_desc* d) {
     if (d->shared_gate_w && d->I_shared == 0) return MOE_ERR_INVALID_ARG;
     if (d->shared_out && d->I_shared > 0) return MOE_ERR_INVALID_ARG;
     const void* ptrs[] = {d->router_w, d->router_logits, d->bias, d->w13, d->w2, d->ws13, d->ws2,
-                          d->shared_gate_w, d->shared_out};
+                          d->shared_gate_w, d->shared_out, d->trace};
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return MOE_ERR_INVALID_ARG;
     return MOE_OK;
@@ -170,6 +170,7 @@ moe_status_t run_router_dense(const moe_layer_desc* d, const bf16* x, float* log
     g.dense = 1;
     g.logits = logits;
     g.logits_copy = copy;
+    g.trace = d->trace ? d->trace + (size_t)MOE_TRACE_ROUTER * MOE_TRACE_MAX_CTAS * MOE_TRACE_FIELDS : nullptr;
     g.err = err;
     GemmMaps m;
     std::memset(&m, 0, sizeof(m));
@@ -271,6 +272,10 @@ size_t moe_workspace_size(const moe_layer_desc* d) {
 int moe_select_path(const moe_layer_desc* d) {
     if (validate_desc(d) != MOE_OK) return -1;
     return resolve_path(d);
+}
+
+size_t moe_trace_size(void) {
+    return (size_t)MOE_TRACE_KERNELS * MOE_TRACE_MAX_CTAS * MOE_TRACE_FIELDS * sizeof(unsigned long long);
 }
 
 moe_status_t moe_token_tiles(const moe_layer_desc* d, int* fc1_rows, int* fc2_rows) {
@@ -376,6 +381,7 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
     bf16* out = static_cast<bf16*>(out_);
     const int T = d->T, H = d->H, I = d->I, E = d->E, K = d->top_k, Is = d->I_shared;
     const int sms = num_sms();
+    if (d->trace && sms > MOE_TRACE_MAX_CTAS) return MOE_ERR_UNSUPPORTED;
     const float rscale = d->routed_scale == 0.0f ? 1.0f : d->routed_scale;
     const bf16* sh_out = static_cast<const bf16*>(d->shared_out);
 
@@ -552,6 +558,7 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
     g1.xsrc = x;
     g1.h = h;
     g1.hs = hs;
+    g1.trace = d->trace ? d->trace + (size_t)MOE_TRACE_FC1 * MOE_TRACE_MAX_CTAS * MOE_TRACE_FIELDS : nullptr;
     g1.zero_ptr = acc;
     g1.zero_n = (size_t)T * H * (Is ? 2 : 1);
     // Upper bound of a grouped GEMM's tiles: at most min(E, T*K) experts have rows, and each
@@ -585,6 +592,7 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
     g2.feat_r = H;
     g2.feat_s = H;
     g2.tiles = tiles2;
+    g2.trace = d->trace ? d->trace + (size_t)MOE_TRACE_FC2 * MOE_TRACE_MAX_CTAS * MOE_TRACE_FIELDS : nullptr;
     g2.acc = acc;
     g2.acc_s = acc_s;
     g2.sgate = gate;

@@ -286,6 +286,9 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = a.E + (a.has_shared ? 1 : 0);
+    // Phase trace (optional): this CTA's row of the kernel's trace block.
+    unsigned long long* trow = a.trace ? a.trace + (size_t)blockIdx.x * MOE_TRACE_FIELDS : nullptr;
+    if (trow && threadIdx.x == 0) trow[MOE_TRACE_ENTRY] = globaltimer_ns();
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kStages; ++s) {
@@ -319,6 +322,7 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    if (trow && threadIdx.x == 0) trow[MOE_TRACE_READY] = globaltimer_ns();
     const uint32_t tmem_base = *tmem_slot;
     const int total = a.dense ? a.nfeat_r * cdiv(a.T, kDenseTokenTile) : s_tiles[G];
     // Tiles are dealt round-robin over the persistent CTAs: at any moment the CTAs work on
@@ -368,6 +372,11 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
                                         ti.row0 + q * BBOX);
                     }
                 }
+            }
+            if (trow) {
+                trow[MOE_TRACE_LOADS_DONE] = globaltimer_ns();
+                trow[MOE_TRACE_UNITS] = (unsigned long long)((total - (int)blockIdx.x + (int)gridDim.x - 1) /
+                                                             (int)gridDim.x);
             }
         }
     } else if (warp == 1) {
@@ -553,6 +562,7 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(tempty_bar(buf));
         }
+        if (trow && threadIdx.x == 64) trow[MOE_TRACE_STORES_DONE] = globaltimer_ns();
     } else if (C::kGather) {
         // ------------------------------------------------------------ FC1 token gather
         const int p = threadIdx.x - (64 + 32 * C::kEpiWarps);  // 0 .. kGatherThreads - 1
@@ -619,6 +629,7 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
         while (globaltimer_ns() - t0 < 50000ull) {
         }
     }
+    if (trow && threadIdx.x == 0) trow[MOE_TRACE_EXIT] = globaltimer_ns();
     if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
     if (MODE == GM_DENSE) pdl_wait();  // the previous kernel is complete before this one is
     pdl_trigger();
@@ -652,6 +663,9 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = a.E + (a.has_shared ? 1 : 0);
+    // Phase trace (optional): this CTA's row of the kernel's trace block.
+    unsigned long long* trow = a.trace ? a.trace + (size_t)blockIdx.x * MOE_TRACE_FIELDS : nullptr;
+    if (trow && threadIdx.x == 0) trow[MOE_TRACE_ENTRY] = globaltimer_ns();
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kStages; ++s) {
@@ -685,6 +699,7 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    if (trow && threadIdx.x == 0) trow[MOE_TRACE_READY] = globaltimer_ns();
     const uint32_t tmem_base = *tmem_slot;
     const int total = a.dense ? a.nfeat_r * cdiv(a.T, kDenseTokenTile) : s_tiles[G];
     const int routed_tiles = (a.dense || !a.has_shared) ? total : s_tiles[a.E];
@@ -707,7 +722,7 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             const uint64_t wpol = l2_policy_evict_first();
-            int it = 0;
+            int it = 0, units = 0;
             while (!*abort_flag && work.next(sg)) {
                 const TileInfo ti = decode_tile<C::kBN>(a, s_tiles, s_offs, G, sg.tile);
                 if (ti.nk == 0) continue;
@@ -751,6 +766,11 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
                     }
                 }
                 if (!ok) break;
+                ++units;
+            }
+            if (trow) {
+                trow[MOE_TRACE_LOADS_DONE] = globaltimer_ns();
+                trow[MOE_TRACE_UNITS] = (unsigned long long)units;
             }
         }
     } else if (warp == 1) {
@@ -984,6 +1004,7 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
             if (lane == 0) mbar_arrive(tempty_bar(buf));
             ++tcount;
         }
+        if (trow && threadIdx.x == 64) trow[MOE_TRACE_STORES_DONE] = globaltimer_ns();
     } else if (C::kGather) {
         // ------------------------------------------------------------ FC1 token gather
         const int p = threadIdx.x - (64 + 32 * C::kEpiWarps);  // 0 .. kGatherThreads - 1
@@ -1050,6 +1071,7 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
         while (globaltimer_ns() - t0 < 50000ull) {
         }
     }
+    if (trow && threadIdx.x == 0) trow[MOE_TRACE_EXIT] = globaltimer_ns();
     if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
     if (MODE == GM_DENSE) pdl_wait();  // the previous kernel is complete before this one is
     pdl_trigger();

@@ -175,6 +175,7 @@ struct GemmArgs {
     float* zero_ptr;         // FC1: buffer zeroed by the epilogue warps before their tiles
     size_t zero_n;           //      (floats, multiple of 4)
     const float* sgate;      // FC2: shared-expert gate per token (acc_s += gate[t] * y), or null
+    unsigned long long* trace;  // this kernel's phase-trace block ([grid][MOE_TRACE_FIELDS]) or null
     int streamk_max;         // stream-K when the call has fewer tiles than this (0: never)
     float* skp;              // FC1 stream-K partial sums, one slot per CTA ([kNA][BN][128] FP32)
     int* done;               // FC1 stream-K per-tile counters (zero on entry, >= streamk_max of them)

@@ -26,7 +26,7 @@ WS_TOPK_IDS, WS_TOPK_W, WS_OFFSETS, WS_PERM = range(4)
 # Every symbol include/moe.h declares.
 EXPORTS = ("moe_router_topk", "moe_permute_workspace_size", "moe_permute", "moe_workspace_size",
            "moe_select_path", "moe_fused_forward", "moe_fused_forward_launches", "moe_fused_forward_plan",
-           "moe_token_tiles",
+           "moe_token_tiles", "moe_trace_size",
            "moe_workspace_region", "moe_fused_forward_timed", "moe_fused_forward_noalloc",
            "moe_noalloc_get_error", "moe_get_error", "moe_status_string")
 
@@ -42,7 +42,7 @@ class LayerDesc(ctypes.Structure):
     _fields_ = [(n, _ci) for n in ("T", "H", "I", "E", "top_k", "act", "score", "renorm", "I_shared", "path")] + [
         ("router_w", _vp), ("router_logits", _vp), ("bias", _vp), ("w13", _vp), ("w2", _vp),
         ("ws13", _vp), ("ws2", _vp), ("routed_scale", ctypes.c_float), ("shared_gate_w", _vp),
-        ("shared_out", _vp)]
+        ("shared_out", _vp), ("trace", _vp)]
 
 
 _lib.moe_router_topk.argtypes = [_vp, _ci, _ci, _ci, _ci, _ci, _vp, _ci, _vp, _vp, _vp, _vp]
@@ -60,6 +60,10 @@ _lib.moe_fused_forward_launches.restype = _ci
 _lib.moe_fused_forward_plan.argtypes = [ctypes.POINTER(LayerDesc), ctypes.POINTER(_ci), _ci]
 _lib.moe_fused_forward_plan.restype = _ci
 KERNEL_NAMES = ("prep", "router", "route", "topk", "refine", "select", "permute", "fc1", "fc2", "finalize")
+_lib.moe_trace_size.argtypes = []
+_lib.moe_trace_size.restype = _sz
+TRACE_FIELDS, TRACE_MAX_CTAS = 8, 1024
+TRACE_KERNELS = ("router", "fc1", "fc2")
 _lib.moe_token_tiles.argtypes = [ctypes.POINTER(LayerDesc), ctypes.POINTER(_ci), ctypes.POINTER(_ci)]
 _lib.moe_token_tiles.restype = _ci
 _lib.moe_workspace_region.argtypes = [ctypes.POINTER(LayerDesc), _ci, ctypes.POINTER(_sz), ctypes.POINTER(_sz)]
@@ -166,13 +170,14 @@ def noalloc_get_error(stream=None) -> int:
 
 def make_desc(T: int, H: int, I: int, E: int, top_k: int, act: str, score: str, renorm: bool, I_shared: int,
               path: str = "auto", router_w=None, router_logits=None, bias=None, w13=None, w2=None, ws13=None,
-              ws2=None, routed_scale: float = 0.0, shared_gate_w=None, shared_out=None) -> LayerDesc:
+              ws2=None, routed_scale: float = 0.0, shared_gate_w=None, shared_out=None, trace=None) -> LayerDesc:
     d = LayerDesc()
     d.T, d.H, d.I, d.E, d.top_k = T, H, I, E, top_k
     d.act, d.score, d.renorm, d.I_shared, d.path = ACT[act], SCORE[score], int(renorm), I_shared, PATH[path]
     d.router_w, d.router_logits, d.bias = _ptr(router_w), _ptr(router_logits), _ptr(bias)
     d.w13, d.w2, d.ws13, d.ws2 = _ptr(w13), _ptr(w2), _ptr(ws13), _ptr(ws2)
     d.routed_scale, d.shared_gate_w, d.shared_out = routed_scale, _ptr(shared_gate_w), _ptr(shared_out)
+    d.trace = _ptr(trace)
     return d
 
 
@@ -194,6 +199,37 @@ def kernel_plan(desc: LayerDesc):
     buf = (_ci * 16)()
     n = _lib.moe_fused_forward_plan(ctypes.byref(desc), buf, 16)
     return [KERNEL_NAMES[buf[i]] for i in range(n)]
+
+
+def trace_buffer(device) -> torch.Tensor:
+    """A zeroed phase-trace buffer for LayerDesc.trace (moe_trace_size bytes)."""
+    n = _lib.moe_trace_size() // 8
+    return torch.zeros(n, dtype=torch.int64, device=device)
+
+
+def trace_summary(trace: torch.Tensor, grid: int) -> dict:
+    """Per traced kernel, from the CTAs' %globaltimer stamps (microseconds): launch skew
+    (last CTA entry - first), median wait for inputs (ready - entry), median load span
+    (last load issued - ready), the tail (last exit - first exit), the whole kernel (last
+    exit - first entry), and the spread of work units per CTA."""
+    t = trace.view(len(TRACE_KERNELS), TRACE_MAX_CTAS, TRACE_FIELDS)[:, :grid].to("cpu").numpy()
+    out = {}
+    for k, name in enumerate(TRACE_KERNELS):
+        r = t[k]
+        live = r[:, 0] > 0
+        if not live.any():
+            continue
+        r = r[live].astype("float64")
+        entry, ready, loads, stores, exit_, units = (r[:, i] for i in range(6))
+        med = lambda v: float(sorted(v)[len(v) // 2])  # noqa: E731
+        out[name] = {"ctas": int(live.sum()),
+                     "launch_skew_us": (entry.max() - entry.min()) / 1e3,
+                     "input_wait_us_median": med(ready - entry) / 1e3,
+                     "load_span_us_median": med(loads - ready) / 1e3,
+                     "tail_us": (exit_.max() - exit_.min()) / 1e3,
+                     "kernel_us": (exit_.max() - entry.min()) / 1e3,
+                     "units_min_max": [int(units.min()), int(units.max())]}
+    return out
 
 
 def token_tiles(desc: LayerDesc):
@@ -250,13 +286,14 @@ class MoELayer:
         self._ws = None
 
     def desc(self, T: int, router_logits: Optional[torch.Tensor] = None,
-             shared_out: Optional[torch.Tensor] = None) -> LayerDesc:
+             shared_out: Optional[torch.Tensor] = None, trace: Optional[torch.Tensor] = None) -> LayerDesc:
         s, w = self.shape, self.w
         Is = s.I_shared if w.get("ws13") is not None else 0
         return make_desc(T, s.H, s.I, s.E, s.K, s.act, s.score, s.renorm, Is, self.path,
                          router_w=w.get("router_w"), router_logits=router_logits, bias=w.get("bias"),
                          w13=w["w13"], w2=w["w2"], ws13=w.get("ws13"), ws2=w.get("ws2"),
-                         routed_scale=self.routed_scale, shared_gate_w=w.get("shared_gate"), shared_out=shared_out)
+                         routed_scale=self.routed_scale, shared_gate_w=w.get("shared_gate"), shared_out=shared_out,
+                         trace=trace)
 
     def workspace(self, desc: LayerDesc, device) -> torch.Tensor:
         need = workspace_size(desc)
@@ -267,11 +304,13 @@ class MoELayer:
         return self._ws
 
     def forward(self, x: torch.Tensor, router_logits: Optional[torch.Tensor] = None, out=None,
-                return_routing: bool = False, stream=None, shared_out: Optional[torch.Tensor] = None):
+                return_routing: bool = False, stream=None, shared_out: Optional[torch.Tensor] = None,
+                trace: Optional[torch.Tensor] = None):
         """``shared_out``: a [T, H] BF16 shared-expert output to add (no internal shared
-        expert); ``out`` may be that same tensor (in-place form)."""
+        expert); ``out`` may be that same tensor (in-place form).  ``trace``: an optional
+        phase-trace buffer (``trace_buffer``)."""
         T = x.shape[0]
-        d = self.desc(T, router_logits, shared_out)
+        d = self.desc(T, router_logits, shared_out, trace)
         ws = self.workspace(d, x.device)
         if out is None:
             out = torch.empty((T, self.shape.H), dtype=torch.bfloat16, device=x.device)
