@@ -54,12 +54,12 @@ __device__ __forceinline__ void shared_gate_row(const GateArgs& g, int row, int 
 // ---------------------------------------------------------------- call prep
 // First kernel of a many-token call.  CTA 0 zeroes the call's counters.  Before the
 // tensor-core router (wr given), the grid's warps also take the E router rows and the T
-// token rows of x, one row each: the FP32 sum of the H squares lies within a relative
+// token rows of x, four rows per warp at a time: the FP32 sum of the H squares lies within a relative
 // H * 2^-24 of the exact value and is scaled up by (1 + 2^-8) (H <= 2^16), so it is an
 // upper bound.  Each CTA's maximum over router rows goes to wpart[blockIdx.x] (consumers
 // take the maximum over the grid's entries: no atomics, nothing to zero first); a token
 // row's bound goes to xn2[t].
-__global__ void __launch_bounds__(256) prep_kernel(int* __restrict__ counters, int n, int* __restrict__ counters2,
+__global__ void __launch_bounds__(256, 1) prep_kernel(int* __restrict__ counters, int n, int* __restrict__ counters2,
                                                    int n2, const bf16* __restrict__ wr, int E, int H,
                                                    float* __restrict__ wpart, const bf16* __restrict__ x, int T,
                                                    float* __restrict__ xn2) {
@@ -75,16 +75,30 @@ __global__ void __launch_bounds__(256) prep_kernel(int* __restrict__ counters, i
         __shared__ float s_max[8];
         float m = 0.0f;
         const int nw = (gridDim.x * blockDim.x) >> 5;
-        for (int r = (blockIdx.x * blockDim.x + tid) >> 5; r < E + T; r += nw) {
-            const bf16* row = r < E ? wr + (size_t)r * H : x + (size_t)(r - E) * H;
-            float ss = 0.0f;
+        // Four rows per pass, so that a lane keeps the loads of four rows in flight.
+        constexpr int kRows = 4;
+        for (int r0 = ((blockIdx.x * blockDim.x + tid) >> 5) * kRows; r0 < E + T; r0 += nw * kRows) {
+            float ss[kRows];
+#pragma unroll
+            for (int j = 0; j < kRows; ++j) ss[j] = 0.0f;
             for (int c = lane; c < (H >> 3); c += 32) {
-                const uint4 v = ld_nc16(row + (size_t)c * 8);
-                ss = dot8(v, v, ss);
+                uint4 v[kRows];
+#pragma unroll
+                for (int j = 0; j < kRows; ++j) {
+                    const int r = r0 + j;
+                    const bf16* row = r < E ? wr + (size_t)r * H : x + (size_t)(r - E) * H;
+                    v[j] = r < E + T ? ld_nc16(row + (size_t)c * 8) : make_uint4(0u, 0u, 0u, 0u);
+                }
+#pragma unroll
+                for (int j = 0; j < kRows; ++j) ss[j] = dot8(v[j], v[j], ss[j]);
             }
-            const float b = warp_sum(ss) * (1.0f + 0x1p-8f);
-            if (r < E) m = fmaxf(m, b);
-            else if (lane == 0) xn2[r - E] = b;
+#pragma unroll
+            for (int j = 0; j < kRows; ++j) {
+                const int r = r0 + j;
+                const float b = warp_sum(ss[j]) * (1.0f + 0x1p-8f);
+                if (r < E) m = fmaxf(m, b);
+                else if (r < E + T && lane == 0) xn2[r - E] = b;
+            }
         }
         if (lane == 0) s_max[tid >> 5] = m;
         __syncthreads();
@@ -95,7 +109,7 @@ __global__ void __launch_bounds__(256) prep_kernel(int* __restrict__ counters, i
     }
 }
 
-int prep_grid(int E, int T, int num_sms) { return std::max(1, std::min(num_sms, cdiv(E + T, 8))); }
+int prep_grid(int E, int T, int num_sms) { return std::max(1, std::min(num_sms, cdiv(E + T, 32))); }
 
 cudaError_t launch_prep(int* counters, int n, int* counters2, int n2, const bf16* wr, int E, int H, float* wpart,
                         const bf16* x, int T, float* xn2, int num_sms, cudaStream_t s) {
