@@ -225,14 +225,14 @@ def roofline_of(acc: dict, dur_s: float, peaks: dict):
 
 # ---------------------------------------------------------------- our arm
 class Bench:
-    def __init__(self, shape, T, device, seed, routing, path="auto"):
+    def __init__(self, shape, T, device, seed, routing, path="auto", schedule="auto"):
         import mixture_experts_layer_35_b200.moe as moe
         self.moe = moe
         self.shape, self.T, self.device = shape, T, device
         self.d = gen.make_layer(shape, T, seed=seed, device=str(device), routing=routing)
         self.logits = self.d["router_logits"]
         w = {k: self.d[k] for k in ("router_w", "bias", "w13", "w2", "ws13", "ws2") if self.d.get(k) is not None}
-        self.layer = moe.MoELayer(shape, w, path=path)
+        self.layer = moe.MoELayer(shape, w, path=path, schedule=schedule)
         self.desc = self.layer.desc(T, self.logits)
         self.ws = self.layer.workspace(self.desc, device)
         self.out = torch.empty((T, shape.H), dtype=torch.bfloat16, device=device)
@@ -451,7 +451,8 @@ def run_ours(args, rank, local, world):
     dist_init(world, "nccl")
     shape = gen.SHORT[args.config]
     peaks, peaks_src = load_peaks()
-    b = Bench(shape, args.T, device, seed=args.seed + rank, routing=args.routing, path=args.path)
+    b = Bench(shape, args.T, device, seed=args.seed + rank, routing=args.routing, path=args.path,
+              schedule=args.schedule)
     per, clk = b.timed(args.steps, args.warmup, world, clocks=True)
     local_ms = float(sum(per))
     total_ms = max_over_ranks(local_ms, world, device)
@@ -487,7 +488,8 @@ def run_ours(args, rank, local, world):
         "dtype": "bf16", "data": "synthetic (seeded generator, random-init weights of the layer's shape)",
         "config": {"workload": f"{shape.name} T={args.T} routing={args.routing}", "tokens_per_step": args.T,
                    "timing": "one CUDA-graph replay of moe_fused_forward per step",
-                   "path": b.path, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "path": b.path, "schedule": args.schedule,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write), steps timed with CUDA events",
                    "distinct_experts": U},
         "roofline": roof,
@@ -542,7 +544,7 @@ def sweep(args, device, peaks):
         shape = gen.SHORT[cfg]
         print(f"sweep: {cfg} T={T}", file=sys.stderr, flush=True)
         try:
-            b = Bench(shape, T, device, seed=1, routing="router", path=args.path)
+            b = Bench(shape, T, device, seed=1, routing="router", path=args.path, schedule=args.schedule)
             per, _ = b.timed(args.sweep_steps, 5)
             med = statistics.median(per)
             U = b.distinct_experts()
@@ -726,6 +728,8 @@ def main(argv=None):
     p.add_argument("--routing", choices=["router", "zipf"], default="router")
     p.add_argument("--path", choices=["auto", "small", "large"], default="auto",
                    help="force an execution path (selector studies); auto = the library's choice")
+    p.add_argument("--schedule", choices=["auto", "static", "dynamic"], default="auto",
+                   help="tile schedule of the grouped GEMMs (auto = the library's choice)")
     p.add_argument("--seed", type=int, default=0)
     p.add_argument("--no-sweep", action="store_true")
     p.add_argument("--sweep-all", action="store_true")

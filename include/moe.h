@@ -165,7 +165,16 @@ typedef struct {
      * CTA took.  Rows of CTAs a kernel did not launch, and blocks of kernels the call did
      * not run, are left as they were.  16-byte aligned. */
     unsigned long long* trace;
+    /* Tile schedule of the many-token path's grouped GEMMs (moe_sched_t): STATIC deals the
+     * tiles round-robin over the persistent CTAs; DYNAMIC lets each CTA take the next tile
+     * of the same list from a device counter whenever its load pipeline is ready for one;
+     * AUTO (0) chooses per call.  Results are identical up to the FP32 order of the
+     * routed combine (already unspecified).  GEMMs that run stream-K (few-token calls)
+     * keep their own schedule. */
+    int schedule;
 } moe_layer_desc;
+
+typedef enum { MOE_SCHED_AUTO = 0, MOE_SCHED_STATIC = 1, MOE_SCHED_DYNAMIC = 2 } moe_sched_t;
 
 enum { MOE_TRACE_ENTRY = 0, MOE_TRACE_READY = 1, MOE_TRACE_LOADS_DONE = 2, MOE_TRACE_STORES_DONE = 3,
        MOE_TRACE_EXIT = 4, MOE_TRACE_UNITS = 5, MOE_TRACE_FIELDS = 8 };

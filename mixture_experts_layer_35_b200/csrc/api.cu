@@ -32,6 +32,8 @@ constexpr size_t kCandPerRow = 32;
 // stream-K per-tile counters.
 inline size_t counter_ints(size_t E) { return 2 * (E + 2) + 4; }
 inline size_t cand_count_int(size_t E) { return 2 * (E + 2); }
+// Next-tile counters of the dynamic schedule (FC1: which = 0, FC2: 1).
+inline size_t dyn_count_int(size_t E, int which) { return 2 * (E + 2) + 1 + which; }
 // Per-CTA router weight-norm bounds of the prep kernel (one per SM at most).
 constexpr size_t kMaxPrepGrid = 1024;
 WsLayout layout(const moe_layer_desc* d) {
@@ -88,6 +90,7 @@ moe_status_t validate_desc(const moe_layer_desc* d) {
         return MOE_ERR_INVALID_ARG;  // NaN or infinite
     if (d->shared_gate_w && d->I_shared == 0) return MOE_ERR_INVALID_ARG;
     if (d->shared_out && d->I_shared > 0) return MOE_ERR_INVALID_ARG;
+    if (d->schedule < MOE_SCHED_AUTO || d->schedule > MOE_SCHED_DYNAMIC) return MOE_ERR_INVALID_ARG;
     const void* ptrs[] = {d->router_w, d->router_logits, d->bias, d->w13, d->w2, d->ws13, d->ws2,
                           d->shared_gate_w, d->shared_out, d->trace};
     for (const void* p : ptrs)
@@ -125,6 +128,15 @@ int auto_path(const moe_layer_desc* d) {
 int resolve_path(const moe_layer_desc* d) {
     if (d->path == MOE_PATH_AUTO) return auto_path(d);
     return d->path;
+}
+// Tile schedule of the many-token path's grouped GEMMs (GEMMs that run stream-K keep
+// theirs).  AUTO takes the dynamic schedule from 256 average rows per expert on: there the
+// round-robin left the CTAs' finishing times 100-150 us apart (Qwen3.6-shaped T = 8192:
+// 775 -> 767 us; Nemotron-shaped T = 8192: 1520 -> 1481 us), while below it the dynamic
+// kernel's FC2 is slower than its tail saving (Qwen3.6-shaped T = 4096: 440 -> 468 us).
+int resolve_schedule(const moe_layer_desc* d) {
+    if (d->schedule != MOE_SCHED_AUTO) return d->schedule;
+    return (long long)d->T * d->top_k >= 256LL * d->E ? MOE_SCHED_DYNAMIC : MOE_SCHED_STATIC;
 }
 
 
@@ -480,6 +492,7 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
     const bool swiglu = d->act == MOE_ACT_SWIGLU;
     const int fc1_mode = swiglu ? GM_FC1_SWIGLU : GM_FC1_RELU2;
     const int bn1 = gemm_token_tile(fc1_mode, T, K, E), bn2 = gemm_token_tile(GM_FC2, T, K, E);
+    const bool dyn = resolve_schedule(d) == MOE_SCHED_DYNAMIC;
     // 2. top-k (also counts the slots per expert; the counters were cleared in step 0)
     if (!mark()) return MOE_ERR_CUDA;
     RefineArgs ra = {x, static_cast<const bf16*>(d->router_w), H, logits_rw, wpart, prep_grid(E, T, sms),
@@ -570,6 +583,7 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
     g1.streamk_max = gemm_streamk_max(fc1_mode, bn1, sms, max_tiles(bn1, g1.nfeat_r, Is ? g1.nfeat_s : 0));
     g1.skp = reinterpret_cast<float*>(w8 + L.skp);
     g1.done = reinterpret_cast<int*>(w8 + L.done);
+    g1.dyn_ctr = dyn ? counts + dyn_count_int(E, 0) : nullptr;
     g1.err = err;
     if (!mark()) return MOE_ERR_CUDA;
     MOE_CK(launch_gemm(fc1_mode, bn1, g1, m1, sms, s, chain));
@@ -601,6 +615,7 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
     g2.streamk_max = gemm_streamk_max(GM_FC2, bn2, sms, max_tiles(bn2, g2.nfeat_r, Is ? g2.nfeat_s : 0));
     g2.skp = nullptr;
     g2.done = nullptr;
+    g2.dyn_ctr = dyn ? counts + dyn_count_int(E, 1) : nullptr;
 
     if (!mark()) return MOE_ERR_CUDA;
     MOE_CK(launch_gemm(GM_FC2, bn2, g2, m2, sms, s, chain));

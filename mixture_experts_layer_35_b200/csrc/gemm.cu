@@ -89,7 +89,11 @@ struct Cfg {
     // stages, and lag 2 of 3, both stall; one warp per stage is slower too).
     static constexpr int kLagMax = 2;
     static constexpr int kMaxGroups = MOE_MAX_EXPERTS + 1;
-    static constexpr size_t kMeta = 256 + (size_t)(kMaxGroups + 1) * 4 * 2 + 64;
+    // Dynamic schedule: a ring of tile ids from the producer to the other roles.
+    static constexpr int kIdSlots = 8;
+    static constexpr int kIdConsumers = 1 + kEpiWarps + kGatherWarps;  // MMA thread, warps
+    static constexpr size_t kRingOff = 256 + (size_t)(kMaxGroups + 1) * 4 * 2 + 64;
+    static constexpr size_t kMeta = kRingOff + (size_t)kIdSlots * (8 + 8 + 4) + 64;
     // As many stages as the 227 KB of shared memory hold (at most 12: the barrier block).
     static constexpr int kStages =
         (int)((227 * 1024 - 1024 - kMeta - kEpiBytes) / kStageBytes) < 12
@@ -263,7 +267,13 @@ __device__ __forceinline__ void combine_chunk(const uint32_t (&v)[32], int mt, f
 
 // Whole tiles dealt round-robin over persistent CTAs (every call except few-token ones,
 // which take gemm_sk_kernel below).
-template <int MODE, int BN>
+// DYN: dynamic tile schedule.  After a round-robin prefix, the producer thread takes each
+// next tile from a device counter (atomicAdd) when its ring is ready for one, and passes
+// every id through a ring of kIdSlots shared-memory slots (mbarriers full/empty) to the MMA
+// thread, the epilogue warps and the gather warps, which take the ids in the same order.
+// The id after the last tile (>= total) ends every role's loop.  Without DYN, all tiles
+// are dealt round-robin.
+template <int MODE, int BN, bool DYN>
 __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
     gemm_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ CUtensorMap tm_a_s,
                 const __grid_constant__ CUtensorMap tm_b_r, const __grid_constant__ CUtensorMap tm_b_s) {
@@ -283,6 +293,11 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int* s_tiles = reinterpret_cast<int*>(meta + 256);
     int* s_offs = s_tiles + C::kMaxGroups + 1;
+    // tile-id ring (DYN): full[kIdSlots], empty[kIdSlots], ids[kIdSlots]
+    const uint32_t ring_u32 = smem_u32(meta + C::kRingOff);
+    auto idfull_bar = [&](int j) { return ring_u32 + 8u * j; };
+    auto idempty_bar = [&](int j) { return ring_u32 + 8u * (C::kIdSlots + j); };
+    volatile int* s_ids = reinterpret_cast<volatile int*>(meta + C::kRingOff + 16 * C::kIdSlots);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = a.E + (a.has_shared ? 1 : 0);
@@ -298,6 +313,12 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
         for (int b = 0; b < 2; ++b) {
             mbar_init(tfull_bar(b), 1);
             mbar_init(tempty_bar(b), C::kEpiWarps);
+        }
+        if (DYN) {
+            for (int j = 0; j < C::kIdSlots; ++j) {
+                mbar_init(idfull_bar(j), 1);
+                mbar_init(idempty_bar(j), C::kIdConsumers);
+            }
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -328,14 +349,47 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
     // Tiles are dealt round-robin over the persistent CTAs: at any moment the CTAs work on
     // neighbouring tiles of the group-major list (one expert's feature and token tiles),
     // which share that expert's weight rows and token rows in L2, and tiles of unequal
-    // cost (ragged token tails) spread evenly.
+    // cost (ragged token tails) spread evenly.  The dynamic schedule takes the tiles in
+    // the same list order, each from the first producer that is ready for one.
+    int dj = 0;  // DYN: this role's position in the tile-id ring
+    // The first three quarters of the rounds (all but at least two) stay round-robin, so
+    // that neighbouring tiles still run side by side; the rest go to whichever CTA is
+    // ready first.
+    const int rr_rounds = DYN ? max(0, (3 * cdiv(total, (int)gridDim.x)) / 4 - 1) : 0;
+    // Producer: the next tile (round-robin prefix, then the counter), published to the
+    // ring (>= total: the end).
+    auto id_produce = [&]() -> int {
+        const int slot = dj % C::kIdSlots;
+        const uint32_t ph = (uint32_t)(dj / C::kIdSlots) & 1u;
+        if (!mbar_wait(idempty_bar(slot), ph ^ 1u, abort_flag, a.err)) return total;
+        int t = dj < rr_rounds ? (int)blockIdx.x + dj * (int)gridDim.x
+                                : rr_rounds * (int)gridDim.x + atomicAdd(a.dyn_ctr, 1);
+        if (t > total) t = total;
+        s_ids[slot] = t;
+        mbar_arrive(idfull_bar(slot));
+        ++dj;
+        return t;
+    };
+    // Consumer (one thread, or every lane of a warp with `warp_wide`): the next id.
+    auto id_consume = [&](bool warp_wide) -> int {
+        const int slot = dj % C::kIdSlots;
+        const uint32_t ph = (uint32_t)(dj / C::kIdSlots) & 1u;
+        if (!mbar_wait(idfull_bar(slot), ph, abort_flag, a.err)) return total;
+        const int t = s_ids[slot];
+        ++dj;
+        if (warp_wide) __syncwarp();
+        if (!warp_wide || lane == 0) mbar_arrive(idempty_bar(slot));
+        return t;
+    };
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             const uint64_t wpol = l2_policy_evict_first();
-            int it = 0;
-            for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
+            int it = 0, ntiles = 0;
+            for (int tile = DYN ? id_produce() : (int)blockIdx.x; tile < total && !*abort_flag;
+                 tile = DYN ? id_produce() : tile + (int)gridDim.x) {
+                ++ntiles;
                 const TileInfo ti = decode_tile<C::kBN>(a, s_tiles, s_offs, G, tile);
                 const bool sh = ti.shared;
                 const CUtensorMap* ta = sh ? &tm_a_s : &tm_a_r;
@@ -375,15 +429,15 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
             }
             if (trow) {
                 trow[MOE_TRACE_LOADS_DONE] = globaltimer_ns();
-                trow[MOE_TRACE_UNITS] = (unsigned long long)((total - (int)blockIdx.x + (int)gridDim.x - 1) /
-                                                             (int)gridDim.x);
+                trow[MOE_TRACE_UNITS] = (unsigned long long)ntiles;
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             int it = 0, tcount = 0;
-            for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x, ++tcount) {
+            for (int tile = DYN ? id_consume(false) : (int)blockIdx.x; tile < total && !*abort_flag;
+                 tile = DYN ? id_consume(false) : tile + (int)gridDim.x, ++tcount) {
                 const TileInfo ti = decode_tile<C::kBN>(a, s_tiles, s_offs, G, tile);
                 const int nk = ti.nk;
                 const int npad = cdiv(ti.n, 16) * 16;
@@ -435,7 +489,8 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
         // (the abort flag is checked through the per-tile wait below)
         // 32-token chunks per half of the epilogue warps (the last may lie past the tile)
         constexpr int kChunks = (C::kBN + 32 * (C::kEpiWarps / 4) - 1) / (32 * (C::kEpiWarps / 4));
-        for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++tcount) {
+        for (int tile = DYN ? id_consume(true) : (int)blockIdx.x; tile < total;
+             tile = DYN ? id_consume(true) : tile + (int)gridDim.x, ++tcount) {
             const TileInfo ti = decode_tile<C::kBN>(a, s_tiles, s_offs, G, tile);
             const int buf = tcount % C::kAccBufs;
             const uint32_t tph = (uint32_t)(tcount / C::kAccBufs) & 1u;
@@ -568,7 +623,8 @@ __global__ void __launch_bounds__(Cfg<MODE, BN>::kThreads, 1)
         const int p = threadIdx.x - (64 + 32 * C::kEpiWarps);  // 0 .. kGatherThreads - 1
         const int chunk = p & 7, rsub = p >> 3;
         int it = 0;
-        for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
+        for (int tile = DYN ? id_consume(true) : (int)blockIdx.x; tile < total && !*abort_flag;
+             tile = DYN ? id_consume(true) : tile + (int)gridDim.x) {
             const TileInfo ti = decode_tile<C::kBN>(a, s_tiles, s_offs, G, tile);
             const int kd = ti.shared ? a.kdim_s : a.kdim;
             const int nk = ti.nk;
@@ -1136,7 +1192,10 @@ static cudaError_t launch_mode(const GemmArgs& a, const GemmMaps& m, int grid, c
         if (a.streamk_max > 0)
             return launch_gemm_kernel(gemm_sk_kernel<MODE, BN, true>, C::kSmem, C::kThreads, a, m, grid, s, pdl);
     }
-    return launch_gemm_kernel(gemm_kernel<MODE, BN>, C::kSmem, C::kThreads, a, m, grid, s, pdl);
+    if constexpr (MODE != GM_DENSE) {
+        if (a.dyn_ctr) return launch_gemm_kernel(gemm_kernel<MODE, BN, true>, C::kSmem, C::kThreads, a, m, grid, s, pdl);
+    }
+    return launch_gemm_kernel(gemm_kernel<MODE, BN, false>, C::kSmem, C::kThreads, a, m, grid, s, pdl);
 }
 
 int gemm_token_tile(int mode, int T, int K, int E) {

@@ -179,6 +179,7 @@ struct GemmArgs {
     int streamk_max;         // stream-K when the call has fewer tiles than this (0: never)
     float* skp;              // FC1 stream-K partial sums, one slot per CTA ([kNA][BN][128] FP32)
     int* done;               // FC1 stream-K per-tile counters (zero on entry, >= streamk_max of them)
+    int* dyn_ctr;            // dynamic tile schedule: the next-tile counter (zero on entry), or null
     int* err;
 };
 struct GemmMaps {

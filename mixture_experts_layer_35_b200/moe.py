@@ -19,6 +19,7 @@ MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUD
 SCORE = {"softmax": 0, "sigmoid": 1}
 ACT = {"swiglu": 0, "relu2": 1}
 PATH = {"auto": 0, "small": 1, "large": 2}
+SCHEDULE = {"auto": 0, "static": 1, "dynamic": 2}  # moe_sched_t
 DT_BF16, DT_FP32 = 0, 1
 DEVERR_BAD_EXPERT_ID, DEVERR_WAIT_TIMEOUT, DEVERR_BAD_INDEX, DEVERR_ROUTER_BOUND = 0x1, 0x2, 0x4, 0x8
 WS_TOPK_IDS, WS_TOPK_W, WS_OFFSETS, WS_PERM = range(4)
@@ -42,7 +43,7 @@ class LayerDesc(ctypes.Structure):
     _fields_ = [(n, _ci) for n in ("T", "H", "I", "E", "top_k", "act", "score", "renorm", "I_shared", "path")] + [
         ("router_w", _vp), ("router_logits", _vp), ("bias", _vp), ("w13", _vp), ("w2", _vp),
         ("ws13", _vp), ("ws2", _vp), ("routed_scale", ctypes.c_float), ("shared_gate_w", _vp),
-        ("shared_out", _vp), ("trace", _vp)]
+        ("shared_out", _vp), ("trace", _vp), ("schedule", _ci)]
 
 
 _lib.moe_router_topk.argtypes = [_vp, _ci, _ci, _ci, _ci, _ci, _vp, _ci, _vp, _vp, _vp, _vp]
@@ -170,7 +171,8 @@ def noalloc_get_error(stream=None) -> int:
 
 def make_desc(T: int, H: int, I: int, E: int, top_k: int, act: str, score: str, renorm: bool, I_shared: int,
               path: str = "auto", router_w=None, router_logits=None, bias=None, w13=None, w2=None, ws13=None,
-              ws2=None, routed_scale: float = 0.0, shared_gate_w=None, shared_out=None, trace=None) -> LayerDesc:
+              ws2=None, routed_scale: float = 0.0, shared_gate_w=None, shared_out=None, trace=None,
+              schedule: str = "auto") -> LayerDesc:
     d = LayerDesc()
     d.T, d.H, d.I, d.E, d.top_k = T, H, I, E, top_k
     d.act, d.score, d.renorm, d.I_shared, d.path = ACT[act], SCORE[score], int(renorm), I_shared, PATH[path]
@@ -178,6 +180,7 @@ def make_desc(T: int, H: int, I: int, E: int, top_k: int, act: str, score: str, 
     d.w13, d.w2, d.ws13, d.ws2 = _ptr(w13), _ptr(w2), _ptr(ws13), _ptr(ws2)
     d.routed_scale, d.shared_gate_w, d.shared_out = routed_scale, _ptr(shared_gate_w), _ptr(shared_out)
     d.trace = _ptr(trace)
+    d.schedule = SCHEDULE[schedule]
     return d
 
 
@@ -276,13 +279,16 @@ def fused_forward_noalloc(desc: LayerDesc, x: torch.Tensor, out: torch.Tensor,
 class MoELayer:
     """A layer whose weights live on the device; ``forward`` enqueues moe_fused_forward."""
 
-    def __init__(self, shape, weights: dict, path: str = "auto", routed_scale: float = 0.0):
+    def __init__(self, shape, weights: dict, path: str = "auto", routed_scale: float = 0.0,
+                 schedule: str = "auto"):
         """``weights``: router_w, bias, w13, w2, and optionally ws13 / ws2 (internal shared
-        expert) and shared_gate (its [H] gate row).  ``routed_scale``: 0 = none."""
+        expert) and shared_gate (its [H] gate row).  ``routed_scale``: 0 = none.
+        ``schedule``: the grouped GEMMs' tile schedule (auto, static, dynamic)."""
         self.shape = shape
         self.w = weights
         self.path = path
         self.routed_scale = routed_scale
+        self.schedule = schedule
         self._ws = None
 
     def desc(self, T: int, router_logits: Optional[torch.Tensor] = None,
@@ -293,7 +299,7 @@ class MoELayer:
                          router_w=w.get("router_w"), router_logits=router_logits, bias=w.get("bias"),
                          w13=w["w13"], w2=w["w2"], ws13=w.get("ws13"), ws2=w.get("ws2"),
                          routed_scale=self.routed_scale, shared_gate_w=w.get("shared_gate"), shared_out=shared_out,
-                         trace=trace)
+                         trace=trace, schedule=self.schedule)
 
     def workspace(self, desc: LayerDesc, device) -> torch.Tensor:
         need = workspace_size(desc)

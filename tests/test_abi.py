@@ -55,6 +55,8 @@ def _fwd(d, x=FAKE * 6, out=FAKE * 7, ws=None, ws_bytes=0):
     ("act", 7, moe.MOE_ERR_INVALID_ARG),
     ("score", 5, moe.MOE_ERR_INVALID_ARG),
     ("path", 9, moe.MOE_ERR_INVALID_ARG),
+    ("schedule", 3, moe.MOE_ERR_INVALID_ARG),
+    ("schedule", -1, moe.MOE_ERR_INVALID_ARG),
     ("T", -1, moe.MOE_ERR_INVALID_ARG),
     ("T", 1 << 20, moe.MOE_ERR_UNSUPPORTED),
     ("I_shared", 12, moe.MOE_ERR_INVALID_ARG),
