@@ -3,7 +3,8 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--config qwen36|nemotron|large_e|tiny] [--T 4096] [--routing router|zipf]
-                    [--no-sweep]
+                    [--workload layer|router_topk] [--path auto|small|large]
+                    [--schedule auto|static|dynamic] [--no-sweep | --sweep-all] [--no-cpu]
 
 A step is one complete layer forward (router logits, top-k, permutation, FC1 + activation,
 FC2 + weighted combine, shared expert, finalize) over T tokens of synthetic input drawn
