@@ -226,14 +226,14 @@ def roofline_of(acc: dict, dur_s: float, peaks: dict):
 
 # ---------------------------------------------------------------- our arm
 class Bench:
-    def __init__(self, shape, T, device, seed, routing, path="auto", schedule="auto"):
+    def __init__(self, shape, T, device, seed, routing, path="auto", schedule="auto", tiles=(0, 0)):
         import mixture_experts_layer_35_b200.moe as moe
         self.moe = moe
         self.shape, self.T, self.device = shape, T, device
         self.d = gen.make_layer(shape, T, seed=seed, device=str(device), routing=routing)
         self.logits = self.d["router_logits"]
         w = {k: self.d[k] for k in ("router_w", "bias", "w13", "w2", "ws13", "ws2") if self.d.get(k) is not None}
-        self.layer = moe.MoELayer(shape, w, path=path, schedule=schedule)
+        self.layer = moe.MoELayer(shape, w, path=path, schedule=schedule, tiles=tiles)
         self.desc = self.layer.desc(T, self.logits)
         self.ws = self.layer.workspace(self.desc, device)
         self.out = torch.empty((T, shape.H), dtype=torch.bfloat16, device=device)
@@ -453,7 +453,7 @@ def run_ours(args, rank, local, world):
     shape = gen.SHORT[args.config]
     peaks, peaks_src = load_peaks()
     b = Bench(shape, args.T, device, seed=args.seed + rank, routing=args.routing, path=args.path,
-              schedule=args.schedule)
+              schedule=args.schedule, tiles=(args.fc1_tile, args.fc2_tile))
     per, clk = b.timed(args.steps, args.warmup, world, clocks=True)
     local_ms = float(sum(per))
     total_ms = max_over_ranks(local_ms, world, device)
@@ -489,7 +489,7 @@ def run_ours(args, rank, local, world):
         "dtype": "bf16", "data": "synthetic (seeded generator, random-init weights of the layer's shape)",
         "config": {"workload": f"{shape.name} T={args.T} routing={args.routing}", "tokens_per_step": args.T,
                    "timing": "one CUDA-graph replay of moe_fused_forward per step",
-                   "path": b.path, "schedule": args.schedule,
+                   "path": b.path, "schedule": args.schedule, "token_tiles": list(b.moe.token_tiles(b.desc)),
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write), steps timed with CUDA events",
                    "distinct_experts": U},
@@ -731,6 +731,8 @@ def main(argv=None):
                    help="force an execution path (selector studies); auto = the library's choice")
     p.add_argument("--schedule", choices=["auto", "static", "dynamic"], default="auto",
                    help="tile schedule of the grouped GEMMs (auto = the library's choice)")
+    p.add_argument("--fc1-tile", type=int, default=0, help="FC1 token rows per tile (0 = the library's choice)")
+    p.add_argument("--fc2-tile", type=int, default=0, help="FC2 token rows per tile (0 = the library's choice)")
     p.add_argument("--seed", type=int, default=0)
     p.add_argument("--no-sweep", action="store_true")
     p.add_argument("--sweep-all", action="store_true")

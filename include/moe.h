@@ -172,6 +172,11 @@ typedef struct {
      * routed combine (already unspecified).  GEMMs that run stream-K (few-token calls)
      * keep their own schedule. */
     int schedule;
+    /* Token rows per tile of the many-token path's grouped GEMMs, 0 = chosen per call from
+     * the average rows per expert (moe_token_tiles reports the choice).  FC1: 32, 64, 128,
+     * or 256 (ReLU^2 only); FC2: 32, 128, 192 or 256; anything else is MOE_ERR_INVALID_ARG.
+     * For tuning: results do not depend on it beyond the FP32 order of the routed combine. */
+    int fc1_tile_rows, fc2_tile_rows;
 } moe_layer_desc;
 
 typedef enum { MOE_SCHED_AUTO = 0, MOE_SCHED_STATIC = 1, MOE_SCHED_DYNAMIC = 2 } moe_sched_t;

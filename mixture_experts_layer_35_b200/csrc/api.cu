@@ -34,6 +34,14 @@ inline size_t counter_ints(size_t E) { return 2 * (E + 2) + 4; }
 inline size_t cand_count_int(size_t E) { return 2 * (E + 2); }
 // Next-tile counters of the dynamic schedule (FC1: which = 0, FC2: 1).
 inline size_t dyn_count_int(size_t E, int which) { return 2 * (E + 2) + 1 + which; }
+// Token rows per grouped-GEMM tile of a call: the caller's choice, else by rows per expert.
+int fc1_tile_rows(const moe_layer_desc* d) {
+    if (d->fc1_tile_rows) return d->fc1_tile_rows;
+    return gemm_token_tile(d->act == MOE_ACT_SWIGLU ? GM_FC1_SWIGLU : GM_FC1_RELU2, d->T, d->top_k, d->E);
+}
+int fc2_tile_rows(const moe_layer_desc* d) {
+    return d->fc2_tile_rows ? d->fc2_tile_rows : gemm_token_tile(GM_FC2, d->T, d->top_k, d->E);
+}
 // Per-CTA router weight-norm bounds of the prep kernel (one per SM at most).
 constexpr size_t kMaxPrepGrid = 1024;
 WsLayout layout(const moe_layer_desc* d) {
@@ -64,9 +72,7 @@ WsLayout layout(const moe_layer_desc* d) {
     L.wpart = take(kMaxPrepGrid * 4);
     L.xn2 = take(T * 4);
     L.roweps = take(T * 4);
-    const int fc1_mode = d->act == MOE_ACT_SWIGLU ? GM_FC1_SWIGLU : GM_FC1_RELU2;
-    L.skp = take(fc1_streamk_bytes(gemm_token_tile(fc1_mode, d->T, d->top_k, d->E), d->act == MOE_ACT_SWIGLU,
-                                   num_sms()));
+    L.skp = take(fc1_streamk_bytes(fc1_tile_rows(d), d->act == MOE_ACT_SWIGLU, num_sms()));
     L.gate = take(d->shared_gate_w ? T * 4 : 0);
     L.total = o;
     return L;
@@ -91,6 +97,10 @@ moe_status_t validate_desc(const moe_layer_desc* d) {
     if (d->shared_gate_w && d->I_shared == 0) return MOE_ERR_INVALID_ARG;
     if (d->shared_out && d->I_shared > 0) return MOE_ERR_INVALID_ARG;
     if (d->schedule < MOE_SCHED_AUTO || d->schedule > MOE_SCHED_DYNAMIC) return MOE_ERR_INVALID_ARG;
+    const int t1 = d->fc1_tile_rows, t2 = d->fc2_tile_rows;
+    if (t1 && t1 != 32 && t1 != 64 && t1 != 128 && !(t1 == 256 && d->act == MOE_ACT_RELU2))
+        return MOE_ERR_INVALID_ARG;
+    if (t2 && t2 != 32 && t2 != 128 && t2 != 192 && t2 != 256) return MOE_ERR_INVALID_ARG;
     const void* ptrs[] = {d->router_w, d->router_logits, d->bias, d->w13, d->w2, d->ws13, d->ws2,
                           d->shared_gate_w, d->shared_out, d->trace};
     for (const void* p : ptrs)
@@ -294,9 +304,8 @@ moe_status_t moe_token_tiles(const moe_layer_desc* d, int* fc1_rows, int* fc2_ro
     const moe_status_t st = validate_desc(d);
     if (st != MOE_OK) return st;
     if (!fc1_rows || !fc2_rows) return MOE_ERR_INVALID_ARG;
-    const int fc1_mode = d->act == MOE_ACT_SWIGLU ? GM_FC1_SWIGLU : GM_FC1_RELU2;
-    *fc1_rows = gemm_token_tile(fc1_mode, d->T, d->top_k, d->E);
-    *fc2_rows = gemm_token_tile(GM_FC2, d->T, d->top_k, d->E);
+    *fc1_rows = fc1_tile_rows(d);
+    *fc2_rows = fc2_tile_rows(d);
     return MOE_OK;
 }
 
@@ -491,7 +500,7 @@ static moe_status_t fused_forward_impl(const moe_layer_desc* d, const void* x_, 
     const bool chain = !timed;  // programmatic overlap between consecutive kernels
     const bool swiglu = d->act == MOE_ACT_SWIGLU;
     const int fc1_mode = swiglu ? GM_FC1_SWIGLU : GM_FC1_RELU2;
-    const int bn1 = gemm_token_tile(fc1_mode, T, K, E), bn2 = gemm_token_tile(GM_FC2, T, K, E);
+    const int bn1 = fc1_tile_rows(d), bn2 = fc2_tile_rows(d);
     const bool dyn = resolve_schedule(d) == MOE_SCHED_DYNAMIC;
     // 2. top-k (also counts the slots per expert; the counters were cleared in step 0)
     if (!mark()) return MOE_ERR_CUDA;

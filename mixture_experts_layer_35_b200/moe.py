@@ -43,7 +43,7 @@ class LayerDesc(ctypes.Structure):
     _fields_ = [(n, _ci) for n in ("T", "H", "I", "E", "top_k", "act", "score", "renorm", "I_shared", "path")] + [
         ("router_w", _vp), ("router_logits", _vp), ("bias", _vp), ("w13", _vp), ("w2", _vp),
         ("ws13", _vp), ("ws2", _vp), ("routed_scale", ctypes.c_float), ("shared_gate_w", _vp),
-        ("shared_out", _vp), ("trace", _vp), ("schedule", _ci)]
+        ("shared_out", _vp), ("trace", _vp), ("schedule", _ci), ("fc1_tile_rows", _ci), ("fc2_tile_rows", _ci)]
 
 
 _lib.moe_router_topk.argtypes = [_vp, _ci, _ci, _ci, _ci, _ci, _vp, _ci, _vp, _vp, _vp, _vp]
@@ -172,7 +172,7 @@ def noalloc_get_error(stream=None) -> int:
 def make_desc(T: int, H: int, I: int, E: int, top_k: int, act: str, score: str, renorm: bool, I_shared: int,
               path: str = "auto", router_w=None, router_logits=None, bias=None, w13=None, w2=None, ws13=None,
               ws2=None, routed_scale: float = 0.0, shared_gate_w=None, shared_out=None, trace=None,
-              schedule: str = "auto") -> LayerDesc:
+              schedule: str = "auto", tiles=(0, 0)) -> LayerDesc:
     d = LayerDesc()
     d.T, d.H, d.I, d.E, d.top_k = T, H, I, E, top_k
     d.act, d.score, d.renorm, d.I_shared, d.path = ACT[act], SCORE[score], int(renorm), I_shared, PATH[path]
@@ -181,6 +181,7 @@ def make_desc(T: int, H: int, I: int, E: int, top_k: int, act: str, score: str, 
     d.routed_scale, d.shared_gate_w, d.shared_out = routed_scale, _ptr(shared_gate_w), _ptr(shared_out)
     d.trace = _ptr(trace)
     d.schedule = SCHEDULE[schedule]
+    d.fc1_tile_rows, d.fc2_tile_rows = tiles
     return d
 
 
@@ -280,15 +281,17 @@ class MoELayer:
     """A layer whose weights live on the device; ``forward`` enqueues moe_fused_forward."""
 
     def __init__(self, shape, weights: dict, path: str = "auto", routed_scale: float = 0.0,
-                 schedule: str = "auto"):
+                 schedule: str = "auto", tiles=(0, 0)):
         """``weights``: router_w, bias, w13, w2, and optionally ws13 / ws2 (internal shared
         expert) and shared_gate (its [H] gate row).  ``routed_scale``: 0 = none.
-        ``schedule``: the grouped GEMMs' tile schedule (auto, static, dynamic)."""
+        ``schedule``: the grouped GEMMs' tile schedule (auto, static, dynamic).
+        ``tiles``: (FC1, FC2) token rows per GEMM tile, 0 = the library's choice."""
         self.shape = shape
         self.w = weights
         self.path = path
         self.routed_scale = routed_scale
         self.schedule = schedule
+        self.tiles = tuple(tiles)
         self._ws = None
 
     def desc(self, T: int, router_logits: Optional[torch.Tensor] = None,
@@ -299,7 +302,7 @@ class MoELayer:
                          router_w=w.get("router_w"), router_logits=router_logits, bias=w.get("bias"),
                          w13=w["w13"], w2=w["w2"], ws13=w.get("ws13"), ws2=w.get("ws2"),
                          routed_scale=self.routed_scale, shared_gate_w=w.get("shared_gate"), shared_out=shared_out,
-                         trace=trace, schedule=self.schedule)
+                         trace=trace, schedule=self.schedule, tiles=self.tiles)
 
     def workspace(self, desc: LayerDesc, device) -> torch.Tensor:
         need = workspace_size(desc)

@@ -57,6 +57,9 @@ def _fwd(d, x=FAKE * 6, out=FAKE * 7, ws=None, ws_bytes=0):
     ("path", 9, moe.MOE_ERR_INVALID_ARG),
     ("schedule", 3, moe.MOE_ERR_INVALID_ARG),
     ("schedule", -1, moe.MOE_ERR_INVALID_ARG),
+    ("fc1_tile_rows", 96, moe.MOE_ERR_INVALID_ARG),
+    ("fc1_tile_rows", 256, moe.MOE_ERR_INVALID_ARG),  # SwiGLU has no 256-row FC1 tile
+    ("fc2_tile_rows", 64, moe.MOE_ERR_INVALID_ARG),
     ("T", -1, moe.MOE_ERR_INVALID_ARG),
     ("T", 1 << 20, moe.MOE_ERR_UNSUPPORTED),
     ("I_shared", 12, moe.MOE_ERR_INVALID_ARG),
@@ -151,6 +154,15 @@ def test_token_tile_widths(act, T, K, E, tiles):
     """Token rows per grouped-GEMM tile follow the average rows per expert T*K/E."""
     d = _desc(T=T, top_k=K, E=E, act=act, I_shared=0)
     assert moe.token_tiles(d) == tiles
+
+
+def test_token_tile_widths_can_be_chosen():
+    d = _desc(T=4096, top_k=8, E=256, act="swiglu", I_shared=0)
+    d.fc1_tile_rows, d.fc2_tile_rows = 64, 256
+    assert moe.token_tiles(d) == (64, 256)
+    d.fc1_tile_rows = 0
+    assert moe.token_tiles(d) == (128, 256)
+    assert moe.workspace_size(d) > 0
 
 
 def test_workspace_regions_lie_inside_the_workspace():

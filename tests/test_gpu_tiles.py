@@ -81,3 +81,23 @@ def test_internal_permutation_full_shapes(shape, T):
     np.testing.assert_array_equal(moe.workspace_view(desc, layer._ws, moe.WS_TOPK_IDS).cpu().numpy().reshape(ids.shape),
                                   ids)
     check_internal_permutation(layer, desc, layer._ws, ids, shape.E)
+
+
+@pytest.mark.parametrize("shape,T,tiles", [(TILE_SW, 300, (64, 256)), (TILE_R2, 300, (256, 128)),
+                                           (TILE_SH, 150, (128, 32))])
+def test_caller_chosen_tile_widths_all_rows(shape, T, tiles):
+    """Token-tile widths forced by the caller (moe_layer_desc.fc1_tile_rows / fc2_tile_rows)
+    instead of the per-call choice: every row against the oracle."""
+    d = _util.device_layer(shape, T, seed=T + 5)
+    layer = moe.MoELayer(shape, _util.weights_of(d), path="large", tiles=tiles)
+    desc = layer.desc(T)
+    assert moe.token_tiles(desc) == tiles
+    out, tw, ti, lg = layer.forward(d["x"], return_routing=True)
+    torch.cuda.synchronize()
+    assert moe.get_error(layer._ws) == 0
+    h = _util.host_copy(d)
+    h["router_logits"] = None
+    ref_out, ref_lg, ref_w, ref_ids = oracle.forward(shape, h)
+    _util.check_fused_routing(ti.cpu().numpy(), tw.cpu().numpy(), lg.cpu().numpy(), ref_ids, ref_w, ref_lg, shape,
+                              h["bias"], False)
+    _util.assert_out_close(gen.bf16_bits(out), ref_out, f"{shape.name} T={T} forced tiles={tiles}")
