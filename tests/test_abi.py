@@ -5,6 +5,7 @@ import os
 import re
 
 import pytest
+import torch
 
 import mixture_experts_layer_35_b200.moe as moe
 from mixture_experts_layer_35_b200 import inputs as gen
@@ -230,3 +231,24 @@ def test_kernel_plan_lists_the_launches_in_order():
     for T in (1, 16, 64, 300, 4096):
         d = _desc(T=T, path="large")
         assert len(moe.kernel_plan(d)) == moe.launches(d)
+
+
+def test_trace_summary_on_a_synthetic_trace():
+    """The host summary of a phase trace (microseconds from %globaltimer nanoseconds):
+    launch skew, median input wait and load span, tail, kernel span and units per CTA;
+    rows of CTAs that did not run (zero entry stamp) are left out."""
+    t = torch.zeros(3 * moe.TRACE_MAX_CTAS * moe.TRACE_FIELDS, dtype=torch.int64)
+    v = t.view(3, moe.TRACE_MAX_CTAS, moe.TRACE_FIELDS)
+    # FC1 (block 1): three CTAs, entry / ready / loads done / stores done / exit / units
+    v[1, 0, :6] = torch.tensor([1000, 3000, 13000, 14000, 20000, 4])
+    v[1, 1, :6] = torch.tensor([2000, 3000, 15000, 16000, 22000, 5])
+    v[1, 2, :6] = torch.tensor([1000, 4000, 12000, 13000, 18000, 4])
+    s = moe.trace_summary(t, 4)
+    assert set(s) == {"fc1"}
+    f = s["fc1"]
+    assert f["ctas"] == 3
+    assert f["launch_skew_us"] == 1.0
+    assert f["input_wait_us_median"] == 2.0  # waits 2, 1, 3 us
+    assert f["load_span_us_median"] == 10.0  # spans 10, 12, 8 us
+    assert f["tail_us"] == 4.0 and f["kernel_us"] == 21.0
+    assert f["units_min_max"] == [4, 5]
